@@ -1,0 +1,342 @@
+"""Pins for the CPU oracle: closed forms, hand cases, brute force, invariants.
+
+None of these compares the oracle with itself: every expected value comes from
+the mathematics of the operator (special cases with a closed form, an explicit
+matrix-product formulation, the chunkwise WY/UT algebra, invariants) or from
+hand-derived fixtures in tests/golden/.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import kda_oracle as orc
+from gated_delta_rule_148_b200 import inputs as gen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def _one(seed, T, dk, dv, la_scale=1.0):
+    """Single-sequence single-head inputs with the standard distributions."""
+    c = gen.random_case(seed, [T], 1, dk, dv, "f32")
+    return (c["q"][:, 0], c["k"][:, 0], c["v"][:, 0], c["log_alpha"][:, 0] * la_scale,
+            c["beta"][:, 0])
+
+
+def _run1(q, k, v, la, beta, S0=None, mask=None):
+    """C oracle on one head / one sequence."""
+    T = q.shape[0]
+    o, fs = orc.prefill(q[:, None], k[:, None], v[:, None], la[:, None], beta[:, None],
+                        np.array([0, T], np.int32), pad_mask=mask,
+                        init_state=None if S0 is None else S0[None, None])
+    return o[:, 0], fs[0, 0]
+
+
+# ---------------------------------------------------------------- hand cases
+@pytest.mark.parametrize("case", json.load(open(GOLDEN))["cases"], ids=lambda c: c["name"])
+def test_hand_cases(case):
+    q, k, v = (np.array(case[x], np.float32) for x in ("q", "k", "v"))
+    la = np.log(np.array(case["alpha"], np.float64)).astype(np.float32)
+    beta = np.array(case["beta"], np.float32)
+    S0 = np.array(case["S0"], np.float32)
+    o, S = _run1(q, k, v, la, beta, S0)
+    np.testing.assert_allclose(o, case["o"], rtol=0, atol=1e-6)
+    np.testing.assert_allclose(S, case["S_final"], rtol=0, atol=1e-6)
+    o2, S2 = orc.brute_force(q, k, v, la, beta, S0)
+    np.testing.assert_allclose(o2, case["o"], rtol=0, atol=1e-6)
+    o3, S3 = orc.chunked(q, k, v, la, beta, 2, S0)
+    np.testing.assert_allclose(o3, case["o"], rtol=0, atol=1e-6)
+    np.testing.assert_allclose(S3, case["S_final"], rtol=0, atol=1e-6)
+
+
+# ---------------------------------------------------------------- closed forms
+def test_beta_zero_is_pure_per_channel_decay():
+    """beta = 0: S_T = Diag(exp(sum log_alpha)) S0 and o_t = (Diag(exp(cumsum)) S0)^T q_t."""
+    T, dk, dv = 37, 12, 9
+    q, k, v, la, _ = _one(1, T, dk, dv)
+    S0 = np.random.default_rng(2).normal(0, 1, (dk, dv)).astype(np.float32)
+    o, S = _run1(q, k, v, la, np.zeros(T, np.float32), S0)
+    G = np.cumsum(la.astype(np.float64), axis=0)
+    np.testing.assert_allclose(S, np.exp(G[-1])[:, None] * S0, rtol=1e-12, atol=1e-14)
+    o_ref = np.stack([(np.exp(G[t])[:, None] * S0).T @ q[t] for t in range(T)])
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-14)
+
+
+def test_unit_gate_zero_beta_keeps_state():
+    """alpha = 1, beta = 0: the state never changes and o_t = S0^T q_t."""
+    T, dk, dv = 20, 8, 16
+    q, k, v, _, _ = _one(3, T, dk, dv)
+    S0 = np.random.default_rng(4).normal(0, 1, (dk, dv)).astype(np.float32)
+    o, S = _run1(q, k, v, np.zeros((T, dk), np.float32), np.zeros(T, np.float32), S0)
+    np.testing.assert_array_equal(S, S0.astype(np.float64))
+    np.testing.assert_allclose(o, q.astype(np.float64) @ S0.astype(np.float64), rtol=1e-13)
+
+
+@pytest.mark.parametrize("dk,dv,T", [(16, 16, 16), (16, 8, 11), (8, 24, 8)])
+def test_orthonormal_keys_exact_retrieval(dk, dv, T):
+    """alpha = 1, beta = 1, orthonormal keys, S0 = 0: S_T^T k_j = v_j for every j."""
+    rng = np.random.default_rng(5)
+    Qm, _ = np.linalg.qr(rng.normal(size=(dk, dk)))
+    k = Qm[:T].astype(np.float32)            # rows orthonormal (to fp32 rounding)
+    v = rng.normal(size=(T, dv)).astype(np.float32)
+    q = rng.normal(size=(T, dk)).astype(np.float32)
+    _, S = _run1(q, k, v, np.zeros((T, dk), np.float32), np.ones(T, np.float32))
+    kd = k.astype(np.float64)
+    # the keys are orthonormal to ~1e-7 after fp32 rounding: exactness holds to that level
+    np.testing.assert_allclose(kd @ S, v, rtol=0, atol=1e-5)
+    # with keys re-orthonormalised in fp64 the retrieval is exact to rounding
+    kk, _ = np.linalg.qr(kd.T)
+    kk = kk.T[:T]
+    o, S2 = orc.brute_force(q, kk, v, np.zeros((T, dk)), np.ones(T))
+    np.testing.assert_allclose(kk @ S2, v, rtol=0, atol=1e-12)
+
+
+def test_delta_rule_overwrite():
+    """alpha = 1, beta = 1, one unit key written twice: reading it returns the second value."""
+    dk, dv = 6, 5
+    rng = np.random.default_rng(6)
+    key = rng.normal(size=dk)
+    key = (key / np.linalg.norm(key)).astype(np.float32)
+    v1 = rng.normal(size=dv).astype(np.float32)
+    v2 = rng.normal(size=dv).astype(np.float32)
+    k = np.stack([key, key])
+    q = np.stack([key, key])
+    o, S = _run1(q, k, np.stack([v1, v2]), np.zeros((2, dk), np.float32), np.ones(2, np.float32))
+    nk = float(key.astype(np.float64) @ key.astype(np.float64))   # 1 up to fp32 rounding
+    np.testing.assert_allclose(o[0], v1 * nk, rtol=1e-6)
+    np.testing.assert_allclose(o[1], v2 * nk, rtol=1e-6)
+    np.testing.assert_allclose(S.T @ key, v2 * nk, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- brute force
+@pytest.mark.parametrize("seed", range(6))
+def test_brute_force_tiny(seed):
+    """Explicit d_k x d_k transition products vs the C oracle on tiny inputs."""
+    rng = np.random.default_rng(100 + seed)
+    T = int(rng.integers(1, 9))
+    dk, dv = int(rng.integers(1, 5)), int(rng.integers(1, 5))
+    q, k, v = (rng.normal(size=(T, d)).astype(np.float32) for d in (dk, dk, dv))
+    la = -np.abs(rng.normal(size=(T, dk))).astype(np.float32)
+    beta = rng.uniform(-0.5, 1.5, size=T).astype(np.float32)
+    S0 = rng.normal(size=(dk, dv)).astype(np.float32)
+    mask = (rng.uniform(size=T) > 0.3).astype(np.uint8)
+    o, S = _run1(q, k, v, la, beta, S0, mask)
+    o2, S2 = orc.brute_force(q, k, v, la, beta, S0, mask)
+    np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S2, rtol=1e-12, atol=1e-12)
+    assert np.all(o[mask == 0] == 0.0)
+
+
+# ---------------------------------------------------------------- chunkwise algebra
+@pytest.mark.parametrize("chunk", [1, 2, 16, 64])
+@pytest.mark.parametrize("T,dk,dv", [(77, 16, 16), (150, 8, 24), (64, 24, 8)])
+def test_chunked_ut_equals_recurrence(chunk, T, dk, dv):
+    q, k, v, la, beta = _one(7, T, dk, dv)
+    S0 = np.random.default_rng(8).normal(0, 0.1, (dk, dv)).astype(np.float32)
+    o, S = _run1(q, k, v, la, beta, S0)
+    o2, S2 = orc.chunked(q, k, v, la, beta, chunk, S0)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-10 * max(1.0, np.abs(o).max()))
+    np.testing.assert_allclose(S2, S, rtol=0, atol=1e-10 * max(1.0, np.abs(S).max()))
+
+
+def test_chunked_handles_pads_as_identity_steps():
+    T, dk, dv = 90, 8, 8
+    q, k, v, la, beta = _one(9, T, dk, dv)
+    mask = np.ones(T, np.uint8)
+    mask[[0, 1, 40, 41, 42, 89]] = 0
+    S0 = np.random.default_rng(10).normal(0, 0.1, (dk, dv)).astype(np.float32)
+    o, S = _run1(q, k, v, la, beta, S0, mask)
+    o2, S2 = orc.chunked(q, k, v, la, beta, 16, S0, mask)
+    np.testing.assert_allclose(o2, o, atol=1e-11)
+    np.testing.assert_allclose(S2, S, atol=1e-11)
+
+
+# ---------------------------------------------------------------- carry / resume
+@pytest.mark.parametrize("split", [1, 31, 64, 99])
+def test_split_sequence_with_carried_state(split):
+    T, dk, dv = 128, 16, 12
+    q, k, v, la, beta = _one(11, T, dk, dv)
+    S0 = np.random.default_rng(12).normal(0, 0.1, (dk, dv)).astype(np.float32)
+    o, S = _run1(q, k, v, la, beta, S0)
+    oa, Sa = _run1(q[:split], k[:split], v[:split], la[:split], beta[:split], S0)
+    # carry the fp64 state exactly: continue with the brute force from Sa
+    ob, Sb = orc.brute_force(q[split:], k[split:], v[split:], la[split:], beta[split:], Sa)
+    np.testing.assert_allclose(np.concatenate([oa, ob]), o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(Sb, S, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_then_decode_continuation():
+    T, H, dk, dv = 40, 3, 8, 8
+    c = gen.random_case(13, [T + 1], H, dk, dv, "f32", init_state=True)
+    o, fs = orc.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], c["cu_seqlens"],
+                        init_state=c["init_state"])
+    o1, fs1 = orc.prefill(c["q"][:T], c["k"][:T], c["v"][:T], c["log_alpha"][:T],
+                          c["beta"][:T], np.array([0, T], np.int32), init_state=c["init_state"])
+    st = fs1.copy()
+    od = orc.decode(c["q"][T:], c["k"][T:], c["v"][T:], c["log_alpha"][T:], c["beta"][T:], st)
+    np.testing.assert_allclose(od[0], o[T], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st, fs, rtol=1e-12, atol=1e-13)
+
+
+def test_decode_mask_leaves_rows_untouched():
+    B, H, d = 6, 2, 8
+    c = gen.random_case(14, [1] * B, H, d, d, "f32", init_state=True)
+    st = c["init_state"].astype(np.float64)
+    before = st.copy()
+    mask = np.array([1, 0, 1, 0, 0, 1], np.uint8)
+    o = orc.decode(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], st, mask)
+    assert np.all(o[mask == 0] == 0.0)
+    np.testing.assert_array_equal(st[mask == 0], before[mask == 0])
+    assert np.all(np.abs(st[mask == 1] - before[mask == 1]).max(axis=(1, 2, 3)) > 0)
+    # active rows equal a one-token prefill per row
+    o2, fs2 = orc.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], c["cu_seqlens"],
+                          init_state=c["init_state"])
+    np.testing.assert_allclose(o[mask == 1], o2[mask == 1], rtol=1e-13)
+    np.testing.assert_allclose(st[mask == 1], fs2[mask == 1], rtol=1e-13)
+
+
+# ---------------------------------------------------------------- packing and padding
+def test_varlen_packing_equals_solo_runs():
+    lengths = [1, 15, 16, 17, 50]
+    H, dk, dv = 2, 8, 12
+    c = gen.random_case(15, lengths, H, dk, dv, "f32", init_state=True)
+    o, fs = orc.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], c["cu_seqlens"],
+                        init_state=c["init_state"])
+    cu = c["cu_seqlens"]
+    for b in range(len(lengths)):
+        sl = slice(cu[b], cu[b + 1])
+        for h in range(H):
+            ob, Sb = orc.brute_force(c["q"][sl, h], c["k"][sl, h], c["v"][sl, h],
+                                     c["log_alpha"][sl, h], c["beta"][sl, h],
+                                     c["init_state"][b, h])
+            np.testing.assert_allclose(o[sl, h], ob, rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(fs[b, h], Sb, rtol=1e-12, atol=1e-13)
+
+
+def _buggy_pads(q, k, v, la, beta, S0, mask):
+    """A planted mistake (test-only): pads zero q/k/v but keep their gates."""
+    q, k, v = q.copy(), k.copy(), v.copy()
+    q[mask == 0] = 0
+    k[mask == 0] = 0
+    v[mask == 0] = 0
+    return orc.brute_force(q, k, v, la, beta, S0)
+
+
+@pytest.mark.parametrize("side", ["left", "right", "interior"])
+def test_padding_equals_unpadded_run(side):
+    """Cached continuation (6 cached positions), 3 valid + 2 pads, then 1 probe position.
+
+    The shape follows the reproduction in "Transformers Community Reports Kimi
+    Linear Cache Bug" (ainews): the baseline is the UNPADDED run, not a padded one.
+    """
+    dk = dv = 8
+    q, k, v, la, beta = _one(16, 6 + 5 + 1, dk, dv)
+    # cached prefix
+    _, Sc = orc.brute_force(q[:6], k[:6], v[:6], la[:6], beta[:6])
+    Sc32 = Sc.astype(np.float32)
+    valid_idx = np.arange(6, 9)
+    # padded continuation: 5 positions, pads where requested, zero q/k/v but random gates
+    pad_pos = {"left": [0, 1], "right": [3, 4], "interior": [1, 3]}[side]
+    mask = np.ones(5, np.uint8)
+    mask[pad_pos] = 0
+    qp, kp, vp = (np.zeros((5, dk), np.float32) for _ in range(3))
+    slots = np.nonzero(mask)[0]
+    qp[slots], kp[slots], vp[slots] = q[valid_idx], k[valid_idx], v[valid_idx]
+    lap = -np.abs(np.random.default_rng(17).normal(size=(5, dk))).astype(np.float32)
+    lap[slots] = la[valid_idx]
+    bp = np.random.default_rng(18).uniform(0.2, 0.9, 5).astype(np.float32)
+    bp[slots] = beta[valid_idx]
+    o_pad, S_pad = _run1(qp, kp, vp, lap, bp, Sc32, mask)
+    o_ref, S_ref = _run1(q[valid_idx], k[valid_idx], v[valid_idx], la[valid_idx],
+                         beta[valid_idx], Sc32)
+    np.testing.assert_array_equal(o_pad[mask == 0], 0.0)
+    np.testing.assert_allclose(o_pad[slots], o_ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(S_pad, S_ref, rtol=1e-13, atol=1e-14)
+    # the probe position after the continuation sees the same state
+    probe = 11
+    p_pad, _ = _run1(q[probe:], k[probe:], v[probe:], la[probe:], beta[probe:],
+                     S_pad.astype(np.float32))
+    p_ref, _ = _run1(q[probe:], k[probe:], v[probe:], la[probe:], beta[probe:],
+                     S_ref.astype(np.float32))
+    np.testing.assert_array_equal(p_pad, p_ref)
+    # positive control: letting pads decay the state (the reported bug) is visible
+    ob, Sb = _buggy_pads(qp, kp, vp, lap, bp, Sc32, mask)
+    assert np.abs(Sb - S_ref).max() > 1e-3
+
+
+# ---------------------------------------------------------------- invariants
+def test_linearity_in_values_and_state():
+    """o(a V1 + b V2, a S1 + b S2) = a o(V1, S1) + b o(V2, S2) for fixed q, k, gates."""
+    T, dk, dv = 30, 8, 6
+    q, k, v1, la, beta = _one(19, T, dk, dv)
+    v1 = v1.astype(np.float64)
+    rng = np.random.default_rng(20)
+    v2 = rng.normal(size=v1.shape)
+    S1, S2 = rng.normal(size=(dk, dv)), rng.normal(size=(dk, dv))
+    a, b = 0.75, -1.5
+    o1, F1 = orc.brute_force(q, k, v1, la, beta, S1)
+    o2, F2 = orc.brute_force(q, k, v2, la, beta, S2)
+    vm = (a * v1 + b * v2)
+    Sm = (a * S1 + b * S2)
+    om, Fm = orc.brute_force(q, k, vm, la, beta, Sm)
+    np.testing.assert_allclose(om, a * o1 + b * o2, atol=1e-12)
+    np.testing.assert_allclose(Fm, a * F1 + b * F2, atol=1e-12)
+    # and the C oracle agrees on the mixed case (inputs exactly representable in fp32)
+    vm32, Sm32 = vm.astype(np.float32), Sm.astype(np.float32)   # representable inputs
+    oc, Fc = _run1(q, k, vm32, la, beta, Sm32)
+    ob, Fb = orc.brute_force(q, k, vm32, la, beta, Sm32)
+    np.testing.assert_allclose(oc, ob, atol=1e-12)
+
+
+def test_contraction_bound():
+    """||S_t||_F <= ||S_{t-1}||_F + |beta| ||k|| ||v|| for unit k, beta in [0,1], alpha <= 1."""
+    T, dk, dv = 50, 8, 8
+    q, k, v, la, beta = _one(21, T, dk, dv)
+    S = np.random.default_rng(22).normal(size=(dk, dv))
+    for t in range(T):
+        prev = np.linalg.norm(S)
+        _, S = orc.brute_force(q[t:t + 1], k[t:t + 1], v[t:t + 1], la[t:t + 1], beta[t:t + 1], S)
+        bound = prev + abs(beta[t]) * np.linalg.norm(k[t]) * np.linalg.norm(v[t])
+        assert np.linalg.norm(S) <= bound * (1 + 1e-12)
+
+
+# ---------------------------------------------------------------- prefix invariance
+def _leaky_chunked(q, k, v, la, beta, chunk):
+    """Planted leak (test-only): every chunk after the first reads the sequence's
+    FINAL state instead of its incoming state -- a reduction over the wrong chunk
+    axis, the defect class of "The Mask Is Not the Model" (dev.to)."""
+    _, S_final = orc.chunked(q, k, v, la, beta, chunk)
+    o_ok, _ = orc.chunked(q, k, v, la, beta, chunk)
+    T = q.shape[0]
+    o = o_ok.copy()
+    for c0 in range(chunk, T, chunk):
+        g = np.cumsum(la[c0:c0 + chunk].astype(np.float64), axis=0)
+        o[c0:c0 + chunk] += (q[c0:c0 + chunk] * np.exp(g)) @ S_final * 1e-3
+    return o, S_final
+
+
+@pytest.mark.parametrize("T", [16 * 3 + 1, 16 * 4 + 7])
+def test_prefix_invariance_with_positive_control(T):
+    """Perturbing position T-1 leaves o[0:T-1] unchanged; a planted leak is caught
+    with onset equal to the chunk size (audit length T exceeds 3 chunks)."""
+    C, dk, dv = 16, 8, 8
+    q, k, v, la, beta = _one(23, T, dk, dv)
+    rng = np.random.default_rng(24)
+
+    def variant(which, fn):
+        qq, kk, vv, ll, bb = q.copy(), k.copy(), v.copy(), la.copy(), beta.copy()
+        if which:
+            qq[T - 1] = rng.normal(size=dk)
+            kk[T - 1] = rng.normal(size=dk)
+            vv[T - 1] = rng.normal(size=dv)
+            ll[T - 1] = -np.abs(rng.normal(size=dk))
+            bb[T - 1] = 0.123
+        return fn(qq, kk, vv, ll, bb)
+
+    for fn in (lambda *a: _run1(*a)[0], lambda *a: orc.chunked(*a, C)[0]):
+        leak, onset, d = orc.prefix_audit(lambda w: variant(w, fn), T, 1)
+        assert not leak and d.max() == 0.0
+    leak, onset, _ = orc.prefix_audit(lambda w: variant(w, lambda *a: _leaky_chunked(*a, C)[0]),
+                                      T, 1)
+    assert leak and onset == C
