@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA operator on B200 (prints one JSON line on rank 0).
+
+Headline workload (one "step"): one kda_prefill over B=1, H=32, T=131072,
+d_k=d_v=128, bf16 q/k/v, fp32 gates and state, chunk 64 -- the long-context
+prefill.  Inputs are resident in HBM before timing and are larger than L2
+(6.4 GB), so no flush is needed between steps.  The same run also measures:
+  * "decode": the batched decode step (256 rows x 32 heads x 128 x 128 fp32
+    state, 26 masked rows per step);
+  * "prefill_sweep": prefill at T = 4096, 16384, 65536 (L2 flushed between
+    iterations);
+  * "e2e": the headline metric through the public API with pinned HOST
+    buffers, host<->device copies inside the timed region;
+  * "cpu_baseline": the fp64 CPU oracle on a bounded sample of the workload.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs the same workload
+on its own GPU with no collective on the data path (the operator shards by
+sequence and head: replicas, weak scaling); the timed region is bracketed by
+barriers and the max time over ranks is reported.
+
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA tokens/s (prefill 4k–128k, batched decode) and % of roofline on 1 B200"
+PREFILL_BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 + log_alpha fp32 + beta + o bf16
+STATE_BYTES = 128 * 128 * 4                  # one (sequence, head) fp32 state
+DECODE_ACTIVE_BYTES = 2 * STATE_BYTES + 768 + 512 + 4 + 256
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--T", type=int, default=131072)
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--no-extras", action="store_true", help="headline prefill line only")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"],
+                    source="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_148_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) of SM clock and throttle reasons during a region."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or parts[0] != self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- helpers
+def to_dev(x, dtype, device, pin=True):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if dtype is not None:
+        t = t.to(dtype)
+    if pin:
+        t = t.pin_memory()
+    return t, t.to(device, non_blocking=False)
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def prefill_setup(T, device):
+    import torch
+    from gated_delta_rule_148_b200 import inputs as gen
+    w = gen.long_prefill(T)
+    inp = gen.prefill_inputs(w)
+    host, dev = {}, {}
+    for key, dt in (("q", torch.bfloat16), ("k", torch.bfloat16), ("v", torch.bfloat16),
+                    ("log_alpha", None), ("beta", None), ("cu_seqlens", None)):
+        host[key], dev[key] = to_dev(inp[key], dt, device)
+    N, H = inp["q"].shape[0], inp["q"].shape[1]
+    dev["o"] = torch.empty((N, H, 128), dtype=torch.bfloat16, device=device)
+    dev["fs"] = torch.empty((1, H, 128, 128), dtype=torch.float32, device=device)
+    return w, inp, host, dev
+
+
+def run_prefill(kda, dev):
+    kda.prefill(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], dev["cu_seqlens"],
+                o=dev["o"], final_state=dev["fs"])
+
+
+def prefill_bytes(T, H):
+    return T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+
+
+def time_loop(fn, K, W, flush_buf=None):
+    """K timed calls after W warm-ups; returns per-call ms (events on the current stream)."""
+    import torch
+    for _ in range(W):
+        fn()
+    torch.cuda.synchronize()
+    if flush_buf is None:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(K):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / K
+    tot = 0.0
+    for _ in range(K):
+        flush_l2(flush_buf)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        tot += s.elapsed_time(e)
+    return tot / K
+
+
+def cpu_baseline(inp, budget_s=10.0):
+    """The fp64 oracle on the first T_s tokens (all heads) of the workload."""
+    from oracle import kda_oracle as orc
+    H = inp["q"].shape[1]
+
+    def run(Ts):
+        cu = np.array([0, Ts], np.int32)
+        t0 = time.perf_counter()
+        orc.prefill(inp["q"][:Ts], inp["k"][:Ts], inp["v"][:Ts], inp["log_alpha"][:Ts],
+                    inp["beta"][:Ts], cu)
+        return time.perf_counter() - t0
+    probe = 512
+    dt = run(probe)
+    Ts = int(min(inp["q"].shape[0], max(probe, probe * budget_s / max(dt, 1e-3))))
+    Ts = max(probe, (Ts // 512) * 512)
+    dt = run(Ts)
+    return {"value": Ts / dt, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"first {Ts} of {inp['q'].shape[0]} tokens, all {H} heads, fp64 "
+                      f"token-by-token C oracle, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- reference arm
+def main_reference(args, rank, world):
+    if rank != 0:
+        return
+    from gated_delta_rule_148_b200 import inputs as gen
+    from oracle import kda_oracle as orc
+    w = gen.long_prefill(args.T)
+    # a bounded sample of the workload per step: its first Ts tokens, all heads
+    Ts_max = 8192
+    inp = gen.prefill_inputs(gen.long_prefill(Ts_max))   # same seed: a prefix of the workload
+    H = inp["q"].shape[1]
+    per_step_budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    t0 = time.perf_counter()
+    orc.prefill(inp["q"][:512], inp["k"][:512], inp["v"][:512], inp["log_alpha"][:512],
+                inp["beta"][:512], np.array([0, 512], np.int32))
+    dt = time.perf_counter() - t0
+    Ts = int(min(Ts_max, max(512, 512 * per_step_budget / max(dt, 1e-3))))
+    Ts = max(512, (Ts // 512) * 512)
+    cu = np.array([0, Ts], np.int32)
+
+    def step():
+        orc.prefill(inp["q"][:Ts], inp["k"][:Ts], inp["v"][:Ts], inp["log_alpha"][:Ts],
+                    inp["beta"][:Ts], cu)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = Ts * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": 1, "seq_len": args.T, "heads": 32,
+                   "d_k": 128, "d_v": 128, "parallelism": "replicas" if args.gpus > 1 else "none",
+                   "l2": "inputs larger than L2"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: first {Ts} of {args.T} tokens, all {H} heads"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def main_ours(args, rank, world, device):
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_148_b200 import kda
+    from gated_delta_rule_148_b200 import inputs as gen
+
+    kda.load()
+    pk = peaks()
+    props = torch.cuda.get_device_properties(device)
+    clocks = ClockSampler("GPU-" + str(props.uuid))
+
+    T = args.T
+    w, inp, host, dev = prefill_setup(T, device)
+    H = 32
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        run_prefill(kda, dev)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        run_prefill(kda, dev)
+    e.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st = kda.get_device_status()
+    if st != kda.KDA_OK:
+        raise RuntimeError("device status after prefill: " + kda.status_string(st))
+    ms_step = ms / K
+    value = T * world / (ms_step / 1e3)
+    algo_bytes = prefill_bytes(T, H)
+    achieved = algo_bytes / (ms_step / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic("prefill"),
+                "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
+                "kernel": "kda prefill (whole kda_prefill call: pre-pass + main kernel)",
+                "algorithmic_bytes_per_launch": algo_bytes,
+                "flops_bound_frac": (141013.0 * T * H / (ms_step / 1e3) / 1e12) / pk["bf16_tflops"]}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": 1, "seq_len": T, "heads": H,
+                       "d_k": 128, "d_v": 128, "chunk": 64, "state": "fp32",
+                       "parallelism": f"replicas{world}" if world > 1 else "none",
+                       "l2": "inputs larger than L2 (6.4 GB per step), no flush"},
+            "roofline": roofline, "clocks": clk, "gpu_launches": 2 * K}
+
+    # ---- e2e through the public API with host buffers
+    Ke = max(1, min(K, 3))
+    o_host = torch.empty(dev["o"].shape, dtype=dev["o"].dtype).pin_memory()
+    fs_host = torch.empty(dev["fs"].shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for key in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens"):
+            dev[key].copy_(host[key], non_blocking=True)
+        run_prefill(kda, dev)
+        o_host.copy_(dev["o"], non_blocking=True)
+        fs_host.copy_(dev["fs"], non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(Ke):
+        e2e_step()
+    e2.record()
+    torch.cuda.synchronize()
+    ms2 = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([ms2], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms2 = float(t.item())
+    h2d = sum(host[k].numel() * host[k].element_size()
+              for k in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens"))
+    d2h = o_host.numel() * o_host.element_size() + fs_host.numel() * 4
+    line["e2e"] = {"value": T * world / (ms2 / Ke / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
+    line["gpu_launches"] += 2 * Ke
+    del o_host, fs_host
+
+    if not args.no_extras:
+        # ---- batched decode
+        wd = gen.batched_decode()
+        state = torch.from_numpy(gen.decode_state(wd)).to(device)
+        pool = []
+        for t in gen.decode_pool(wd):
+            pool.append({k: torch.from_numpy(t[k]).to(device).to(torch.bfloat16)
+                         if k in ("q", "k", "v") else torch.from_numpy(t[k]).to(device)
+                         for k in ("q", "k", "v", "log_alpha", "beta")})
+        Dsteps = args.decode_steps
+        masks = torch.from_numpy(np.stack([gen.decode_mask(wd, i) for i in range(Dsteps + W)])
+                                 ).to(device)
+        o_dec = torch.empty((wd.decode_rows, wd.H, wd.dv), dtype=torch.bfloat16, device=device)
+        it = [0]
+
+        def dstep():
+            i = it[0]
+            d = pool[i % len(pool)]
+            kda.decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state, mask=masks[i],
+                       o=o_dec)
+            it[0] += 1
+        dms = time_loop(dstep, Dsteps, W)
+        if world > 1:
+            t = torch.tensor([dms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            dms = float(t.item())
+        active = wd.decode_rows - wd.decode_masked
+        dbytes = (active * wd.H * DECODE_ACTIVE_BYTES + wd.decode_masked * wd.H * 256
+                  + wd.decode_rows)
+        dach = dbytes / (dms / 1e3) / 1e9
+        line["decode"] = {
+            "workload": wd.name, "value": active * world / (dms / 1e3), "unit": "tokens/s",
+            "us_per_step": dms * 1e3, "steps": Dsteps,
+            "roofline": {"bound": "hbm", "achieved": dach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": dach / pk["hbm_gbs"], "traffic": recorded_traffic("decode"),
+                         "algorithmic_bytes_per_launch": dbytes}}
+        line["gpu_launches"] += Dsteps
+        del state, pool, masks, o_dec
+
+        # ---- prefill sweep (smaller T; L2 flushed between iterations)
+        sweep = {}
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        for Ts in (4096, 16384, 65536):
+            if Ts >= T:
+                continue
+            _, _, _, dv_ = prefill_setup(Ts, device)
+            mss = time_loop(lambda: run_prefill(kda, dv_), max(3, K), W,
+                            flush_buf=flush if Ts <= 16384 else None)
+            ach = prefill_bytes(Ts, H) / (mss / 1e3) / 1e9
+            sweep[str(Ts)] = {"tokens_per_s": Ts / (mss / 1e3), "ms": mss,
+                              "hbm_frac": ach / pk["hbm_gbs"],
+                              "l2": "flushed" if Ts <= 16384 else "inputs larger than L2"}
+            line["gpu_launches"] += 2 * (max(3, K))
+            del dv_
+        sweep[str(T)] = {"tokens_per_s": T / (ms_step / 1e3), "ms": ms_step,
+                         "hbm_frac": roofline["frac"], "l2": "inputs larger than L2"}
+        line["prefill_sweep"] = sweep
+        del flush
+
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        main_reference(args, rank, world)
+        return
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    try:
+        main_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+// C ABI of libkda.so: argument validation, dispatch, device error word.
+//
+// Every entry point validates on the host first and launches nothing on an
+// argument error.  See include/kda.h for the contract of each call.
+#include <cstring>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+
+// Per-device error word (bits of ERR_BIT_*); kernels OR into it.
+__device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned *g_err_ptr[kMaxDevices];   // cached device address, per device
+
+kda_status error_word(unsigned **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+  if (g_err_ptr[dev] == nullptr) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return KDA_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<unsigned *>(ptr);
+  }
+  *out = g_err_ptr[dev];
+  return KDA_OK;
+}
+
+struct Range {
+  const void *p;
+  size_t bytes;
+};
+
+bool overlap(Range a, Range b) {
+  if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+  const uintptr_t a0 = (uintptr_t)a.p, a1 = a0 + a.bytes;
+  const uintptr_t b0 = (uintptr_t)b.p, b1 = b0 + b.bytes;
+  return a0 < b1 && b0 < a1;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+size_t elem_bytes(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
+
+size_t spans_bytes(int num_seqs) {
+  const size_t raw = sizeof(SeqSpan) * (size_t)(num_seqs > 0 ? num_seqs : 0);
+  return (raw + 255) / 256 * 256;
+}
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+int kda_version(void) { return (1 << 16) | 0; }
+
+const char *kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: configuration not supported";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call failed";
+    case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+    case KDA_ERR_DEVICE_CHECK: return "KDA_ERR_DEVICE_CHECK: a device-side argument check failed";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+size_t kda_prefill_workspace_size(const kda_prefill_args *a) {
+  if (!a) return 0;
+  return spans_bytes(a->num_seqs);
+}
+
+kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->dtype != KDA_F32 && a->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (a->num_seqs < 0 || a->total_tokens < 0 || a->H < 1) return KDA_ERR_INVALID_ARG;
+  if (a->dk <= 0 || a->dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (!head_dim_ok(a->dk) || !head_dim_ok(a->dv)) return KDA_ERR_UNSUPPORTED;
+  int chunk = a->chunk;
+  if (chunk == 0) chunk = (a->dtype == KDA_BF16) ? 64 : 16;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if (a->num_seqs == 0) return a->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+  if (!a->cu_seqlens) return KDA_ERR_INVALID_ARG;
+  const size_t N = (size_t)a->total_tokens, H = (size_t)a->H;
+  const size_t es = elem_bytes(a->dtype);
+  const Range q{a->q, N * H * a->dk * es}, k{a->k, N * H * a->dk * es};
+  const Range v{a->v, N * H * a->dv * es}, la{a->log_alpha, N * H * a->dk * 4};
+  const Range be{a->beta, N * H * 4}, cu{a->cu_seqlens, 4 * ((size_t)a->num_seqs + 1)};
+  const Range mk{a->pad_mask, a->pad_mask ? N : 0};
+  const size_t sbytes = (size_t)a->num_seqs * H * a->dk * a->dv * 4;
+  const Range s0{a->init_state, a->init_state ? sbytes : 0};
+  const Range s1{a->final_state, a->final_state ? sbytes : 0};
+  const Range o{a->o, N * H * a->dv * es};
+  const Range ws{a->workspace, a->workspace ? a->workspace_bytes : 0};
+  if (N > 0 && (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->o))
+    return KDA_ERR_INVALID_ARG;
+  const void *need16[] = {a->q, a->k, a->v, (const void *)a->log_alpha, a->o,
+                          (const void *)a->init_state, (const void *)a->final_state};
+  for (const void *p : need16)
+    if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+  if (!aligned(a->beta, 4) || !aligned(a->cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+  if (a->pad_mask) {
+    if (!a->workspace || a->workspace_bytes < kda_prefill_workspace_size(a)) return KDA_ERR_INVALID_ARG;
+    if (!aligned(a->workspace, 256)) return KDA_ERR_INVALID_ARG;
+  }
+  // o and final_state must not overlap any input; init/final may coincide exactly
+  const Range inputs[] = {q, k, v, la, be, cu, mk, s0, ws};
+  for (const Range &r : inputs) {
+    if (overlap(o, r)) return KDA_ERR_INVALID_ARG;
+    if (overlap(s1, r) && !(r.p == s0.p && s1.p == s0.p)) return KDA_ERR_INVALID_ARG;
+  }
+  if (overlap(o, s1)) return KDA_ERR_INVALID_ARG;
+  if (overlap(ws, q) || overlap(ws, k) || overlap(ws, v) || overlap(ws, la) || overlap(ws, be) ||
+      overlap(ws, cu) || overlap(ws, mk) || overlap(ws, s0))
+    return KDA_ERR_INVALID_ARG;
+
+  unsigned *err = nullptr;
+  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  PrefillParams p;
+  p.num_seqs = a->num_seqs;
+  p.N = a->total_tokens;
+  p.H = a->H;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.chunk = chunk;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.log_alpha = a->log_alpha;
+  p.beta = a->beta;
+  p.cu = a->cu_seqlens;
+  p.mask = a->pad_mask;
+  p.init_state = a->init_state;
+  p.o = a->o;
+  p.final_state = a->final_state;
+  p.err = err;
+  SeqSpan *spans = a->pad_mask ? static_cast<SeqSpan *>(a->workspace) : nullptr;
+  p.spans = nullptr;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = a->dtype == KDA_BF16;
+  if (launch_prefill_prepass(p, bf16, spans, s) != cudaSuccess) return KDA_ERR_CUDA;
+  p.spans = spans;
+  cudaError_t e = prefill_tc_supported(p, bf16) ? launch_prefill_tc(p, s)
+                                                : launch_prefill_simt(p, bf16, s);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode(const kda_decode_args *a, void *stream) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->dtype != KDA_F32 && a->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (!head_dim_ok(a->dk) || !head_dim_ok(a->dv)) return KDA_ERR_UNSUPPORTED;
+  if (a->B == 0) return KDA_OK;
+  if (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->state || !a->o)
+    return KDA_ERR_INVALID_ARG;
+  const size_t B = (size_t)a->B, H = (size_t)a->H, es = elem_bytes(a->dtype);
+  const Range q{a->q, B * H * a->dk * es}, k{a->k, B * H * a->dk * es};
+  const Range v{a->v, B * H * a->dv * es}, la{a->log_alpha, B * H * a->dk * 4};
+  const Range be{a->beta, B * H * 4}, mk{a->mask, a->mask ? B : 0};
+  const Range st{a->state, B * H * a->dk * a->dv * 4}, o{a->o, B * H * a->dv * es};
+  if (!aligned(a->state, 16) || !aligned(a->beta, 4) || !aligned(a->log_alpha, 4))
+    return KDA_ERR_INVALID_ARG;
+  if (!aligned(a->q, es) || !aligned(a->k, es) || !aligned(a->v, es) || !aligned(a->o, es))
+    return KDA_ERR_INVALID_ARG;
+  const Range others[] = {q, k, v, la, be, mk};
+  for (const Range &r : others)
+    if (overlap(o, r) || overlap(st, r)) return KDA_ERR_INVALID_ARG;
+  if (overlap(o, st)) return KDA_ERR_INVALID_ARG;
+  unsigned *err = nullptr;
+  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  DecodeParams p;
+  p.B = a->B;
+  p.H = a->H;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.log_alpha = a->log_alpha;
+  p.beta = a->beta;
+  p.mask = a->mask;
+  p.state = a->state;
+  p.o = a->o;
+  p.err = err;
+  return launch_decode(p, a->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_get_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
+  unsigned *err = nullptr;
+  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+  if (word == 0) return KDA_OK;
+  const unsigned zero = 0;
+  if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+  if (word & ERR_BIT_TIMEOUT) return KDA_ERR_DEVICE_TIMEOUT;
+  return KDA_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// Internal declarations shared by the translation units of libkda.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Bits latched in the per-device error word.
+enum : unsigned {
+  ERR_BIT_CHECK = 1u,     // device-side argument check failed
+  ERR_BIT_TIMEOUT = 2u,   // a bounded wait ran out
+};
+
+// Per-sequence span of positions a prefill kernel processes: [begin, end)
+// in packed rows.  Rows of the sequence outside the span are edge pads.
+struct SeqSpan {
+  int begin;
+  int end;
+  int seq_begin;   // cu[b]
+  int pad_inside;  // 1 if a pad sits strictly inside [begin, end)
+};
+
+struct PrefillParams {
+  int num_seqs, N, H, dk, dv, chunk;
+  const void *q, *k, *v;
+  const float *log_alpha, *beta;
+  const int32_t *cu;
+  const uint8_t *mask;
+  const float *init_state;
+  void *o;
+  float *final_state;
+  const SeqSpan *spans;   // NULL: spans are [cu[b], cu[b+1])
+  unsigned *err;          // device error word
+};
+
+struct DecodeParams {
+  int B, H, dk, dv;
+  const void *q, *k, *v;
+  const float *log_alpha, *beta;
+  const uint8_t *mask;
+  float *state;
+  void *o;
+  unsigned *err;
+};
+
+// Launchers (return a CUDA error code; argument checks happen before).
+cudaError_t launch_prefill_prepass(const PrefillParams &p, bool bf16, SeqSpan *spans,
+                                   cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, cudaStream_t s);
+cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t s);
+bool prefill_tc_supported(const PrefillParams &p, bool bf16);
+cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+  return __uint_as_float(((unsigned)h) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  // round to nearest even; inputs here are finite
+  unsigned u = __float_as_uint(f);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+template <bool BF16>
+__device__ __forceinline__ float load_elem(const void *base, size_t idx) {
+  if (BF16) return bf16_to_f32(reinterpret_cast<const uint16_t *>(base)[idx]);
+  return reinterpret_cast<const float *>(base)[idx];
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_elem(void *base, size_t idx, float val) {
+  if (BF16) reinterpret_cast<uint16_t *>(base)[idx] = f32_to_bf16_rne(val);
+  else reinterpret_cast<float *>(base)[idx] = val;
+}
+
+__device__ __forceinline__ bool device_error_latched(const unsigned *err) {
+  return *reinterpret_cast<const volatile unsigned *>(err) != 0u;
+}
+
+}  // namespace kda

@@ -14,13 +14,17 @@ q, k and v are rounded to bf16 (round to nearest even) for bf16 workloads; the
 arrays returned here always hold float32 values, which represent bf16 values
 exactly, so the CPU side can read them without a conversion step.
 
-Random streams: one numpy PCG64 SeedSequence per workload; each tensor is
-drawn from its own spawned child stream (q, k, v, log_alpha, beta, state,
-structure), so that generating one tensor never shifts another.
+Random streams: numpy PCG64.  Each tensor has its own stream id (q, k, v,
+log_alpha, beta, state, structure), and its flattened elements are drawn in
+blocks of 2**22, block i from SeedSequence([seed, stream, sub, i]); so the
+values do not depend on how many threads fill the blocks, and generating one
+tensor never shifts another.
 """
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, List, Optional, Sequence
 
 import numpy as np
@@ -85,35 +89,76 @@ def _child(seed: int, stream: str, sub: int = 0) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(ss))
 
 
+_BLOCK = 1 << 22
+_WORKERS = max(1, min(16, os.cpu_count() or 1))
+
+
+def _blocks(n: int):
+    return [(i, i * _BLOCK, min(n, (i + 1) * _BLOCK)) for i in range((n + _BLOCK - 1) // _BLOCK)]
+
+
+def _par(fn, items):
+    if len(items) <= 1:
+        return [fn(it) for it in items]
+    with ThreadPoolExecutor(_WORKERS) as ex:
+        return list(ex.map(fn, items))
+
+
+def _rows_map(fn, x: np.ndarray) -> np.ndarray:
+    """Apply ``fn`` to blocks of leading rows of x in parallel (fn is row-local)."""
+    lead = x.shape[0]
+    per = max(1, _BLOCK // max(1, x[0].size))
+    spans = [(a, min(lead, a + per)) for a in range(0, lead, per)]
+
+    def one(sp):
+        x[sp[0]:sp[1]] = fn(x[sp[0]:sp[1]])
+    _par(one, spans)
+    return x
+
+
 def round_bf16(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    """Round float32 values to the nearest bf16 (ties to even); returns float32.
+
+    Finite inputs only (the uint32 sum cannot overflow below the NaN range)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+
+    def rnd(blk):
+        u = blk.view(np.uint32)
+        u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+        return u.view(np.float32)
+    return _rows_map(rnd, x.copy()) if x.ndim else rnd(x.reshape(1)).reshape(())
 
 
 def _normal(seed: int, stream: str, shape, scale: float = 1.0, loc: float = 0.0) -> np.ndarray:
-    rng = _child(seed, stream)
-    out = rng.standard_normal(size=shape, dtype=np.float32)
-    if scale != 1.0:
-        out *= np.float32(scale)
-    if loc != 0.0:
-        out += np.float32(loc)
-    return out
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    sid = _STREAMS.index(stream)
+
+    def fill(blk):
+        i, a, b = blk
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, sid, 0, i])))
+        g.standard_normal(out=out[a:b], dtype=np.float32)
+        if scale != 1.0:
+            out[a:b] *= np.float32(scale)
+        if loc != 0.0:
+            out[a:b] += np.float32(loc)
+    _par(fill, _blocks(n))
+    return out.reshape(shape)
 
 
 def _unit_rows(x: np.ndarray) -> np.ndarray:
-    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True, dtype=np.float32), dtype=np.float32)
-    return (x / np.maximum(n, np.float32(1e-30))).astype(np.float32)
+    def f(blk):
+        n = np.sqrt(np.sum(blk * blk, axis=-1, keepdims=True, dtype=np.float32), dtype=np.float32)
+        return (blk / np.maximum(n, np.float32(1e-30))).astype(np.float32)
+    return _rows_map(f, x)
 
 
 def _softplus(x: np.ndarray) -> np.ndarray:
-    return np.logaddexp(np.float32(0.0), x).astype(np.float32)
+    return _rows_map(lambda b: np.logaddexp(np.float32(0.0), b).astype(np.float32), x)
 
 
 def _sigmoid(x: np.ndarray) -> np.ndarray:
-    return (1.0 / (1.0 + np.exp(-x))).astype(np.float32)
+    return _rows_map(lambda b: (1.0 / (1.0 + np.exp(-b))).astype(np.float32), x)
 
 
 def token_tensors(seed: int, N: int, H: int, dk: int, dv: int, dtype: str) -> Dict[str, np.ndarray]:
@@ -123,7 +168,8 @@ def token_tensors(seed: int, N: int, H: int, dk: int, dv: int, dtype: str) -> Di
     v = _normal(seed, "v", (N, H, dv))
     if dtype == "bf16":
         q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
-    log_alpha = -_softplus(_normal(seed, "log_alpha", (N, H, dk), loc=-2.0))
+    log_alpha = _softplus(_normal(seed, "log_alpha", (N, H, dk), loc=-2.0))
+    np.negative(log_alpha, out=log_alpha)
     beta = _sigmoid(_normal(seed, "beta", (N, H)))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)
 

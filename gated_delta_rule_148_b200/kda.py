@@ -1,0 +1,228 @@
+"""Python binding of libkda.so (argument marshalling only).
+
+Every step of the operator runs in the CUDA library; this module only checks
+that the tensors are CUDA tensors of the right dtype and shape, fills the C
+argument structs declared in include/kda.h and calls them on the current
+torch stream.  There is no CPU path: without the CUDA library, a GPU, or with
+host tensors, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+_lib = None
+_lock = threading.Lock()
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_CUDA = 3
+KDA_ERR_DEVICE_TIMEOUT = 4
+KDA_ERR_DEVICE_CHECK = 5
+KDA_F32 = 0
+KDA_BF16 = 1
+
+EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
+            "kda_status_string", "kda_version")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class PrefillArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("num_seqs", ctypes.c_int),
+                ("total_tokens", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("log_alpha", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
+                ("pad_mask", ctypes.c_void_p), ("init_state", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("final_state", ctypes.c_void_p),
+                ("chunk", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("q", ctypes.c_void_p),
+                ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("log_alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("mask", ctypes.c_void_p), ("state", ctypes.c_void_p), ("o", ctypes.c_void_p)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load(build_if_stale: bool = True) -> ctypes.CDLL:
+    """Load libkda.so (compiling it with nvcc first if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_stale:
+                from . import build as _build
+                _build.build()
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"libkda.so not found at {_LIB_PATH}; build it first")
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.kda_prefill.argtypes = [ctypes.POINTER(PrefillArgs), ctypes.c_void_p]
+            lib.kda_prefill.restype = ctypes.c_int
+            lib.kda_prefill_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs)]
+            lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
+            lib.kda_decode.argtypes = [ctypes.POINTER(DecodeArgs), ctypes.c_void_p]
+            lib.kda_decode.restype = ctypes.c_int
+            lib.kda_get_device_status.argtypes = [ctypes.c_void_p]
+            lib.kda_get_device_status.restype = ctypes.c_int
+            lib.kda_status_string.argtypes = [ctypes.c_int]
+            lib.kda_status_string.restype = ctypes.c_char_p
+            lib.kda_version.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_cuda(name: str, t: Optional[torch.Tensor], dtype=None, shape=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the operator has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def prefill_args(q, k, v, log_alpha, beta, cu_seqlens, pad_mask=None, init_state=None,
+                 o=None, final_state=None, chunk: int = 0, workspace=None) -> PrefillArgs:
+    """Fill a kda_prefill_args struct from tensors (no validation beyond shapes)."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    a = PrefillArgs()
+    a.dtype = _dtype_code(q)
+    a.num_seqs = cu_seqlens.numel() - 1
+    a.total_tokens = N
+    a.H, a.dk, a.dv = H, dk, dv
+    a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
+    a.log_alpha, a.beta, a.cu_seqlens = _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens)
+    a.pad_mask, a.init_state = _ptr(pad_mask), _ptr(init_state)
+    a.o, a.final_state = _ptr(o), _ptr(final_state)
+    a.chunk = int(chunk)
+    a.workspace = _ptr(workspace)
+    a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return a
+
+
+def prefill_workspace_bytes(num_seqs: int) -> int:
+    a = PrefillArgs()
+    a.num_seqs = int(num_seqs)
+    return int(load().kda_prefill_workspace_size(ctypes.byref(a)))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+            beta: torch.Tensor, cu_seqlens: torch.Tensor, pad_mask: Optional[torch.Tensor] = None,
+            init_state: Optional[torch.Tensor] = None, o: Optional[torch.Tensor] = None,
+            final_state: Optional[torch.Tensor] = None, chunk: int = 0,
+            workspace: Optional[torch.Tensor] = None, want_final_state: bool = True,
+            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """KDA chunkwise prefill (kda_prefill).  Returns (o, final_state).
+
+    q, k [N,H,dk] and v [N,H,dv] bf16 or fp32; log_alpha [N,H,dk] fp32; beta [N,H] fp32;
+    cu_seqlens [B+1] int32; pad_mask [N] uint8 or None; init_state [B,H,dk,dv] fp32 or None.
+    Outputs are allocated here when not given (torch allocates; the library does not).
+    """
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    B = cu_seqlens.numel() - 1
+    _check_cuda("q", q, shape=(N, H, dk))
+    _check_cuda("k", k, dtype=q.dtype, shape=(N, H, dk))
+    _check_cuda("v", v, dtype=q.dtype, shape=(N, H, dv))
+    _check_cuda("log_alpha", log_alpha, torch.float32, (N, H, dk))
+    _check_cuda("beta", beta, torch.float32, (N, H))
+    _check_cuda("cu_seqlens", cu_seqlens, torch.int32, (B + 1,))
+    _check_cuda("pad_mask", pad_mask, torch.uint8, (N,))
+    _check_cuda("init_state", init_state, torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _check_cuda("o", o, q.dtype, (N, H, dv))
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_cuda("final_state", final_state, torch.float32, (B, H, dk, dv))
+    if pad_mask is not None and workspace is None:
+        workspace = torch.empty(prefill_workspace_bytes(B), dtype=torch.uint8, device=q.device)
+    a = prefill_args(q, k, v, log_alpha, beta, cu_seqlens, pad_mask, init_state, o, final_state,
+                     chunk, workspace)
+    st = lib.kda_prefill(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill")
+    return o, final_state
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+           beta: torch.Tensor, state: torch.Tensor, mask: Optional[torch.Tensor] = None,
+           o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One KDA decode step (kda_decode); ``state`` [B,H,dk,dv] fp32 is updated in place."""
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    _check_cuda("q", q, shape=(B, H, dk))
+    _check_cuda("k", k, q.dtype, (B, H, dk))
+    _check_cuda("v", v, q.dtype, (B, H, dv))
+    _check_cuda("log_alpha", log_alpha, torch.float32, (B, H, dk))
+    _check_cuda("beta", beta, torch.float32, (B, H))
+    _check_cuda("mask", mask, torch.uint8, (B,))
+    _check_cuda("state", state, torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check_cuda("o", o, q.dtype, (B, H, dv))
+    a = DecodeArgs()
+    a.dtype = _dtype_code(q)
+    a.B, a.H, a.dk, a.dv = B, H, dk, dv
+    a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
+    a.log_alpha, a.beta, a.mask = _ptr(log_alpha), _ptr(beta), _ptr(mask)
+    a.state, a.o = _ptr(state), _ptr(o)
+    st = lib.kda_decode(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode")
+    return o
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the latched device status."""
+    return int(load().kda_get_device_status(_stream_handle(stream)))
+
+
+def raw_prefill(args: PrefillArgs, stream=None) -> int:
+    """Call kda_prefill with a prepared struct; returns the status code."""
+    return int(load().kda_prefill(ctypes.byref(args), _stream_handle(stream)))

@@ -1,0 +1,167 @@
+/*
+ * kda.h -- C ABI of libkda.so, the B200 (sm_100a) Kimi Delta Attention operator.
+ *
+ * The operator (per sequence b, head h; state S is d_k x d_v, fp32):
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = S_t^T q_t,            alpha_t = exp(log_alpha_t) in (0, 1]^{d_k}
+ * Sources: "Kimi Linear's 75% KV cache cut comes from making three of every
+ * four layers recurrent" (theclarity.today), third paragraph (per-channel
+ * decay, removal of the old projection onto the key, write of the new pair)
+ * and fourth paragraph (chunked kernels with the WY representation: a chunk's
+ * rank-1 updates become triangular solves and tensor-core matrix products);
+ * "Kimi Linear wlasnie pokonal pelna uwage na wlasnych warunkach" (remio.ai),
+ * section "Jak Kimi Linear wykorzystuje inteligentniejsza pamiec
+ * rekurencyjna" (delta rule, finer-grained gates than Gated DeltaNet,
+ * blockwise algorithm with a diagonal-plus-low-rank transition, fixed-size
+ * recurrent state).
+ *
+ * Padding: a position whose pad_mask entry is 0 neither decays nor writes the
+ * state and its output is exactly 0, whatever its gate and input values
+ * ("Transformers Community Reports Kimi Linear Cache Bug: Padding May Change
+ * Subsequent Inference State", ainews, paragraphs on the reproduction and the
+ * follow-up investigation).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, on the
+ *     current CUDA device.  The library allocates no device memory.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Nothing is synchronised.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched; no output is touched in that case.
+ *   - Errors found on the device (an invalid cu_seqlens, a bounded wait that
+ *     ran out) are latched in a per-device library word and reported by
+ *     kda_get_device_status().  Kernels that follow a failed check on the same
+ *     stream return without writing.
+ *   - No C++ exception crosses the ABI.
+ *   - Layouts are row-major and contiguous.  N = total packed tokens,
+ *     B = sequences (prefill) or rows (decode), H = heads.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,    /* bad pointer, size, alignment, overlap, dtype */
+  KDA_ERR_UNSUPPORTED = 2,    /* valid but not built: head dims, chunk size */
+  KDA_ERR_CUDA = 3,           /* a CUDA runtime call failed (launch, attribute) */
+  KDA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up */
+  KDA_ERR_DEVICE_CHECK = 5    /* a device-side argument check failed */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/*
+ * Chunkwise prefill over a packed variable-length batch.
+ *
+ * Fields (all device pointers, caller-owned):
+ *   dtype        type of q, k, v and o.  log_alpha, beta and the states are
+ *                always fp32.
+ *   num_seqs     B >= 0 sequences; total_tokens N >= 0; H >= 1 heads;
+ *   dk, dv       head dimensions, each 64 or 128.
+ *   q, k         [N, H, dk]; v [N, H, dv]; 16-byte aligned.
+ *   log_alpha    [N, H, dk] fp32, natural log of the forget gate; finite and
+ *                <= 0 (values outside that range are not checked and give
+ *                unspecified results).  16-byte aligned.
+ *   beta         [N, H] fp32, finite.
+ *   cu_seqlens   [B+1] int32: cu[0] = 0, non-decreasing, cu[B] = N; sequence b
+ *                owns packed rows [cu[b], cu[b+1]).  Checked on the device
+ *                (KDA_ERR_DEVICE_CHECK, nothing written).
+ *   pad_mask     [N] uint8, 1 = valid, 0 = pad; NULL = all valid.  A pad is an
+ *                identity step with o = 0.  Pads at the two ends of a sequence
+ *                are skipped outright, so a run with edge pads is bit-identical
+ *                to the unpadded run; pads between valid tokens are identity
+ *                steps inside a chunk (equal to the unpadded run up to
+ *                rounding).  Requires a workspace.
+ *   init_state   [B, H, dk, dv] fp32 (dv contiguous), 16-byte aligned; NULL = 0.
+ *   o            [N, H, dv] of dtype; must not overlap any input.
+ *   final_state  [B, H, dk, dv] fp32 or NULL (not written).  It may be the same
+ *                pointer as init_state (in-place update) but may not otherwise
+ *                overlap an input.
+ *   chunk        0 (default: 64 for bf16, 16 for fp32), 16, 32 or 64.  The
+ *                result is defined by the recurrence and does not depend on the
+ *                chunk size beyond rounding.
+ *   workspace    device scratch of kda_prefill_workspace_size() bytes,
+ *                256-byte aligned; may be NULL only when pad_mask is NULL.
+ * Numerics: bf16 inputs take the tensor-core path (bf16 operands, fp32
+ * accumulation, fp32 state); fp32 inputs take an fp32 CUDA-core path.  o is
+ * rounded once (round to nearest even) to its dtype.
+ */
+typedef struct {
+  kda_dtype dtype;
+  int num_seqs;
+  int total_tokens;
+  int H;
+  int dk;
+  int dv;
+  const void *q;
+  const void *k;
+  const void *v;
+  const float *log_alpha;
+  const float *beta;
+  const int32_t *cu_seqlens;
+  const uint8_t *pad_mask;
+  const float *init_state;
+  void *o;
+  float *final_state;
+  int chunk;
+  void *workspace;
+  size_t workspace_bytes;
+} kda_prefill_args;
+
+/* Bytes of workspace kda_prefill() needs for these arguments (reads only the
+ * sizes).  Returns 0 if args is NULL. */
+size_t kda_prefill_workspace_size(const kda_prefill_args *args);
+
+/* Enqueue one prefill.  Returns KDA_OK or an argument/launch error. */
+kda_status kda_prefill(const kda_prefill_args *args, void *stream);
+
+/*
+ * One decode step: one new token for each of B independent rows, all heads.
+ *   q, k [B, H, dk]; v [B, H, dv] of dtype; log_alpha [B, H, dk] fp32;
+ *   beta [B, H] fp32; mask [B] uint8 (1 = active, NULL = all active);
+ *   state [B, H, dk, dv] fp32, updated in place, 16-byte aligned;
+ *   o [B, H, dv] of dtype, must not overlap any other argument.
+ * A masked row's state is neither read nor written and its o is written as 0.
+ * The step is: S' = Diag(alpha) S; p = S'^T k; S = S' + k (beta (v - p))^T;
+ * o = S^T q.
+ */
+typedef struct {
+  kda_dtype dtype;
+  int B;
+  int H;
+  int dk;
+  int dv;
+  const void *q;
+  const void *k;
+  const void *v;
+  const float *log_alpha;
+  const float *beta;
+  const uint8_t *mask;
+  float *state;
+  void *o;
+} kda_decode_args;
+
+kda_status kda_decode(const kda_decode_args *args, void *stream);
+
+/* Synchronise `stream`, then return and clear the error latched on the
+ * current device by earlier kernels (KDA_OK if none). */
+kda_status kda_get_device_status(void *stream);
+
+/* Static string for a status code; never NULL. */
+const char *kda_status_string(kda_status status);
+
+/* ABI version: (major << 16) | minor. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */
