@@ -85,6 +85,8 @@ def load(build_if_stale: bool = True) -> ctypes.CDLL:
             lib.kda_status_string.argtypes = [ctypes.c_int]
             lib.kda_status_string.restype = ctypes.c_char_p
             lib.kda_version.restype = ctypes.c_int
+            lib.kda_prefill_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), ctypes.c_void_p]
+            lib.kda_prefill_noalloc.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -226,3 +228,20 @@ def get_device_status(stream=None) -> int:
 def raw_prefill(args: PrefillArgs, stream=None) -> int:
     """Call kda_prefill with a prepared struct; returns the status code."""
     return int(load().kda_prefill(ctypes.byref(args), _stream_handle(stream)))
+
+
+NOALLOC_MAX_SEQS = 4096
+
+
+def prefill_noalloc(q, k, v, log_alpha, beta, cu_seqlens, o, final_state=None,
+                    pad_mask=None, init_state=None, chunk: int = 0, stream=None):
+    """kda_prefill_noalloc: the prefill with its scratch taken from a fixed array inside
+    the library, for callers that cannot allocate device memory at call time.  The
+    outputs ``o`` (and ``final_state``, if wanted) must be given; nothing is allocated."""
+    lib = load()
+    a = prefill_args(q, k, v, log_alpha, beta, cu_seqlens, pad_mask, init_state, o,
+                     final_state, chunk, None)
+    st = lib.kda_prefill_noalloc(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill_noalloc")
+    return o, final_state

@@ -123,6 +123,25 @@ size_t kda_prefill_workspace_size(const kda_prefill_args *args);
 kda_status kda_prefill(const kda_prefill_args *args, void *stream);
 
 /*
+ * kda_prefill without a workspace argument.  The pages have no counterpart to
+ * this call: it serves callers that cannot call cudaMalloc where they run the
+ * operator (an engine whose device memory is owned up front by a host
+ * framework that passes operators only their tensors, or a serving loop in
+ * which cudaMalloc/cudaFree are not allowed because they may synchronise the
+ * device).  Same arguments and results as kda_prefill; args->workspace and
+ * args->workspace_bytes are ignored.  The scratch comes from a fixed device
+ * array inside the library, sized for KDA_NOALLOC_MAX_SEQS sequences (64 KiB,
+ * held by every GPU that loads the library until exit); a batch with more
+ * sequences returns KDA_ERR_INVALID_ARG and launches nothing.  All calls on a
+ * device share that array: calls whose kernels may overlap on the GPU race and
+ * must be ordered by the caller.  The first call on each device looks up the
+ * array's device address; make it before any stream capture.  Allocates no
+ * memory.
+ */
+#define KDA_NOALLOC_MAX_SEQS 4096
+kda_status kda_prefill_noalloc(const kda_prefill_args *args, void *stream);
+
+/*
  * One decode step: one new token for each of B independent rows, all heads.
  *   q, k [B, H, dk]; v [B, H, dv] of dtype; log_alpha [B, H, dk] fp32;
  *   beta [B, H] fp32; mask [B] uint8 (1 = active, NULL = all active);
