@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--T", type=int, default=131072)
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-extras", action="store_true", help="headline prefill line only")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="time one workload only (for profiling runs)")
     return ap.parse_args()
 
 
@@ -70,24 +72,18 @@ def peaks():
                     source="fallback")
 
 
-def kernel_source_hash():
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "gated_delta_rule_148_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
-    return h.hexdigest()[:16]
-
-
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's source file is
+    unchanged since the capture (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-        e = d.get(kernel)
-        if e and e.get("source_hash") == kernel_source_hash():
+            e = json.load(f).get(kernel)
+        if not e:
+            return None
+        with open(os.path.join(ROOT, e["source"]), "rb") as fh:
+            h = hashlib.sha256(fh.read()).hexdigest()[:16]
+        if h == e.get("source_hash"):
             return e.get("dram_bytes_per_launch")
     except Exception:
         pass
@@ -380,7 +376,42 @@ def main_ours(args, rank, world, device):
     del o_host, fs_host
 
     if not args.no_extras:
-        # ---- batched decode
+        line["decode"] = bench_decode(args, world, device, pk)
+        line["gpu_launches"] += args.decode_steps
+        # ---- prefill sweep (smaller T; L2 flushed between iterations)
+        sweep = {}
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        for Ts in (4096, 16384, 65536):
+            if Ts >= T:
+                continue
+            _, _, _, dv_ = prefill_setup(Ts, device)
+            mss = time_loop(lambda: run_prefill(kda, dv_), max(3, K), W,
+                            flush_buf=flush if Ts <= 16384 else None)
+            ach = prefill_bytes(Ts, H) / (mss / 1e3) / 1e9
+            sweep[str(Ts)] = {"tokens_per_s": Ts / (mss / 1e3), "ms": mss,
+                              "hbm_frac": ach / pk["hbm_gbs"],
+                              "l2": "flushed" if Ts <= 16384 else "inputs larger than L2"}
+            line["gpu_launches"] += 2 * (max(3, K))
+            del dv_
+        sweep[str(T)] = {"tokens_per_s": T / (ms_step / 1e3), "ms": ms_step,
+                         "hbm_frac": roofline["frac"], "l2": "inputs larger than L2"}
+        line["prefill_sweep"] = sweep
+        del flush
+
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(args, world, device, pk):
+    """Batched decode: 256 rows x 32 heads, 26 masked rows per step; per-step time."""
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_148_b200 import kda
+    from gated_delta_rule_148_b200 import inputs as gen
+    W = args.warmup
+    if True:
         wd = gen.batched_decode()
         state = torch.from_numpy(gen.decode_state(wd)).to(device)
         pool = []
@@ -409,39 +440,20 @@ def main_ours(args, rank, world, device):
         dbytes = (active * wd.H * DECODE_ACTIVE_BYTES + wd.decode_masked * wd.H * 256
                   + wd.decode_rows)
         dach = dbytes / (dms / 1e3) / 1e9
-        line["decode"] = {
+        return {
             "workload": wd.name, "value": active * world / (dms / 1e3), "unit": "tokens/s",
             "us_per_step": dms * 1e3, "steps": Dsteps,
             "roofline": {"bound": "hbm", "achieved": dach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": dach / pk["hbm_gbs"], "traffic": recorded_traffic("decode"),
                          "algorithmic_bytes_per_launch": dbytes}}
-        line["gpu_launches"] += Dsteps
-        del state, pool, masks, o_dec
 
-        # ---- prefill sweep (smaller T; L2 flushed between iterations)
-        sweep = {}
-        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-        for Ts in (4096, 16384, 65536):
-            if Ts >= T:
-                continue
-            _, _, _, dv_ = prefill_setup(Ts, device)
-            mss = time_loop(lambda: run_prefill(kda, dv_), max(3, K), W,
-                            flush_buf=flush if Ts <= 16384 else None)
-            ach = prefill_bytes(Ts, H) / (mss / 1e3) / 1e9
-            sweep[str(Ts)] = {"tokens_per_s": Ts / (mss / 1e3), "ms": mss,
-                              "hbm_frac": ach / pk["hbm_gbs"],
-                              "l2": "flushed" if Ts <= 16384 else "inputs larger than L2"}
-            line["gpu_launches"] += 2 * (max(3, K))
-            del dv_
-        sweep[str(T)] = {"tokens_per_s": T / (ms_step / 1e3), "ms": ms_step,
-                         "hbm_frac": roofline["frac"], "l2": "inputs larger than L2"}
-        line["prefill_sweep"] = sweep
-        del flush
 
-    if rank == 0 and world == 1:
-        line["cpu_baseline"] = cpu_baseline(inp)
+def main_decode_only(args, rank, world, device):
+    from gated_delta_rule_148_b200 import kda
+    kda.load()
+    d = bench_decode(args, world, device, peaks())
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps({"metric": METRIC, "decode": d}), flush=True)
 
 
 def main():
@@ -460,7 +472,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
     try:
-        main_ours(args, rank, world, device)
+        if args.only == "decode":
+            main_decode_only(args, rank, world, device)
+        else:
+            if args.only == "prefill":
+                args.no_extras = True
+            main_ours(args, rank, world, device)
     finally:
         if world > 1:
             import torch.distributed as dist
