@@ -149,6 +149,23 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- helpers
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The max of a per-rank timing over all ranks (NCCL on the GPU, gloo on the CPU)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    on_gpu = device is not None and dist.get_backend() == "nccl"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device if on_gpu else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def to_dev(x, dtype, device, pin=True):
     import torch
     t = torch.from_numpy(np.ascontiguousarray(x))
@@ -313,16 +330,12 @@ def main_ours(args, rank, world, device):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e), world, device)
     st = kda.get_device_status()
     if st != kda.KDA_OK:
         raise RuntimeError("device status after prefill: " + kda.status_string(st))
     ms_step = ms / K
-    value = T * world / (ms_step / 1e3)
+    value = aggregate_rate(T, world, ms_step)
     algo_bytes = prefill_bytes(T, H)
     achieved = algo_bytes / (ms_step / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -362,15 +375,11 @@ def main_ours(args, rank, world, device):
         e2e_step()
     e2.record()
     torch.cuda.synchronize()
-    ms2 = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([ms2], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms2 = float(t.item())
+    ms2 = max_over_ranks(s2.elapsed_time(e2), world, device)
     h2d = sum(host[k].numel() * host[k].element_size()
               for k in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens"))
     d2h = o_host.numel() * o_host.element_size() + fs_host.numel() * 4
-    line["e2e"] = {"value": T * world / (ms2 / Ke / 1e3), "unit": "tokens/s",
+    line["e2e"] = {"value": aggregate_rate(T, world, ms2 / Ke), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
     line["gpu_launches"] += 2 * Ke
     del o_host, fs_host
@@ -431,17 +440,13 @@ def bench_decode(args, world, device, pk):
             kda.decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state, mask=masks[i],
                        o=o_dec)
             it[0] += 1
-        dms = time_loop(dstep, Dsteps, W)
-        if world > 1:
-            t = torch.tensor([dms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dms = float(t.item())
+        dms = max_over_ranks(time_loop(dstep, Dsteps, W), world, device)
         active = wd.decode_rows - wd.decode_masked
         dbytes = (active * wd.H * DECODE_ACTIVE_BYTES + wd.decode_masked * wd.H * 256
                   + wd.decode_rows)
         dach = dbytes / (dms / 1e3) / 1e9
         return {
-            "workload": wd.name, "value": active * world / (dms / 1e3), "unit": "tokens/s",
+            "workload": wd.name, "value": aggregate_rate(active, world, dms), "unit": "tokens/s",
             "us_per_step": dms * 1e3, "steps": Dsteps,
             "roofline": {"bound": "hbm", "achieved": dach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": dach / pk["hbm_gbs"], "traffic": recorded_traffic("decode"),

@@ -21,8 +21,11 @@
 //   state: [-W ; Q G] (128 x 128) . S  (accumulated on U_v)  -> U (rows 0-63), (Q G) S (64-127)
 //   out:   [0 ; M] (128 x 64) . U  (accumulated)            -> O (rows 64-127)
 //   S:     (K e^{g_C-g})^T (128 x 64) . U  (accumulated on Diag(e^{g_C}) S)
-// CUDA cores: the cumsum, the exponentials, masks, the 64 x 64 unit-lower
-// inverse (fp32, blocked 16 x 16), bf16 packing and the epilogue.
+// CUDA cores: the cumsum, the exponentials, masks, bf16 packing and the
+// epilogue; the 64 x 64 unit-lower inverse is blocked 16 x 16 with its block
+// products on warp-level tensor-core MMAs (kda_tril_inv.cuh).
+// 256 threads: thread t owns TMEM lane t % 128 and half (t / 128) of the
+// 64 columns of every accumulator it reads.
 //
 // Exactness: masked and tail rows enter as zeros (and identity gates);
 // upper-triangle entries are zeroed by selection before any product uses
@@ -35,6 +38,7 @@
 
 #include "kda_internal.cuh"
 #include "kda_tc.cuh"
+#include "kda_tril_inv.cuh"
 
 namespace kda {
 namespace {
@@ -44,7 +48,7 @@ using namespace tc;
 constexpr int kC = 64;       // chunk
 constexpr int kDK = 128;     // key dim
 constexpr int kNV = 64;      // d_v columns per CTA
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 
 // Shared-memory map (bytes from a 1024-aligned base).
@@ -57,14 +61,17 @@ constexpr uint32_t OFF_SB = OFF_V + 64 * 128;         // S (bf16)           128 
 constexpr uint32_t OFF_UB = OFF_SB + 128 * 128;       // U (bf16)            64 x 64
 constexpr uint32_t OFF_STQ = OFF_UB + 64 * 128;       // staging q  [64][128] bf16
 constexpr uint32_t OFF_STK = OFF_STQ + 64 * 256;      // staging k  [64][128] bf16
-constexpr uint32_t OFF_STG = OFF_STK + 64 * 256;      // staging log_alpha -> g [64][128] f32
+constexpr uint32_t OFF_STG = OFF_STK + 64 * 256;      // staging log_alpha [64][128] f32
 constexpr uint32_t OFF_STB = OFF_STG + 64 * 512;      // staging beta [64] f32
-// The inverse scratch aliases the staging buffers: the next chunk is staged
+// The inverse's scratch aliases the staging buffers: the next chunk is staged
 // only after the inverse is done.
-constexpr uint32_t OFF_AS = OFF_STQ;                  // A [64][65] f32 (in q/k staging)
-constexpr uint32_t OFF_TS = OFF_STG;                  // T [64][65] f32 (in g staging)
+constexpr uint32_t OFF_AS = OFF_STQ;                  // A [64][65] f32
+constexpr uint32_t OFF_XS = OFF_AS + 64 * 65 * 4;     // 8 x 16 x 17 f32 per-warp scratch
+constexpr uint32_t OFF_TS = OFF_STG;                  // T [64][65] f32
 constexpr uint32_t SMEM_USED = OFF_STB + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
+static_assert(OFF_XS + 8 * 16 * 17 * 4 <= OFF_STG, "inverse scratch must fit the q/k staging");
+static_assert(OFF_TS + 64 * 65 * 4 <= OFF_STB, "T must fit the g staging");
 
 // TMEM columns
 constexpr uint32_t TM_S = 0, TM_D1 = 64, TM_G = 128, TM_W = 192, TM_COLS = 256;
@@ -90,8 +97,7 @@ __device__ __forceinline__ void stage_chunk(const PrefillParams &p, const SeqSpa
   const int H = p.H;
   const uint32_t sq = smem_u32(base + OFF_STQ), sk = smem_u32(base + OFF_STK);
   const uint32_t sg = smem_u32(base + OFF_STG);
-  // q, k: 64 rows x 16 chunks of 16 B each
-  for (int e = tid; e < kC * 16; e += kThreads) {
+  for (int e = tid; e < kC * 16; e += kThreads) {       // q, k: 64 rows x 16 x 16 B
     const int r = e >> 4, ch = e & 15;
     const int pos = c0 + r;
     const bool ok = row_valid(p, sp, pos);
@@ -99,8 +105,7 @@ __device__ __forceinline__ void stage_chunk(const PrefillParams &p, const SeqSpa
     cp_async16(sq + r * 256 + ch * 16, (const uint16_t *)p.q + gi, ok ? 16u : 0u);
     cp_async16(sk + r * 256 + ch * 16, (const uint16_t *)p.k + gi, ok ? 16u : 0u);
   }
-  // log_alpha: 64 rows x 32 chunks of 16 B
-  for (int e = tid; e < kC * 32; e += kThreads) {
+  for (int e = tid; e < kC * 32; e += kThreads) {       // log_alpha: 64 rows x 32 x 16 B
     const int r = e >> 5, ch = e & 31;
     const int pos = c0 + r;
     const bool ok = row_valid(p, sp, pos);
@@ -109,7 +114,7 @@ __device__ __forceinline__ void stage_chunk(const PrefillParams &p, const SeqSpa
   }
   if (tid < kC) {
     const int pos = c0 + tid;
-    float* sb = reinterpret_cast<float *>(base + OFF_STB);
+    float *sb = reinterpret_cast<float *>(base + OFF_STB);
     sb[tid] = row_valid(p, sp, pos) ? p.beta[(size_t)pos * H + h] : 0.f;
   }
 }
@@ -127,57 +132,22 @@ __device__ __forceinline__ void stage_v(const PrefillParams &p, const SeqSpan &s
   }
 }
 
-__device__ __forceinline__ void st_bf16(unsigned char *tile, uint32_t off, float x) {
-  *reinterpret_cast<uint16_t *>(tile + off) = f32_to_bf16_rne(x);
+__device__ __forceinline__ void st_u32(unsigned char *tile, uint32_t off, uint32_t x) {
+  *reinterpret_cast<uint32_t *>(tile + off) = x;
 }
 
-// 64 x 64 unit-lower inverse T = (I + A)^{-1} in fp32, blocked by 16.
-// A is strictly lower (row-major, stride 65) in As; T goes to Ts (stride 65).
-__device__ void unit_lower_inverse(const float *As, float *Ts, int tid) {
-  constexpr int S = 65;
-  // diagonal 16 x 16 blocks: 64 threads, thread (blk, j) owns column j of block blk
-  if (tid < 64) {
-    const int blk = tid >> 4, j = tid & 15;
-    const int o = blk * 16;
-    for (int r = 0; r < 16; ++r) {
-      float t;
-      if (r < j) t = 0.f;
-      else if (r == j) t = 1.f;
-      else {
-        t = 0.f;
-        for (int i = j; i < r; ++i) t = fmaf(As[(o + r) * S + o + i], Ts[(o + i) * S + o + j], t);
-        t = -t;
-      }
-      Ts[(o + r) * S + o + j] = t;
-    }
+// 32 fp32 values -> bf16 into 4 consecutive 16-byte chunks (c0..c0+3) of row r.
+__device__ __forceinline__ void store_row32(unsigned char *tile, int R, int r, int chunk0,
+                                            const float *v) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
+    pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+    pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+    pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+    *reinterpret_cast<uint4 *>(tile + row_tile_chunk(r, 0, chunk0 + (j >> 3), R)) = pk;
   }
-  __syncthreads();
-  // off-diagonal blocks by distance d: T_ab = -D_a * sum_{m=b}^{a-1} A_am T_mb
-  for (int d = 1; d <= 3; ++d) {
-    const int nblk = 4 - d;                 // blocks (a, b) with a - b = d
-    // X = sum_m A_am T_mb for each block: nblk * 256 entries; write into Ts block (a,b)
-    // as a temporary, then multiply by D_a.
-    __shared__ float X[3][16][17];
-    for (int e = tid; e < nblk * 256; e += kThreads) {
-      const int q = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      const int b = q, a = q + d;
-      float acc = 0.f;
-      for (int m = b; m < a; ++m)
-        for (int i = 0; i < 16; ++i)
-          acc = fmaf(As[(a * 16 + rr) * S + m * 16 + i], Ts[(m * 16 + i) * S + b * 16 + cc], acc);
-      X[q][rr][cc] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < nblk * 256; e += kThreads) {
-      const int q = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      const int b = q, a = q + d;
-      float acc = 0.f;
-      for (int i = 0; i <= rr; ++i) acc = fmaf(Ts[(a * 16 + rr) * S + a * 16 + i], X[q][i][cc], acc);
-      Ts[(a * 16 + rr) * S + b * 16 + cc] = -acc;
-    }
-    __syncthreads();
-  }
-  // entries above the diagonal blocks are never read
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -187,11 +157,15 @@ prefill_tc_kernel(PrefillParams p) {
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ float gC_sh[kDK];
   __shared__ float beta_sh[kC];
+  __shared__ float part_sh[4][kDK];
 
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lr = tid & 127;          // TMEM lane of this thread
+  const int wg = tid >> 7;           // column half
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
   if (device_error_latched(p.err)) return;
   const int tiles = p.dv / kNV;
@@ -205,7 +179,7 @@ prefill_tc_kernel(PrefillParams p) {
   // ---- set-up: TMEM, barrier, zero rows of [T_b | 0 | M]
   if (warp == 0) tmem_alloc(&tmem_base_sh, TM_COLS);
   if (tid == 0) mbar_init(&mma_bar, 1);
-  for (int e = tid; e < 64 * 8; e += kThreads) {     // rows 64..127 of TBM = 0
+  for (int e = tid; e < 64 * 8; e += kThreads) {
     const int r = 64 + (e >> 3), ch = e & 7;
     *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(r, 0, ch, 192)) = make_uint4(0, 0, 0, 0);
   }
@@ -213,19 +187,16 @@ prefill_tc_kernel(PrefillParams p) {
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = tmem_base_sh;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);   // + accumulator base column
   uint32_t phase = 0;
   bool ok = true;
 
-  // initial state into TMEM (thread tid owns state row tid)
-  {
+  {   // initial state: thread owns row lr, columns wg*32 .. +31
     float v[32];
-    for (int half = 0; half < 2; ++half) {
-      for (int j = 0; j < 32; ++j)
-        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32 + j]
-                            : 0.f;
-      tmem_st32(tm + lane_base + TM_S + half * 32, v);
-    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32 + j] : 0.f;
+    tmem_st32(tm + my_cols + TM_S, v);
     tmem_st_wait();
   }
 
@@ -235,9 +206,8 @@ prefill_tc_kernel(PrefillParams p) {
   const uint32_t sUB = smem_u32(base + OFF_UB);
   float *As = reinterpret_cast<float *>(base + OFF_AS);
   float *Ts = reinterpret_cast<float *>(base + OFF_TS);
+  float *Xs = reinterpret_cast<float *>(base + OFF_XS);
   const float *stb = reinterpret_cast<const float *>(base + OFF_STB);
-  static_assert(OFF_AS + 64 * 65 * 4 <= OFF_STG, "A scratch must fit the q/k staging");
-  static_assert(OFF_TS + 64 * 65 * 4 <= OFF_STB, "T scratch must fit the g staging");
 
   if (sp.begin < sp.end) {
     stage_chunk(p, sp, sp.begin, h, base, tid);
@@ -248,36 +218,60 @@ prefill_tc_kernel(PrefillParams p) {
   for (int c0 = sp.begin; c0 < sp.end; c0 += kC) {
     cp_async_wait_all();
     __syncthreads();
-    // ---- P1: cumsum and operand tiles (thread = key channel)
+    // ---- P1: cumsum and operand tiles.  Thread: channels 2cp, 2cp+1; rows 16qt..16qt+15
     {
-      const int c = tid;
-      float *sg = reinterpret_cast<float *>(base + OFF_STG);
-      float g = 0.f;
-      for (int r = 0; r < kC; ++r) {
-        g += sg[r * kDK + c];
-        sg[r * kDK + c] = g;
+      const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
+      const float *sg = reinterpret_cast<const float *>(base + OFF_STG);
+      float g0[16], g1[16];
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 la = *reinterpret_cast<const float2 *>(sg + (qt * 16 + i) * kDK + c);
+        s0 += la.x;
+        s1 += la.y;
+        g0[i] = s0;
+        g1[i] = s1;
       }
-      const float gC = g;
-      gC_sh[c] = gC;
+      part_sh[qt][c] = s0;
+      part_sh[qt][c + 1] = s1;
       if (tid < kC) beta_sh[tid] = stb[tid];
-      const uint16_t *sq = reinterpret_cast<const uint16_t *>(base + OFF_STQ);
-      const uint16_t *sk = reinterpret_cast<const uint16_t *>(base + OFF_STK);
-      for (int r = 0; r < kC; ++r) {
-        const float gr = sg[r * kDK + c];
-        const float qv = bf16_to_f32(sq[r * kDK + c]);
-        const float kv = bf16_to_f32(sk[r * kDK + c]);
-        const float e1 = __expf(gr);                   // <= 1
-        const float e2 = __expf(gC - gr);              // <= 1
-        const float e3 = __expf(fminf(-gr, 80.f));     // >= 1
-        st_bf16(base + OFF_QKW, row_tile_off(64 + r, c, 192), qv * e1);
-        st_bf16(base + OFF_QKW, row_tile_off(128 + r, c, 192), kv * e1);
-        st_bf16(base + OFF_KH, row_tile_off(r, c, 64), kv * e3);
-        st_bf16(base + OFF_KT, row_tile_off(r, c, 64), kv * e2);
+      __syncthreads();
+      float off0 = 0.f, off1 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q < qt) {
+          off0 += part_sh[q][c];
+          off1 += part_sh[q][c + 1];
+        }
+      }
+      const float gC0 = part_sh[0][c] + part_sh[1][c] + part_sh[2][c] + part_sh[3][c];
+      const float gC1 = part_sh[0][c + 1] + part_sh[1][c + 1] + part_sh[2][c + 1] + part_sh[3][c + 1];
+      if (qt == 0) {
+        gC_sh[c] = gC0;
+        gC_sh[c + 1] = gC1;
+      }
+      const float en0 = __expf(fminf(-gC0, 80.f)), en1 = __expf(fminf(-gC1, 80.f));
+      const uint32_t *sq = reinterpret_cast<const uint32_t *>(base + OFF_STQ);
+      const uint32_t *sk = reinterpret_cast<const uint32_t *>(base + OFF_STK);
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int r = qt * 16 + i;
+        const float ga = g0[i] + off0, gb = g1[i] + off1;
+        const uint32_t qq = sq[r * 64 + cp], kk = sk[r * 64 + cp];
+        const float qa = __uint_as_float(qq << 16), qb = __uint_as_float(qq & 0xFFFF0000u);
+        const float ka = __uint_as_float(kk << 16), kb = __uint_as_float(kk & 0xFFFF0000u);
+        const float e1a = __expf(ga), e1b = __expf(gb);              // e^{g}       <= 1
+        const float e2a = __expf(gC0 - ga), e2b = __expf(gC1 - gb);  // e^{g_C - g} <= 1
+        const float e3a = e2a * en0, e3b = e2b * en1;                // e^{-g}
+        st_u32(base + OFF_QKW, row_tile_off(64 + r, c, 192), pack_bf16x2(qa * e1a, qb * e1b));
+        st_u32(base + OFF_QKW, row_tile_off(128 + r, c, 192), pack_bf16x2(ka * e1a, kb * e1b));
+        st_u32(base + OFF_KH, row_tile_off(r, c, 64), pack_bf16x2(ka * e3a, kb * e3b));
+        st_u32(base + OFF_KT, row_tile_off(r, c, 64), pack_bf16x2(ka * e2a, kb * e2b));
       }
     }
     fence_async_smem();
     __syncthreads();
-    // ---- Gram
+    // ---- Gram: [Q G ; K G] (K e^{-g})^T
     if (tid == 0) {
       fence_after_sync();
       const uint32_t id = idesc_bf16(128, 64, 0, 0);
@@ -289,51 +283,44 @@ prefill_tc_kernel(PrefillParams p) {
     phase++;
     if (!ok) break;
     fence_after_sync();
-    // ---- P3: M rows (lanes 0-63) -> TBM rows 128..191; A rows (lanes 64-127) -> As
+    // ---- P3: M rows (lanes 0-63) -> TBM rows 128..191; beta * A rows (lanes 64-127) -> As
     {
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + TM_G + half * 32, v);
-        if (tid < kC) {
-          const int r = tid;
-          for (int j = 0; j < 32; j += 8) {
-            uint4 pk;
-            const int i0 = half * 32 + j;
-            pk.x = pack_bf16x2(i0 + 0 <= r ? v[j + 0] : 0.f, i0 + 1 <= r ? v[j + 1] : 0.f);
-            pk.y = pack_bf16x2(i0 + 2 <= r ? v[j + 2] : 0.f, i0 + 3 <= r ? v[j + 3] : 0.f);
-            pk.z = pack_bf16x2(i0 + 4 <= r ? v[j + 4] : 0.f, i0 + 5 <= r ? v[j + 5] : 0.f);
-            pk.w = pack_bf16x2(i0 + 6 <= r ? v[j + 6] : 0.f, i0 + 7 <= r ? v[j + 7] : 0.f);
-            *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(128 + r, 0, i0 >> 3, 192)) = pk;
-          }
-        } else {
-          const int r = tid - kC;
-          for (int j = 0; j < 32; ++j) {
-            const int i = half * 32 + j;
-            As[r * 65 + i] = (i < r) ? beta_sh[r] * v[j] : 0.f;
-          }
+      tmem_ld32(tm + my_cols + TM_G, v);
+      if (lr < kC) {
+        const int r = lr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (wg * 32 + j <= r) ? v[j] : 0.f;
+        store_row32(base + OFF_TBM, 192, 128 + r, wg * 4, v);
+      } else {
+        const int r = lr - kC;
+        const float br = beta_sh[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int i = wg * 32 + j;
+          As[r * 65 + i] = (i < r) ? br * v[j] : 0.f;
         }
       }
     }
     __syncthreads();
     // ---- P4: T = (I + A)^{-1};  T_b = T Diag(beta) -> TBM rows 0..63
-    unit_lower_inverse(As, Ts, tid);
-    __syncthreads();
+    tri::unit_lower_inverse_64(As, Ts, Xs, tid);
     {
-      // thread pairs (row r, half): 64 rows x 2 halves of 32 columns
-      const int r = tid >> 1, hh = tid & 1;
-      for (int j = 0; j < 32; j += 8) {
-        const int i0 = hh * 32 + j;
-        float t[8];
-        for (int u = 0; u < 8; ++u) {
-          const int i = i0 + u;
-          t[u] = (i <= r) ? Ts[r * 65 + i] * beta_sh[i] : 0.f;
-        }
+      const int r = tid >> 2, qq = tid & 3;      // row r, columns 16qq .. 16qq+15
+      float t[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = qq * 16 + u;
+        t[u] = (i <= r) ? Ts[r * 65 + i] * beta_sh[i] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; j += 8) {
         uint4 pk;
-        pk.x = pack_bf16x2(t[0], t[1]);
-        pk.y = pack_bf16x2(t[2], t[3]);
-        pk.z = pack_bf16x2(t[4], t[5]);
-        pk.w = pack_bf16x2(t[6], t[7]);
-        *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(r, 0, i0 >> 3, 192)) = pk;
+        pk.x = pack_bf16x2(t[j + 0], t[j + 1]);
+        pk.y = pack_bf16x2(t[j + 2], t[j + 3]);
+        pk.z = pack_bf16x2(t[j + 4], t[j + 5]);
+        pk.w = pack_bf16x2(t[j + 6], t[j + 7]);
+        *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(r, 0, (qq * 16 + j) >> 3, 192)) = pk;
       }
     }
     fence_async_smem();
@@ -358,35 +345,27 @@ prefill_tc_kernel(PrefillParams p) {
     phase++;
     if (!ok) break;
     fence_after_sync();
-    // ---- P6: -W into QKW rows 0..63 (thread = channel c); S -> bf16 tile, S *= e^{g_C}
+    // ---- P6: -W into QKW rows 0..63 (lane = channel); S -> bf16 tile; S *= e^{g_C}
     {
-      const int c = tid;
+      const int c = lr;
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + TM_W + half * 32, v);
-        for (int j = 0; j < 32; ++j) st_bf16(base + OFF_QKW, row_tile_off(half * 32 + j, c, 192), -v[j]);
-      }
+      tmem_ld32(tm + my_cols + TM_W, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        *reinterpret_cast<uint16_t *>(base + OFF_QKW + row_tile_off(wg * 32 + j, c, 192)) =
+            f32_to_bf16_rne(-v[j]);
+      tmem_ld32(tm + my_cols + TM_S, v);
+      store_row32(base + OFF_SB, 128, c, wg * 4, v);
       const float decay = __expf(gC_sh[c]);
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + TM_S + half * 32, v);
-        for (int j = 0; j < 32; j += 8) {
-          uint4 pk;
-          pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
-          pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
-          pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
-          pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-          *reinterpret_cast<uint4 *>(base + OFF_SB + row_tile_chunk(c, 0, (half * 32 + j) >> 3, 128)) = pk;
-        }
-        for (int j = 0; j < 32; ++j) v[j] *= decay;
-        tmem_st32(tm + lane_base + TM_S + half * 32, v);
-      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= decay;
+      tmem_st32(tm + my_cols + TM_S, v);
       tmem_st_wait();
     }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
-    // V slice of the next chunk (the U_v product that read V is complete)
-    if (c0 + kC < sp.end) {
+    if (c0 + kC < sp.end) {        // the U_v product that read V is complete
       stage_v(p, sp, c0 + kC, h, dv0, base, tid);
       cp_async_commit();
     }
@@ -403,21 +382,10 @@ prefill_tc_kernel(PrefillParams p) {
     if (!ok) break;
     fence_after_sync();
     // ---- P8: U (lanes 0-63) -> bf16 tile
-    {
+    if ((warp & 3) < 2) {
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + TM_D1 + half * 32, v);
-        if (tid < kC) {
-          for (int j = 0; j < 32; j += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
-            pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
-            pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
-            pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-            *reinterpret_cast<uint4 *>(base + OFF_UB + row_tile_chunk(tid, 0, (half * 32 + j) >> 3, 64)) = pk;
-          }
-        }
-      }
+      tmem_ld32(tm + my_cols + TM_D1, v);
+      store_row32(base + OFF_UB, 64, lr, wg * 4, v);
     }
     fence_async_smem();
     fence_before_sync();
@@ -438,25 +406,22 @@ prefill_tc_kernel(PrefillParams p) {
     if (!ok) break;
     fence_after_sync();
     // ---- P10: O (lanes 64-127) -> global
-    {
+    if ((warp & 3) >= 2) {
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + TM_D1 + half * 32, v);
-        if (tid >= kC) {
-          const int r = tid - kC;
-          const int pos = c0 + r;
-          if (pos < sp.end) {
-            const bool valid = p.mask == nullptr || p.mask[pos] != 0;
-            uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + half * 32;
-            for (int j = 0; j < 32; j += 8) {
-              uint4 pk;
-              pk.x = valid ? pack_bf16x2(v[j + 0], v[j + 1]) : 0u;
-              pk.y = valid ? pack_bf16x2(v[j + 2], v[j + 3]) : 0u;
-              pk.z = valid ? pack_bf16x2(v[j + 4], v[j + 5]) : 0u;
-              pk.w = valid ? pack_bf16x2(v[j + 6], v[j + 7]) : 0u;
-              *reinterpret_cast<uint4 *>(orow + j) = pk;
-            }
-          }
+      tmem_ld32(tm + my_cols + TM_D1, v);
+      const int r = lr - kC;
+      const int pos = c0 + r;
+      if (pos < sp.end) {
+        const bool valid = p.mask == nullptr || p.mask[pos] != 0;
+        uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * 32;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 pk;
+          pk.x = valid ? pack_bf16x2(v[j + 0], v[j + 1]) : 0u;
+          pk.y = valid ? pack_bf16x2(v[j + 2], v[j + 3]) : 0u;
+          pk.z = valid ? pack_bf16x2(v[j + 4], v[j + 5]) : 0u;
+          pk.w = valid ? pack_bf16x2(v[j + 6], v[j + 7]) : 0u;
+          *reinterpret_cast<uint4 *>(orow + j) = pk;
         }
       }
     }
@@ -470,12 +435,11 @@ prefill_tc_kernel(PrefillParams p) {
     mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
   } else if (p.final_state) {
     float v[32];
-    for (int half = 0; half < 2; ++half) {
-      tmem_ld32(tm + lane_base + TM_S + half * 32, v);
-      float *dst = p.final_state + (((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32;
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-    }
+    tmem_ld32(tm + my_cols + TM_S, v);
+    float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
   }
   cp_async_wait_all();
   fence_before_sync();
