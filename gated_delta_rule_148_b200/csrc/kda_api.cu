@@ -72,8 +72,16 @@ const char *kda_status_string(kda_status s) {
   return "KDA_ERR_UNKNOWN";
 }
 
+// Whether a call may take the two-kernel tensor-core path (given enough workspace).
+bool split_eligible(const kda_prefill_args *a) {
+  const int chunk = a->chunk == 0 ? (a->dtype == KDA_BF16 ? 64 : 16) : a->chunk;
+  return a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 && chunk == 64 && a->num_seqs > 0 &&
+         a->total_tokens >= 0 && a->H >= 1;
+}
+
 size_t kda_prefill_workspace_size(const kda_prefill_args *a) {
   if (!a) return 0;
+  if (split_eligible(a)) return prefill_split_workspace(a->total_tokens, a->num_seqs, a->H);
   return spans_bytes(a->num_seqs);
 }
 
@@ -106,10 +114,11 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   for (const void *p : need16)
     if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
   if (!aligned(a->beta, 4) || !aligned(a->cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
-  if (a->pad_mask) {
-    if (!a->workspace || a->workspace_bytes < kda_prefill_workspace_size(a)) return KDA_ERR_INVALID_ARG;
-    if (!aligned(a->workspace, 256)) return KDA_ERR_INVALID_ARG;
-  }
+  // A pad mask needs at least the span table; a larger workspace (up to
+  // kda_prefill_workspace_size) only selects a faster path.
+  if (a->pad_mask && (!a->workspace || a->workspace_bytes < spans_bytes(a->num_seqs)))
+    return KDA_ERR_INVALID_ARG;
+  if (a->workspace && !aligned(a->workspace, 256)) return KDA_ERR_INVALID_ARG;
   // o and final_state must not overlap any input; init/final may coincide exactly
   const Range inputs[] = {q, k, v, la, be, cu, mk, s0, ws};
   for (const Range &r : inputs) {
@@ -141,14 +150,20 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   p.o = a->o;
   p.final_state = a->final_state;
   p.err = err;
-  SeqSpan *spans = a->pad_mask ? static_cast<SeqSpan *>(a->workspace) : nullptr;
-  p.spans = nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = a->dtype == KDA_BF16;
+  p.spans = nullptr;
+  // Two-kernel path when the workspace holds the per-chunk items; otherwise the
+  // fused tensor-core kernel (or the CUDA-core kernel for other shapes).
+  const bool split = prefill_split_supported(p, bf16) && a->workspace &&
+                     a->workspace_bytes >= prefill_split_workspace(a->total_tokens, a->num_seqs, a->H);
+  SeqSpan *spans = (split || a->pad_mask) ? static_cast<SeqSpan *>(a->workspace) : nullptr;
   if (launch_prefill_prepass(p, bf16, spans, s) != cudaSuccess) return KDA_ERR_CUDA;
   p.spans = spans;
-  cudaError_t e = prefill_tc_supported(p, bf16) ? launch_prefill_tc(p, s)
-                                                : launch_prefill_simt(p, bf16, s);
+  cudaError_t e;
+  if (split) e = launch_prefill_split(p, spans, a->workspace, s);
+  else if (prefill_tc_supported(p, bf16)) e = launch_prefill_tc(p, s);
+  else e = launch_prefill_simt(p, bf16, s);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

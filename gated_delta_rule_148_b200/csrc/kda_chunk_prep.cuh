@@ -1,0 +1,175 @@
+// Per-chunk intra work of the tensor-core prefill, shared by the fused kernel
+// and the intra kernel of the two-kernel path.  All functions run on 256
+// threads (two warpgroups); thread t owns TMEM lane t % 128 and the column half
+// t / 128 of any 64-column accumulator it reads.
+//
+// Chunk algebra (C = 64 rows, g = inclusive per-channel cumsum of log_alpha in
+// the chunk, a_r = e^{log_alpha_r}; "Kimi Linear's 75% KV cache cut ...",
+// theclarity.today, fourth paragraph, WY form of a chunk):
+//   e^{g_r} = prod_{j<=r} a_j,  e^{g_C - g_r} = prod_{j>r} a_j,  e^{-g_r} = e^{g_C - g_r} / e^{g_C}
+//   Q G = q e^{g},  K G = k e^{g},  K e^{-g},  K e^{g_C - g}  (bf16 operand tiles)
+#pragma once
+
+#include "kda_internal.cuh"
+#include "kda_tc.cuh"
+
+namespace kda {
+namespace prep {
+
+using namespace tc;
+
+constexpr int kC = 64;
+constexpr int kDK = 128;
+
+struct PrepTiles {
+  unsigned char *qg;      // Q G rows (K-major row tile `qg_R` rows, starting row `qg_row0`)
+  int qg_R, qg_row0;
+  unsigned char *kg;      // K G rows (same tile as qg in both kernels)
+  int kg_R, kg_row0;
+  unsigned char *kh;      // K e^{-g}      (64-row tile)
+  unsigned char *kt;      // K e^{g_C - g} (64-row tile)
+};
+
+// P1.  Thread: channels 2cp, 2cp+1 (cp = tid % 64), rows 16qt..16qt+15 (qt = tid / 64).
+// Reads staged q, k ([64][128] bf16) and log_alpha ([64][128] f32); rows whose bit is
+// clear in `valid` count as zero.  Writes the four operand tiles, decay[c] = e^{g_C}
+// (qt == 0 threads) and beta_out (threads 0..63 copy beta_in).  Contains one
+// __syncthreads(); must be called by all 256 threads.
+__device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint16_t *sk16,
+                                                const float *sg, const uint32_t *valid,
+                                                const PrepTiles &t, float (*part)[kDK],
+                                                float *decay, const float *beta_in,
+                                                float *beta_out, int tid) {
+  const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
+  const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
+  float a0[16], a1[16];
+  float t0 = 1.f, t1 = 1.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float2 la = *reinterpret_cast<const float2 *>(sg + (qt * 16 + i) * kDK + c);
+    if (!((vbits >> i) & 1u)) la = make_float2(0.f, 0.f);
+    a0[i] = __expf(la.x);
+    a1[i] = __expf(la.y);
+    t0 *= a0[i];
+    t1 *= a1[i];
+  }
+  part[qt][c] = t0;
+  part[qt][c + 1] = t1;
+  if (tid < kC) beta_out[tid] = beta_in[tid];
+  __syncthreads();
+  float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float x0 = part[q][c], x1 = part[q][c + 1];
+    if (q < qt) { pre0 *= x0; pre1 *= x1; }
+    if (q > qt) { suf0 *= x0; suf1 *= x1; }
+  }
+  const float GC0 = pre0 * t0 * suf0, GC1 = pre1 * t1 * suf1;   // e^{g_C}
+  if (qt == 0) {
+    decay[c] = GC0;
+    decay[c + 1] = GC1;
+  }
+  // e^{-g_C}, clamped where e^{g_C} underflows (outside the tensor-core path's domain)
+  const float inv0 = GC0 > 1e-35f ? 1.f / GC0 : 1e35f, inv1 = GC1 > 1e-35f ? 1.f / GC1 : 1e35f;
+  const uint32_t *sq = reinterpret_cast<const uint32_t *>(sq16);
+  const uint32_t *sk = reinterpret_cast<const uint32_t *>(sk16);
+  const int kb = c >> 6, ch = (c & 63) >> 3;
+  const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
+  const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
+  const uint32_t col64 = (uint32_t)(kb * 64 * 128 + (c & 7) * 2);
+  // forward: e^{g_r} -> Q G and K G
+  float e0 = pre0, e1 = pre1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = qt * 16 + i;                      // r & 7 == i & 7 (row offsets are multiples of 8)
+    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
+    const bool vr = (vbits >> i) & 1u;
+    const uint32_t qq = vr ? sq[r * 64 + cp] : 0u, kk = vr ? sk[r * 64 + cp] : 0u;
+    const float qa = __uint_as_float(qq << 16), qb = __uint_as_float(qq & 0xFFFF0000u);
+    const float ka = __uint_as_float(kk << 16), kb2 = __uint_as_float(kk & 0xFFFF0000u);
+    e0 *= a0[i];
+    e1 *= a1[i];
+    *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) =
+        pack_bf16x2(qa * e0, qb * e1);
+    *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
+        pack_bf16x2(ka * e0, kb2 * e1);
+  }
+  // backward: e^{g_C - g_r} -> K e^{g_C - g} and K e^{-g}
+  float s0 = suf0, s1 = suf1;
+#pragma unroll
+  for (int i = 15; i >= 0; --i) {
+    const int r = qt * 16 + i;
+    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
+    const bool vr = (vbits >> i) & 1u;
+    const uint32_t kk = vr ? sk[r * 64 + cp] : 0u;
+    const float ka = __uint_as_float(kk << 16), kb2 = __uint_as_float(kk & 0xFFFF0000u);
+    const uint32_t rr = (uint32_t)(r * 128) + sw;
+    *reinterpret_cast<uint32_t *>(t.kt + col64 + rr) = pack_bf16x2(ka * s0, kb2 * s1);
+    *reinterpret_cast<uint32_t *>(t.kh + col64 + rr) = pack_bf16x2(ka * (s0 * inv0), kb2 * (s1 * inv1));
+    s0 *= a0[i];
+    s1 *= a1[i];
+  }
+}
+
+// 32 fp32 values -> bf16 into 4 consecutive 16-byte chunks (chunk0..chunk0+3) of row r
+// of a K-major row tile with R rows and one 64-column block.
+__device__ __forceinline__ void store_row32(unsigned char *tile, int R, int r, int chunk0,
+                                            const float *v) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
+    pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+    pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+    pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+    *reinterpret_cast<uint4 *>(tile + row_tile_chunk(r, 0, chunk0 + (j >> 3), R)) = pk;
+  }
+}
+
+// P3.  The Gram accumulator (TMEM, 64 columns at `gram_col`) holds M in lanes 0-63
+// and A / beta in lanes 64-127.  Writes tril_0(M) as bf16 into rows m_row0.. of the
+// 64-column tile `mtile` (R rows) and beta_r * tril_{-1}(A) into As ([64][65] f32).
+__device__ __forceinline__ void extract_gram(uint32_t tm_cols, unsigned char *mtile, int mR,
+                                             int m_row0, float *As, const float *beta, int tid) {
+  const int lr = tid & 127, wg = tid >> 7;
+  float v[32];
+  tmem_ld32(tm_cols, v);
+  if (lr < kC) {
+    const int r = lr;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = (wg * 32 + j <= r) ? v[j] : 0.f;
+    store_row32(mtile, mR, m_row0 + r, wg * 4, v);
+  } else {
+    const int r = lr - kC;
+    const float br = beta[r];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int i = wg * 32 + j;
+      As[r * 65 + i] = (i < r) ? br * v[j] : 0.f;
+    }
+  }
+}
+
+// T_b = T Diag(beta) (lower part of T in Ts [64][65] f32) -> bf16 rows 0..63 of `ttile` (R rows).
+__device__ __forceinline__ void pack_tb(const float *Ts, const float *beta, unsigned char *ttile,
+                                        int R, int tid) {
+  const int r = tid >> 2, qq = tid & 3;      // row r, columns 16qq .. 16qq+15
+  float t[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int i = qq * 16 + u;
+    t[u] = (i <= r) ? Ts[r * 65 + i] * beta[i] : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; j += 8) {
+    uint4 pk;
+    pk.x = pack_bf16x2(t[j + 0], t[j + 1]);
+    pk.y = pack_bf16x2(t[j + 2], t[j + 3]);
+    pk.z = pack_bf16x2(t[j + 4], t[j + 5]);
+    pk.w = pack_bf16x2(t[j + 6], t[j + 7]);
+    *reinterpret_cast<uint4 *>(ttile + row_tile_chunk(r, 0, (qq * 16 + j) >> 3, R)) = pk;
+  }
+}
+
+}  // namespace prep
+}  // namespace kda

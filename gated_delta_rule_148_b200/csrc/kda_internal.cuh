@@ -51,8 +51,12 @@ struct DecodeParams {
 cudaError_t launch_prefill_prepass(const PrefillParams &p, bool bf16, SeqSpan *spans,
                                    cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams &p, bool bf16, cudaStream_t s);
-cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t s);
+cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t s);  // may return
+                                                                          // cudaErrorNotSupported
 bool prefill_tc_supported(const PrefillParams &p, bool bf16);
+bool prefill_split_supported(const PrefillParams &p, bool bf16);
+size_t prefill_split_workspace(int N, int B, int H);
+cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
 
 // ---------------------------------------------------------------- helpers

@@ -271,9 +271,20 @@ prefill_prepass_kernel(PrefillParams p, SeqSpan *spans) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(p.err, ERR_BIT_CHECK);
     return;
   }
-  if (p.mask == nullptr || spans == nullptr) return;
+  if (spans == nullptr) return;
   const int b = blockIdx.x;
   const int beg = p.cu[b], end = p.cu[b + 1];
+  if (p.mask == nullptr) {      // no pads: the span is the whole sequence
+    if (tid == 0) {
+      SeqSpan sp;
+      sp.seq_begin = beg;
+      sp.begin = beg;
+      sp.end = end;
+      sp.pad_inside = 0;
+      spans[b] = sp;
+    }
+    return;
+  }
   int first = INT_MAX, last = -1, count = 0;
   for (int pos = beg + tid; pos < end; pos += blockDim.x) {
     if (p.mask[pos]) {
@@ -313,7 +324,7 @@ prefill_prepass_kernel(PrefillParams p, SeqSpan *spans) {
 
 cudaError_t launch_prefill_prepass(const PrefillParams &p, bool bf16, SeqSpan *spans,
                                    cudaStream_t s) {
-  const unsigned grid = (p.num_seqs > 0 && p.mask && spans) ? (unsigned)p.num_seqs : 1u;
+  const unsigned grid = (p.num_seqs > 0 && spans) ? (unsigned)p.num_seqs : 1u;
   if (bf16) prefill_prepass_kernel<true><<<grid, 256, 0, s>>>(p, spans);
   else prefill_prepass_kernel<false><<<grid, 256, 0, s>>>(p, spans);
   return cudaGetLastError();

@@ -1,0 +1,558 @@
+// Two-kernel tensor-core prefill: the state-independent work of every chunk
+// runs fully in parallel, the state pass runs once per (sequence, head, d_v
+// slice).  Same chunk algebra as the fused kernel (kda_prefill_tc.cu):
+//   intra (one CTA per chunk and head, all SMs):  Q G, K e^{g_C-g}, M = tril(Q G (K e^{-g})^T),
+//     T_b = (I + beta tril(K G (K e^{-g})^T))^{-1} Diag(beta), W = T_b K G, U_v = T_b V, e^{g_C}
+//   state pass (one CTA per sequence, head, 64 columns of d_v; chunks in order):
+//     U = U_v - W S;  O = (Q G) S + M U;  S <- Diag(e^{g_C}) S + (K e^{g_C-g})^T U
+// ("Kimi Linear's 75% KV cache cut ...", theclarity.today, fourth paragraph:
+// chunks and the WY representation; "Kimi Linear wlasnie pokonal ...",
+// remio.ai: blockwise algorithm with a diagonal-plus-low-rank transition.)
+//
+// The intra kernel writes each (chunk, head) item to the workspace in the exact
+// 128-byte-swizzled shared-memory tile layout the state pass consumes, with
+// bulk (TMA) stores; the state pass streams items back with bulk loads into
+// two alternating buffers.  Workspace per item (74 752 bytes):
+//   [0, 32768)      [-W ; Q G]  128 x 128 bf16 row tile
+//   [32768, 49152)  K e^{g_C-g}  64 x 128 bf16 row tile
+//   [49152, 65536)  U_v          64 rows x 128 bf16, two 64-column blocks (MN-major tile)
+//   [65536, 73728)  M            64 x 64 bf16 row tile
+//   [73728, 74240)  e^{g_C}      128 fp32
+#include <climits>
+
+#include <cudaTypedefs.h>
+
+#include "kda_internal.cuh"
+#include "kda_tc.cuh"
+#include "kda_tril_inv.cuh"
+#include "kda_chunk_prep.cuh"
+
+namespace kda {
+namespace split {
+
+using namespace tc;
+
+constexpr int kC = 64, kDK = 128, kNV = 64;
+constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
+
+// ---- item layout
+constexpr uint32_t IT_WQ = 0, IT_KT = 32768, IT_UV = 49152, IT_M = 65536, IT_GC = 73728;
+constexpr uint32_t ITEM_BYTES = 74752;
+
+// ---- workspace layout
+__host__ __device__ inline size_t ws_spans_bytes(int B) { return ((size_t)B * 16 + 255) / 256 * 256; }
+__host__ __device__ inline size_t ws_cbase_off(int B) { return ws_spans_bytes(B); }
+__host__ __device__ inline size_t ws_items_off(int B) {
+  return (ws_cbase_off(B) + (size_t)(B + 1) * 4 + 1023) / 1024 * 1024;
+}
+__host__ __device__ inline size_t max_chunks(int N, int B) { return (size_t)N / kC + (size_t)B; }
+__host__ __device__ inline size_t ws_total(int N, int B, int H) {
+  return ws_items_off(B) + max_chunks(N, B) * (size_t)H * ITEM_BYTES;
+}
+
+// ============================================================ chunk index
+// chunk_base[b] = number of 64-row chunks of sequences 0..b-1 (spans after edge pads).
+__global__ void __launch_bounds__(1024) chunk_index_kernel(PrefillParams p, const SeqSpan *spans,
+                                                           int *cbase) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  if (device_error_latched(p.err)) return;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < p.num_seqs; b0 += 1024) {
+    const int b = b0 + tid;
+    int n = 0;
+    if (b < p.num_seqs) n = (spans[b].end - spans[b].begin + kC - 1) / kC;
+    int x = n;   // inclusive warp scan
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = warp_tot[lane], u = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, u, o);
+        if (lane >= o) u += y;
+      }
+      warp_tot[lane] = u - t;   // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int excl = carry + warp_tot[w] + x - n;
+    if (b < p.num_seqs) cbase[b] = excl;
+    __syncthreads();
+    if (tid == 1023) carry = excl + n;
+    __syncthreads();
+  }
+  if (tid == 0) cbase[p.num_seqs] = carry;
+}
+
+// ============================================================ intra kernel (A)
+struct IntraMaps {
+  CUtensorMap q, k, la;   // [N, H, 128] boxes {128, 1, 64}
+  CUtensorMap v;          // [N, H, dv] boxes {64, 1, 64}, 128-byte swizzle
+};
+
+constexpr int kThreadsA = 256;
+constexpr uint32_t A_QKW = 0;                       // [-W | Q G | K G] 192 x 128
+constexpr uint32_t A_KH = A_QKW + 192 * 256;        // K e^{-g}       64 x 128
+constexpr uint32_t A_KT = A_KH + 64 * 256;          // K e^{g_C - g}  64 x 128
+constexpr uint32_t A_TBM = A_KT + 64 * 256;         // [T_b | 0 | M]  192 x 64
+constexpr uint32_t A_V = A_TBM + 192 * 128;         // V  64 rows x 2 blocks of 64
+constexpr uint32_t A_UV = A_V + 64 * 256;           // U_v 64 rows x 2 blocks of 64
+constexpr uint32_t A_STQ = A_UV + 64 * 256;         // staging q [64][128] bf16
+constexpr uint32_t A_STK = A_STQ + 64 * 256;        // staging k
+constexpr uint32_t A_STG = A_STK + 64 * 256;        // staging log_alpha [64][128] f32
+constexpr uint32_t A_AS = A_STQ;                    // A [64][65] f32 (aliases staging)
+constexpr uint32_t A_XS = A_AS + 64 * 65 * 4;       // inverse scratch
+constexpr uint32_t A_TS = A_STG;                    // T [64][65] f32
+constexpr uint32_t A_USED = A_STG + 64 * 512;
+constexpr uint32_t A_SMEM = A_USED + 1024;
+static_assert(A_XS + 8 * 16 * 17 * 4 <= A_STG, "scratch fits the q/k staging");
+constexpr uint32_t A_TM_G = 0, A_TM_W = 64, A_TM_UV = 128, A_TM_COLS = 256;
+constexpr uint32_t kStageBytesA = 64 * 256 * 2 + 64 * 512 + 2 * 64 * 128;   // q, k, log_alpha, V
+
+__device__ __forceinline__ bool row_ok(const PrefillParams &p, const SeqSpan &sp, int pos) {
+  return pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
+}
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqSpan *spans,
+             const int *cbase, unsigned char *items) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ __align__(8) uint64_t stage_bar;
+  __shared__ uint32_t valid_sh[2];
+  __shared__ __align__(16) float decay_sh[kDK];
+  __shared__ float beta_sh[kC];
+  __shared__ float beta_st[kC];
+  __shared__ float part_sh[4][kDK];
+
+  if (device_error_latched(p.err)) return;
+  const int H = p.H;
+  const int gchunk = blockIdx.x / H, h = blockIdx.x % H;
+  const int nchunks = cbase[p.num_seqs];
+  if (gchunk >= nchunks) return;
+  // sequence of this chunk: the last b with cbase[b] <= gchunk
+  int lo = 0, hi = p.num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const SeqSpan sp = spans[b];
+  const int c0 = sp.begin + (gchunk - cbase[b]) * kC;
+
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char *base = smem_raw + pad;
+  const int tid = threadIdx.x, warp = tid >> 5, lr = tid & 127, wg = tid >> 7;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+  if (warp == 0) tmem_alloc(&tmem_base_sh, A_TM_COLS);
+  if (tid == 0) {
+    mbar_init(&mma_bar, 1);
+    mbar_init(&stage_bar, 1);
+  }
+  for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0 | M] = 0
+    const int r = 64 + (e >> 3), ch = e & 7;
+    *reinterpret_cast<uint4 *>(base + A_TBM + row_tile_chunk(r, 0, ch, 192)) = make_uint4(0, 0, 0, 0);
+  }
+  if (tid < kC) {
+    const bool ok = row_ok(p, sp, c0 + tid);
+    const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
+    if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
+    beta_st[tid] = ok ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = tmem_base_sh;
+  const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&stage_bar, kStageBytesA);
+    tma_load_3d(smem_u32(base + A_STQ), &maps.q, 0, h, c0, &stage_bar);
+    tma_load_3d(smem_u32(base + A_STK), &maps.k, 0, h, c0, &stage_bar);
+    tma_load_3d(smem_u32(base + A_STG), &maps.la, 0, h, c0, &stage_bar);
+    tma_load_3d(smem_u32(base + A_V), &maps.v, 0, h, c0, &stage_bar);
+    tma_load_3d(smem_u32(base + A_V + 64 * 128), &maps.v, 64, h, c0, &stage_bar);
+  }
+  bool ok = __syncthreads_and(mbar_wait(&stage_bar, 0, kWaitCycles));
+  uint32_t phase = 0;
+  if (ok) {
+    // zero V rows of invalid positions (tail of the sequence, pads)
+    if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
+      for (int e = tid; e < kC * 16; e += kThreadsA) {
+        const int r = e >> 4, blk = (e >> 3) & 1, ch = e & 7;
+        if (!((valid_sh[r >> 5] >> (r & 31)) & 1u))
+          *reinterpret_cast<uint4 *>(base + A_V + row_tile_chunk(r, blk, ch, kC)) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    prep::PrepTiles t;
+    t.qg = base + A_QKW; t.qg_R = 192; t.qg_row0 = 64;
+    t.kg = base + A_QKW; t.kg_R = 192; t.kg_row0 = 128;
+    t.kh = base + A_KH;
+    t.kt = base + A_KT;
+    prep::decay_and_tiles(reinterpret_cast<const uint16_t *>(base + A_STQ),
+                          reinterpret_cast<const uint16_t *>(base + A_STK),
+                          reinterpret_cast<const float *>(base + A_STG), valid_sh, t, part_sh,
+                          decay_sh, beta_st, beta_sh, tid);
+    fence_async_smem();
+    __syncthreads();
+    // ---- Gram: [Q G ; K G] (K e^{-g})^T
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t id = idesc_bf16(128, 64, 0, 0);
+      const uint32_t sQKW = smem_u32(base + A_QKW), sKH = smem_u32(base + A_KH);
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(tm + A_TM_G, desc_kmajor(sQKW, 192, 64, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
+      mma_commit(&mma_bar);
+    }
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    phase++;
+  }
+  if (ok) {
+    fence_after_sync();
+    float *As = reinterpret_cast<float *>(base + A_AS);
+    float *Ts = reinterpret_cast<float *>(base + A_TS);
+    float *Xs = reinterpret_cast<float *>(base + A_XS);
+    prep::extract_gram(tm + my_cols + A_TM_G, base + A_TBM, 192, 128, As, beta_sh, tid);
+    __syncthreads();
+    tri::unit_lower_inverse_64(As, Ts, Xs, tid);
+    prep::pack_tb(Ts, beta_sh, base + A_TBM, 192, tid);
+    fence_async_smem();
+    __syncthreads();
+    // ---- W^T = (K G)^T T_b^T ;  [U_v ; 0] = [T_b ; 0] V   (N = 128: all of d_v)
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t sQKW = smem_u32(base + A_QKW), sTBM = smem_u32(base + A_TBM);
+      const uint32_t sV = smem_u32(base + A_V);
+      const uint32_t idw = idesc_bf16(128, 64, 1, 0);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tm + A_TM_W, desc_mnmajor(sQKW, 192, 128, s), desc_kmajor(sTBM, 192, 0, s), idw, s > 0);
+      const uint32_t idu = idesc_bf16(128, 128, 0, 1);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tm + A_TM_UV, desc_kmajor(sTBM, 192, 0, s), desc_mnmajor(sV, 64, 0, s), idu, s > 0);
+      mma_commit(&mma_bar);
+    }
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    phase++;
+  }
+  if (ok) {
+    fence_after_sync();
+    // -W into rows 0..63 of the [-W | Q G | K G] tile (lane = key channel)
+    {
+      float v[32];
+      tmem_ld32(tm + my_cols + A_TM_W, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        *reinterpret_cast<__nv_bfloat16 *>(base + A_QKW + row_tile_off(wg * 32 + j, lr, 192)) =
+            __float2bfloat16_rn(-v[j]);
+    }
+    // U_v rows (lanes 0-63): columns 64 wg .. 64 wg + 63 -> block wg of the U_v tile
+    if ((warp & 3) < 2) {
+      float v[32];
+      const uint32_t col = lane_base + A_TM_UV + (uint32_t)(wg * 64);
+      tmem_ld32(tm + col, v);
+      prep::store_row32(base + A_UV + wg * 64 * 128, 64, lr, 0, v);
+      tmem_ld32(tm + col + 32, v);
+      prep::store_row32(base + A_UV + wg * 64 * 128, 64, lr, 4, v);
+    }
+    fence_async_smem();
+    __syncthreads();
+    // ---- bulk stores of the item
+    if (tid == 0) {
+      unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
+      bulk_store(it + IT_WQ, base + A_QKW, 128 * 128);                       // block 0 rows 0..127
+      bulk_store(it + IT_WQ + 128 * 128, base + A_QKW + 192 * 128, 128 * 128);  // block 1 rows 0..127
+      bulk_store(it + IT_KT, base + A_KT, 64 * 256);
+      bulk_store(it + IT_UV, base + A_UV, 64 * 256);
+      bulk_store(it + IT_M, base + A_TBM + 128 * 128, 64 * 128);
+      bulk_store(it + IT_GC, decay_sh, kDK * 4);
+      bulk_commit();
+      bulk_wait_read();
+    }
+  }
+  if (!ok) {
+    if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
+    // let whatever timed out (the staging loads or a product) finish, bounded
+    mbar_wait(&stage_bar, 0, kWaitCycles);
+    if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after_sync();
+    tmem_dealloc(tm, A_TM_COLS);
+  }
+}
+
+// ============================================================ state pass (B)
+constexpr int kThreadsB = 128;
+constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
+constexpr uint32_t BUF_BYTES = 66560;
+constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
+constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES, B_UB = B_SB + 128 * 128;
+constexpr uint32_t B_USED = B_UB + 64 * 128;
+constexpr uint32_t B_SMEM = B_USED + 1024;
+constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 128;
+
+__device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int tile,
+                                          uint64_t *bar) {
+  mbar_arrive_expect_tx(bar, BUF_TX);
+  bulk_load(buf + BUF_WQ, it + IT_WQ, 32768, bar);
+  bulk_load(buf + BUF_KT, it + IT_KT, 16384, bar);
+  bulk_load(buf + BUF_UV, it + IT_UV + tile * 8192, 8192, bar);
+  bulk_load(buf + BUF_M, it + IT_M, 8192, bar);
+  bulk_load(buf + BUF_GC, it + IT_GC, 512, bar);
+}
+
+__global__ void __launch_bounds__(kThreadsB, 1)
+state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsigned char *items) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ __align__(8) uint64_t load_bar[2];
+
+  if (device_error_latched(p.err)) return;
+  const int tiles = p.dv / kNV;
+  const int tile = blockIdx.x % tiles;
+  const int h = (blockIdx.x / tiles) % p.H;
+  const int b = blockIdx.x / (tiles * p.H);
+  const int dv0 = tile * kNV;
+  const int H = p.H, DV = p.dv;
+  const SeqSpan sp = spans[b];
+  const int nch = (sp.end - sp.begin + kC - 1) / kC;
+  const int cb = cbase[b];
+
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char *base = smem_raw + pad;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  if (warp == 0) tmem_alloc(&tmem_base_sh, B_TM_COLS);
+  if (tid == 0) {
+    mbar_init(&mma_bar, 1);
+    mbar_init(&load_bar[0], 1);
+    mbar_init(&load_bar[1], 1);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = tmem_base_sh;
+  {   // initial state: thread owns state row tid (64 columns)
+    float v[32];
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32 + j] : 0.f;
+      tmem_st32(tm + lane_base + B_TM_S + half * 32, v);
+    }
+    tmem_st_wait();
+  }
+  if (tid == 0) {
+    for (int j = 0; j < 2 && j < nch; ++j)
+      load_item(base + (j ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES, tile,
+                &load_bar[j]);
+  }
+  const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
+  uint32_t phase = 0;
+  bool ok = true;
+  int loads_issued = nch < 2 ? nch : 2;   // item loads issued so far (thread 0's view)
+  int loads_waited = 0;
+
+  for (int j = 0; j < nch; ++j) {
+    const int c0 = sp.begin + j * kC;
+    unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
+    const uint32_t sbuf = smem_u32(buf);
+    ok = __syncthreads_and(mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles));
+    if (!ok) break;
+    loads_waited = j + 1;
+    // ---- S -> bf16 operand; S *= e^{g_C}
+    {
+      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[tid];
+      float v[32];
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tm + lane_base + B_TM_S + half * 32, v);
+        prep::store_row32(base + B_SB, 128, tid, half * 4, v);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
+        tmem_st32(tm + lane_base + B_TM_S + half * 32, v);
+      }
+      tmem_st_wait();
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    // ---- [-W S ; (Q G) S] = [-W ; Q G] S
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t id = idesc_bf16(128, 64, 0, 1);
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(tm + B_TM_D1, desc_kmajor(sbuf + BUF_WQ, 128, 0, s), desc_mnmajor(sSB, 128, 0, s), id, s > 0);
+      mma_commit(&mma_bar);
+    }
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    phase++;
+    if (!ok) break;
+    fence_after_sync();
+    // ---- U = U_v - W S (lanes 0-63) -> bf16 operand
+    if (warp < 2) {
+      const int r = tid;
+      float v[32];
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tm + lane_base + B_TM_D1 + half * 32, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, half * 4 + q, kC));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
+            v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+          }
+        }
+        prep::store_row32(base + B_UB, 64, r, half * 4, v);
+      }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t ido = idesc_bf16(128, 64, 0, 1);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tm + B_TM_D1, desc_kmajor(sbuf + BUF_UV, 128, 0, s), desc_mnmajor(sUB, 64, 0, s), ido, 1);
+      const uint32_t ids = idesc_bf16(128, 64, 1, 1);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tm + B_TM_S, desc_mnmajor(sbuf + BUF_KT, 64, 0, s), desc_mnmajor(sUB, 64, 0, s), ids, 1);
+      mma_commit(&mma_bar);
+    }
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    phase++;
+    if (!ok) break;
+    fence_after_sync();
+    // ---- O (lanes 64-127) -> global
+    if (warp >= 2) {
+      const int r = tid - kC;
+      const int pos = c0 + r;
+      float v[32];
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tm + lane_base + B_TM_D1 + half * 32, v);
+        if (pos < sp.end) {
+          const bool valid = p.mask == nullptr || p.mask[pos] != 0;
+          uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + half * 32;
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 8) {
+            uint4 pk;
+            pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
+            pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
+            pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
+            pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
+            *reinterpret_cast<uint4 *>(orow + jj) = pk;
+          }
+        }
+      }
+    }
+    fence_before_sync();
+    __syncthreads();
+    // this buffer is free: stream chunk j + 2 into it
+    if (j + 2 < nch) {
+      if (tid == 0)
+        load_item(buf, items + ((size_t)(cb + j + 2) * H + h) * ITEM_BYTES, tile, &load_bar[j & 1]);
+      loads_issued = j + 3;
+    }
+  }
+
+  if (!ok) {
+    if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
+    mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+  } else if (p.final_state) {
+    float v[32];
+    for (int half = 0; half < 2; ++half) {
+      tmem_ld32(tm + lane_base + B_TM_S + half * 32, v);
+      float *dst = p.final_state + (((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32;
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 4)
+        *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+    }
+  }
+  // item loads still in flight after a timeout land (bounded) before the CTA exits
+  for (int jj = loads_waited; jj < loads_issued; ++jj)
+    mbar_wait(&load_bar[jj & 1], (jj >> 1) & 1, kWaitCycles);
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after_sync();
+    tmem_dealloc(tm, B_TM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool encode_3d(CUtensorMap *map, CUtensorMapDataType dt, size_t esize, const void *ptr, int inner,
+               int H, int N, int box_inner, CUtensorMapSwizzle swz) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)(N > 0 ? N : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * H};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, 64u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace split
+
+bool prefill_split_supported(const PrefillParams &p, bool bf16) {
+  return bf16 && p.dk == split::kDK && p.dv == 128 && p.chunk == split::kC;
+}
+
+size_t prefill_split_workspace(int N, int B, int H) { return split::ws_total(N, B, H); }
+
+// spans: B entries already written by the pre-pass; ws: workspace base.
+cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s) {
+  using namespace split;
+  if (p.num_seqs == 0) return cudaSuccess;
+  unsigned char *w = static_cast<unsigned char *>(ws);
+  int *cbase = reinterpret_cast<int *>(w + ws_cbase_off(p.num_seqs));
+  unsigned char *items = w + ws_items_off(p.num_seqs);
+  chunk_index_kernel<<<1, 1024, 0, s>>>(p, spans, cbase);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  IntraMaps maps;
+  if (!encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
+  e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
+  if (e != cudaSuccess) return e;
+  const size_t gridA = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
+  if (gridA > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+  intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, maps, spans, cbase, items);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / kNV);
+  state_kernel<<<gridB, kThreadsB, B_SMEM, s>>>(p, spans, cbase, items);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

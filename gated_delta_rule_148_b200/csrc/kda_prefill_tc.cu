@@ -36,9 +36,12 @@
 // such limit).
 #include <climits>
 
+#include <cudaTypedefs.h>
+
 #include "kda_internal.cuh"
 #include "kda_tc.cuh"
 #include "kda_tril_inv.cuh"
+#include "kda_chunk_prep.cuh"
 
 namespace kda {
 namespace {
@@ -90,72 +93,53 @@ __device__ __forceinline__ bool row_valid(const PrefillParams &p, const SeqSpan 
   return pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
 }
 
-// Stage q, k, log_alpha (and beta) of the chunk starting at c0 with cp.async;
-// invalid rows are zero-filled without reading global memory.
-__device__ __forceinline__ void stage_chunk(const PrefillParams &p, const SeqSpan &sp, int c0,
-                                            int h, unsigned char *base, int tid) {
-  const int H = p.H;
-  const uint32_t sq = smem_u32(base + OFF_STQ), sk = smem_u32(base + OFF_STK);
-  const uint32_t sg = smem_u32(base + OFF_STG);
-  for (int e = tid; e < kC * 16; e += kThreads) {       // q, k: 64 rows x 16 x 16 B
-    const int r = e >> 4, ch = e & 15;
-    const int pos = c0 + r;
-    const bool ok = row_valid(p, sp, pos);
-    const size_t gi = ((size_t)(ok ? pos : 0) * H + h) * kDK + ch * 8;
-    cp_async16(sq + r * 256 + ch * 16, (const uint16_t *)p.q + gi, ok ? 16u : 0u);
-    cp_async16(sk + r * 256 + ch * 16, (const uint16_t *)p.k + gi, ok ? 16u : 0u);
-  }
-  for (int e = tid; e < kC * 32; e += kThreads) {       // log_alpha: 64 rows x 32 x 16 B
-    const int r = e >> 5, ch = e & 31;
-    const int pos = c0 + r;
-    const bool ok = row_valid(p, sp, pos);
-    const size_t gi = ((size_t)(ok ? pos : 0) * H + h) * kDK + ch * 4;
-    cp_async16(sg + r * 512 + ch * 16, p.log_alpha + gi, ok ? 16u : 0u);
+// Tensor maps of the inputs (built on the host for each call).
+struct TmaMaps {
+  CUtensorMap q, k, la;   // [N, H, 128] boxes {128, 1, 64}, no swizzle (staging rows)
+  CUtensorMap v;          // [N, H, dv]  boxes {64, 1, 64}, 128-byte swizzle (MMA operand tile)
+};
+
+constexpr uint32_t kStageBytes = 64 * 256 * 2 + 64 * 512;   // q + k + log_alpha of one chunk
+constexpr uint32_t kVBytes = 64 * 128;
+
+// Issue the TMA loads of q, k, log_alpha for the chunk starting at packed row c0
+// (one thread), and load beta (threads 0..63; invalid rows get 0).
+__device__ __forceinline__ void stage_chunk(const PrefillParams &p, const TmaMaps &m,
+                                            const SeqSpan &sp, int c0, int h, unsigned char *base,
+                                            uint64_t *bar, int tid) {
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, kStageBytes);
+    tma_load_3d(smem_u32(base + OFF_STQ), &m.q, 0, h, c0, bar);
+    tma_load_3d(smem_u32(base + OFF_STK), &m.k, 0, h, c0, bar);
+    tma_load_3d(smem_u32(base + OFF_STG), &m.la, 0, h, c0, bar);
   }
   if (tid < kC) {
     const int pos = c0 + tid;
     float *sb = reinterpret_cast<float *>(base + OFF_STB);
-    sb[tid] = row_valid(p, sp, pos) ? p.beta[(size_t)pos * H + h] : 0.f;
+    sb[tid] = row_valid(p, sp, pos) ? p.beta[(size_t)pos * p.H + h] : 0.f;
   }
 }
 
-// V slice (64 rows x 64 columns) into the MN-major V tile.
-__device__ __forceinline__ void stage_v(const PrefillParams &p, const SeqSpan &sp, int c0, int h,
-                                        int dv0, unsigned char *base, int tid) {
-  const uint32_t sv = smem_u32(base + OFF_V);
-  for (int e = tid; e < kC * 8; e += kThreads) {
-    const int r = e >> 3, ch = e & 7;
-    const int pos = c0 + r;
-    const bool ok = row_valid(p, sp, pos);
-    const size_t gi = ((size_t)(ok ? pos : 0) * p.H + h) * p.dv + dv0 + ch * 8;
-    cp_async16(sv + row_tile_chunk(r, 0, ch, kC), (const uint16_t *)p.v + gi, ok ? 16u : 0u);
+// TMA load of the V slice (64 rows x 64 columns) straight into its MMA tile.
+__device__ __forceinline__ void stage_v(const TmaMaps &m, int c0, int h, int dv0,
+                                        unsigned char *base, uint64_t *bar, int tid) {
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, kVBytes);
+    tma_load_3d(smem_u32(base + OFF_V), &m.v, dv0, h, c0, bar);
   }
 }
 
-__device__ __forceinline__ void st_u32(unsigned char *tile, uint32_t off, uint32_t x) {
-  *reinterpret_cast<uint32_t *>(tile + off) = x;
-}
-
-// 32 fp32 values -> bf16 into 4 consecutive 16-byte chunks (c0..c0+3) of row r.
-__device__ __forceinline__ void store_row32(unsigned char *tile, int R, int r, int chunk0,
-                                            const float *v) {
-#pragma unroll
-  for (int j = 0; j < 32; j += 8) {
-    uint4 pk;
-    pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
-    pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
-    pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
-    pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-    *reinterpret_cast<uint4 *>(tile + row_tile_chunk(r, 0, chunk0 + (j >> 3), R)) = pk;
-  }
-}
+using prep::store_row32;
 
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(PrefillParams p) {
+prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
-  __shared__ float gC_sh[kDK];
+  __shared__ __align__(8) uint64_t stage_bar;
+  __shared__ __align__(8) uint64_t v_bar;
+  __shared__ uint32_t valid_sh[2];      // validity bits of the chunk's 64 rows
+  __shared__ float decay_sh[kDK];      // e^{g_C} per key channel
   __shared__ float beta_sh[kC];
   __shared__ float part_sh[4][kDK];
 
@@ -178,7 +162,11 @@ prefill_tc_kernel(PrefillParams p) {
 
   // ---- set-up: TMEM, barrier, zero rows of [T_b | 0 | M]
   if (warp == 0) tmem_alloc(&tmem_base_sh, TM_COLS);
-  if (tid == 0) mbar_init(&mma_bar, 1);
+  if (tid == 0) {
+    mbar_init(&mma_bar, 1);
+    mbar_init(&stage_bar, 1);
+    mbar_init(&v_bar, 1);
+  }
   for (int e = tid; e < 64 * 8; e += kThreads) {
     const int r = 64 + (e >> 3), ch = e & 7;
     *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(r, 0, ch, 192)) = make_uint4(0, 0, 0, 0);
@@ -210,64 +198,30 @@ prefill_tc_kernel(PrefillParams p) {
   const float *stb = reinterpret_cast<const float *>(base + OFF_STB);
 
   if (sp.begin < sp.end) {
-    stage_chunk(p, sp, sp.begin, h, base, tid);
-    stage_v(p, sp, sp.begin, h, dv0, base, tid);
-    cp_async_commit();
+    stage_chunk(p, maps, sp, sp.begin, h, base, &stage_bar, tid);
+    stage_v(maps, sp.begin, h, dv0, base, &v_bar, tid);
   }
+  uint32_t chunk_idx = 0;
 
-  for (int c0 = sp.begin; c0 < sp.end; c0 += kC) {
-    cp_async_wait_all();
-    __syncthreads();
-    // ---- P1: cumsum and operand tiles.  Thread: channels 2cp, 2cp+1; rows 16qt..16qt+15
+  for (int c0 = sp.begin; c0 < sp.end; c0 += kC, ++chunk_idx) {
+    // validity of the chunk's rows (tail rows and pads enter as identity steps)
+    if (tid < kC) {
+      const unsigned bits = __ballot_sync(0xFFFFFFFFu, row_valid(p, sp, c0 + tid));
+      if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
+    }
+    ok = __syncthreads_and(mbar_wait(&stage_bar, chunk_idx & 1, kWaitCycles));
+    if (!ok) break;
+    // ---- P1: decay products and operand tiles
     {
-      const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
-      const float *sg = reinterpret_cast<const float *>(base + OFF_STG);
-      float g0[16], g1[16];
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float2 la = *reinterpret_cast<const float2 *>(sg + (qt * 16 + i) * kDK + c);
-        s0 += la.x;
-        s1 += la.y;
-        g0[i] = s0;
-        g1[i] = s1;
-      }
-      part_sh[qt][c] = s0;
-      part_sh[qt][c + 1] = s1;
-      if (tid < kC) beta_sh[tid] = stb[tid];
-      __syncthreads();
-      float off0 = 0.f, off1 = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q < qt) {
-          off0 += part_sh[q][c];
-          off1 += part_sh[q][c + 1];
-        }
-      }
-      const float gC0 = part_sh[0][c] + part_sh[1][c] + part_sh[2][c] + part_sh[3][c];
-      const float gC1 = part_sh[0][c + 1] + part_sh[1][c + 1] + part_sh[2][c + 1] + part_sh[3][c + 1];
-      if (qt == 0) {
-        gC_sh[c] = gC0;
-        gC_sh[c + 1] = gC1;
-      }
-      const float en0 = __expf(fminf(-gC0, 80.f)), en1 = __expf(fminf(-gC1, 80.f));
-      const uint32_t *sq = reinterpret_cast<const uint32_t *>(base + OFF_STQ);
-      const uint32_t *sk = reinterpret_cast<const uint32_t *>(base + OFF_STK);
-#pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
-        const int r = qt * 16 + i;
-        const float ga = g0[i] + off0, gb = g1[i] + off1;
-        const uint32_t qq = sq[r * 64 + cp], kk = sk[r * 64 + cp];
-        const float qa = __uint_as_float(qq << 16), qb = __uint_as_float(qq & 0xFFFF0000u);
-        const float ka = __uint_as_float(kk << 16), kb = __uint_as_float(kk & 0xFFFF0000u);
-        const float e1a = __expf(ga), e1b = __expf(gb);              // e^{g}       <= 1
-        const float e2a = __expf(gC0 - ga), e2b = __expf(gC1 - gb);  // e^{g_C - g} <= 1
-        const float e3a = e2a * en0, e3b = e2b * en1;                // e^{-g}
-        st_u32(base + OFF_QKW, row_tile_off(64 + r, c, 192), pack_bf16x2(qa * e1a, qb * e1b));
-        st_u32(base + OFF_QKW, row_tile_off(128 + r, c, 192), pack_bf16x2(ka * e1a, kb * e1b));
-        st_u32(base + OFF_KH, row_tile_off(r, c, 64), pack_bf16x2(ka * e3a, kb * e3b));
-        st_u32(base + OFF_KT, row_tile_off(r, c, 64), pack_bf16x2(ka * e2a, kb * e2b));
-      }
+      prep::PrepTiles t;
+      t.qg = base + OFF_QKW; t.qg_R = 192; t.qg_row0 = 64;
+      t.kg = base + OFF_QKW; t.kg_R = 192; t.kg_row0 = 128;
+      t.kh = base + OFF_KH;
+      t.kt = base + OFF_KT;
+      prep::decay_and_tiles(reinterpret_cast<const uint16_t *>(base + OFF_STQ),
+                            reinterpret_cast<const uint16_t *>(base + OFF_STK),
+                            reinterpret_cast<const float *>(base + OFF_STG), valid_sh, t, part_sh,
+                            decay_sh, stb, beta_sh, tid);
     }
     fence_async_smem();
     __syncthreads();
@@ -284,51 +238,26 @@ prefill_tc_kernel(PrefillParams p) {
     if (!ok) break;
     fence_after_sync();
     // ---- P3: M rows (lanes 0-63) -> TBM rows 128..191; beta * A rows (lanes 64-127) -> As
-    {
-      float v[32];
-      tmem_ld32(tm + my_cols + TM_G, v);
-      if (lr < kC) {
-        const int r = lr;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = (wg * 32 + j <= r) ? v[j] : 0.f;
-        store_row32(base + OFF_TBM, 192, 128 + r, wg * 4, v);
-      } else {
-        const int r = lr - kC;
-        const float br = beta_sh[r];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = wg * 32 + j;
-          As[r * 65 + i] = (i < r) ? br * v[j] : 0.f;
-        }
-      }
-    }
+    prep::extract_gram(tm + my_cols + TM_G, base + OFF_TBM, 192, 128, As, beta_sh, tid);
     __syncthreads();
     // ---- P4: T = (I + A)^{-1};  T_b = T Diag(beta) -> TBM rows 0..63
     tri::unit_lower_inverse_64(As, Ts, Xs, tid);
-    {
-      const int r = tid >> 2, qq = tid & 3;      // row r, columns 16qq .. 16qq+15
-      float t[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = qq * 16 + u;
-        t[u] = (i <= r) ? Ts[r * 65 + i] * beta_sh[i] : 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < 16; j += 8) {
-        uint4 pk;
-        pk.x = pack_bf16x2(t[j + 0], t[j + 1]);
-        pk.y = pack_bf16x2(t[j + 2], t[j + 3]);
-        pk.z = pack_bf16x2(t[j + 4], t[j + 5]);
-        pk.w = pack_bf16x2(t[j + 6], t[j + 7]);
-        *reinterpret_cast<uint4 *>(base + OFF_TBM + row_tile_chunk(r, 0, (qq * 16 + j) >> 3, 192)) = pk;
-      }
-    }
+    prep::pack_tb(Ts, beta_sh, base + OFF_TBM, 192, tid);
     fence_async_smem();
     __syncthreads();
     // the staging buffers are free: stream the next chunk's q, k, log_alpha, beta
-    if (c0 + kC < sp.end) {
-      stage_chunk(p, sp, c0 + kC, h, base, tid);
-      cp_async_commit();
+    if (c0 + kC < sp.end) stage_chunk(p, maps, sp, c0 + kC, h, base, &stage_bar, tid);
+    // V of this chunk must have landed; zero its invalid rows
+    ok = __syncthreads_and(mbar_wait(&v_bar, chunk_idx & 1, kWaitCycles));
+    if (!ok) break;
+    if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
+      for (int e = tid; e < kC * 8; e += kThreads) {
+        const int r = e >> 3, ch = e & 7;
+        if (!((valid_sh[r >> 5] >> (r & 31)) & 1u))
+          *reinterpret_cast<uint4 *>(base + OFF_V + row_tile_chunk(r, 0, ch, kC)) = make_uint4(0, 0, 0, 0);
+      }
+      fence_async_smem();
+      __syncthreads();
     }
     // ---- W^T = (K G)^T T_b^T ;  [U_v ; 0] = [T_b ; 0] V
     if (tid == 0) {
@@ -352,11 +281,11 @@ prefill_tc_kernel(PrefillParams p) {
       tmem_ld32(tm + my_cols + TM_W, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        *reinterpret_cast<uint16_t *>(base + OFF_QKW + row_tile_off(wg * 32 + j, c, 192)) =
-            f32_to_bf16_rne(-v[j]);
+        *reinterpret_cast<__nv_bfloat16 *>(base + OFF_QKW + row_tile_off(wg * 32 + j, c, 192)) =
+            __float2bfloat16_rn(-v[j]);
       tmem_ld32(tm + my_cols + TM_S, v);
       store_row32(base + OFF_SB, 128, c, wg * 4, v);
-      const float decay = __expf(gC_sh[c]);
+      const float decay = decay_sh[c];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] *= decay;
       tmem_st32(tm + my_cols + TM_S, v);
@@ -365,10 +294,7 @@ prefill_tc_kernel(PrefillParams p) {
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
-    if (c0 + kC < sp.end) {        // the U_v product that read V is complete
-      stage_v(p, sp, c0 + kC, h, dv0, base, tid);
-      cp_async_commit();
-    }
+    if (c0 + kC < sp.end) stage_v(maps, c0 + kC, h, dv0, base, &v_bar, tid);   // U_v read V
     // ---- [U ; (Q G) S] += [-W ; Q G] S
     if (tid == 0) {
       fence_after_sync();
@@ -441,7 +367,6 @@ prefill_tc_kernel(PrefillParams p) {
     for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
   }
-  cp_async_wait_all();
   fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -456,13 +381,51 @@ bool prefill_tc_supported(const PrefillParams &p, bool bf16) {
   return bf16 && p.dk == kDK && (p.dv % kNV) == 0 && p.chunk == kC;
 }
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool encode_3d(CUtensorMap *map, CUtensorMapDataType dt, size_t esize, const void *ptr, int inner,
+               int H, int N, int box_inner, CUtensorMapSwizzle swz) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)(N > 0 ? N : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * H};
+  const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, 64u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t s) {
   if (p.num_seqs == 0) return cudaSuccess;
+  TmaMaps maps;
+  if (!encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.num_seqs * p.H * (p.dv / kNV);
-  prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(p);
+  prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(p, maps);
   return cudaGetLastError();
 }
 

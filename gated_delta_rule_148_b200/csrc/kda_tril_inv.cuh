@@ -77,22 +77,25 @@ __device__ __forceinline__ void store_acc(float *Z, int ldz, const float (&acc)[
 }
 
 // scratch: 8 warps x 16 x 17 floats.  Must be called by all 256 threads.
-__device__ __forceinline__ void unit_lower_inverse_64(const float *As, float *Ts, float *scratch,
-                                                      int tid) {
+__device__ __forceinline__ void unit_lower_inverse_64(const float *__restrict__ As,
+                                                      float *__restrict__ Ts,
+                                                      float *__restrict__ scratch, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  // ---- diagonal blocks: thread (blk, j) holds column j of D_blk in registers
+  // ---- diagonal blocks: thread (blk, j) holds column j of D_blk in registers.
+  // Right-looking: once t[i] is known it is folded into every later row, so
+  // the dependency depth is 16 steps rather than 120 sequential FMAs.
   if (tid < 64) {
     const int blk = tid >> 4, j = tid & 15, o = blk * 16;
-    float t[16];
+    float acc[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
 #pragma unroll
-      for (int i = 0; i < r; ++i) acc = fmaf(As[(o + r) * LD + o + i], t[i], acc);
-      t[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
+    for (int i = 0; i < 16; ++i) {
+      const float ti = (i < j) ? 0.f : (i == j ? 1.f : -acc[i]);
+      Ts[(o + i) * LD + o + j] = ti;
+#pragma unroll
+      for (int r = i + 1; r < 16; ++r) acc[r] = fmaf(As[(o + r) * LD + o + i], ti, acc[r]);
     }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Ts[(o + r) * LD + o + j] = t[r];
   }
   __syncthreads();
   // ---- off-diagonal blocks by distance

@@ -181,10 +181,15 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     _check_cuda("final_state", final_state, torch.float32, (B, H, dk, dv))
-    if pad_mask is not None and workspace is None:
-        workspace = torch.empty(prefill_workspace_bytes(B), dtype=torch.uint8, device=q.device)
     a = prefill_args(q, k, v, log_alpha, beta, cu_seqlens, pad_mask, init_state, o, final_state,
                      chunk, workspace)
+    if workspace is None:
+        # the library states its own need (span table; per-chunk items of the two-kernel path)
+        nbytes = int(lib.kda_prefill_workspace_size(ctypes.byref(a)))
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+            a.workspace = _ptr(workspace)
+            a.workspace_bytes = nbytes
     st = lib.kda_prefill(ctypes.byref(a), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_prefill")

@@ -87,8 +87,13 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  *   chunk        0 (default: 64 for bf16, 16 for fp32), 16, 32 or 64.  The
  *                result is defined by the recurrence and does not depend on the
  *                chunk size beyond rounding.
- *   workspace    device scratch of kda_prefill_workspace_size() bytes,
- *                256-byte aligned; may be NULL only when pad_mask is NULL.
+ *   workspace    device scratch, 256-byte aligned.  kda_prefill_workspace_size()
+ *                bytes select the fastest path (for bf16, d_k = d_v = 128,
+ *                chunk 64: a two-kernel path that stores each chunk's
+ *                intermediate tiles, about 73 KB per 64 tokens and head).  A
+ *                smaller workspace selects a fused single-kernel path; a pad
+ *                mask needs at least 16 bytes per sequence (rounded up to 256).
+ *                May be NULL when pad_mask is NULL.
  * Numerics: bf16 inputs take the tensor-core path (bf16 operands, fp32
  * accumulation, fp32 state); fp32 inputs take an fp32 CUDA-core path.  o is
  * rounded once (round to nearest even) to its dtype.
@@ -115,8 +120,8 @@ typedef struct {
   size_t workspace_bytes;
 } kda_prefill_args;
 
-/* Bytes of workspace kda_prefill() needs for these arguments (reads only the
- * sizes).  Returns 0 if args is NULL. */
+/* Bytes of workspace for the fastest path of kda_prefill() with these
+ * arguments (reads only dtype, sizes and chunk).  Returns 0 if args is NULL. */
 size_t kda_prefill_workspace_size(const kda_prefill_args *args);
 
 /* Enqueue one prefill.  Returns KDA_OK or an argument/launch error. */
