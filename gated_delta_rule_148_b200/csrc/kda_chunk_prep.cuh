@@ -111,6 +111,94 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
   }
 }
 
+// P1 reading q, k, log_alpha straight from global memory (rows of the chunk at
+// packed positions c0 .. c0+63 of head h; invalid rows count as zero).  Besides the
+// shared tiles (Q G and K G rows of `t.qg/t.kg`, K e^{-g} in `t.kh`), it writes
+// Q G into rows 64.. of the 128-row output tile `gq` and K e^{g_C - g} into the
+// 64-row output tile `gkt` (global memory, same swizzled layout), and e^{g_C} into
+// `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
+__device__ __forceinline__ void decay_and_tiles_global(
+    const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
+    const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
+    float *gdecay, float (*part)[kDK], float *decay, int tid) {
+  const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
+  const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
+  float a0[16], a1[16];
+  uint32_t qv[16], kv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool vr = (vbits >> i) & 1u;
+    const size_t row = ((size_t)(c0 + qt * 16 + i) * H + h) * kDK + c;
+    float2 la = make_float2(0.f, 0.f);
+    qv[i] = 0u;
+    kv[i] = 0u;
+    if (vr) {
+      la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
+      qv[i] = __ldg(reinterpret_cast<const unsigned int *>(q + row));
+      kv[i] = __ldg(reinterpret_cast<const unsigned int *>(k + row));
+    }
+    a0[i] = la.x;
+    a1[i] = la.y;
+  }
+  float t0 = 1.f, t1 = 1.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    a0[i] = __expf(a0[i]);
+    a1[i] = __expf(a1[i]);
+    t0 *= a0[i];
+    t1 *= a1[i];
+  }
+  part[qt][c] = t0;
+  part[qt][c + 1] = t1;
+  __syncthreads();
+  float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    const float x0 = part[qq][c], x1 = part[qq][c + 1];
+    if (qq < qt) { pre0 *= x0; pre1 *= x1; }
+    if (qq > qt) { suf0 *= x0; suf1 *= x1; }
+  }
+  const float GC0 = pre0 * t0 * suf0, GC1 = pre1 * t1 * suf1;   // e^{g_C}
+  if (qt == 0) {
+    decay[c] = GC0;
+    decay[c + 1] = GC1;
+    *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
+  }
+  const float inv0 = GC0 > 1e-35f ? 1.f / GC0 : 1e35f, inv1 = GC1 > 1e-35f ? 1.f / GC1 : 1e35f;
+  const int kb = c >> 6, ch = (c & 63) >> 3;
+  const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
+  const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
+  const uint32_t col128 = (uint32_t)(kb * 128 * 128 + (c & 7) * 2);
+  const uint32_t col64 = (uint32_t)(kb * 64 * 128 + (c & 7) * 2);
+  float e0 = pre0, e1 = pre1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = qt * 16 + i;
+    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
+    const float qa = __uint_as_float(qv[i] << 16), qb = __uint_as_float(qv[i] & 0xFFFF0000u);
+    const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
+    e0 *= a0[i];
+    e1 *= a1[i];
+    const uint32_t qgv = pack_bf16x2(qa * e0, qb * e1);
+    *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
+    *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
+    *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
+        pack_bf16x2(ka * e0, kb2 * e1);
+  }
+  float s0 = suf0, s1 = suf1;
+#pragma unroll
+  for (int i = 15; i >= 0; --i) {
+    const int r = qt * 16 + i;
+    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
+    const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
+    const uint32_t rr = (uint32_t)(r * 128) + sw;
+    *reinterpret_cast<uint32_t *>(gkt + col64 + rr) = pack_bf16x2(ka * s0, kb2 * s1);
+    *reinterpret_cast<uint32_t *>(t.kh + col64 + rr) = pack_bf16x2(ka * (s0 * inv0), kb2 * (s1 * inv1));
+    s0 *= a0[i];
+    s1 *= a1[i];
+  }
+}
+
 // 32 fp32 values -> bf16 into 4 consecutive 16-byte chunks (chunk0..chunk0+3) of row r
 // of a K-major row tile with R rows and one 64-column block.
 __device__ __forceinline__ void store_row32(unsigned char *tile, int R, int r, int chunk0,

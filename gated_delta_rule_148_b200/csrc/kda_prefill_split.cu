@@ -92,45 +92,37 @@ __global__ void __launch_bounds__(1024) chunk_index_kernel(PrefillParams p, cons
 }
 
 // ============================================================ intra kernel (A)
-struct IntraMaps {
-  CUtensorMap q, k, la;   // [N, H, 128] boxes {128, 1, 64}
-  CUtensorMap v;          // [N, H, dv] boxes {64, 1, 64}, 128-byte swizzle
-};
-
+// One CTA per (chunk, head); ~100 KB of shared memory so two CTAs share an SM
+// and hide each other's load and tensor-core latency.  q, k, log_alpha are read
+// straight from global memory; V arrives by TMA; every output goes straight to
+// the workspace item.
 constexpr int kThreadsA = 256;
-constexpr uint32_t A_QKW = 0;                       // [-W | Q G | K G] 192 x 128
-constexpr uint32_t A_KH = A_QKW + 192 * 256;        // K e^{-g}       64 x 128
-constexpr uint32_t A_KT = A_KH + 64 * 256;          // K e^{g_C - g}  64 x 128
-constexpr uint32_t A_TBM = A_KT + 64 * 256;         // [T_b | 0 | M]  192 x 64
-constexpr uint32_t A_V = A_TBM + 192 * 128;         // V  64 rows x 2 blocks of 64
-constexpr uint32_t A_UV = A_V + 64 * 256;           // U_v 64 rows x 2 blocks of 64
-constexpr uint32_t A_STQ = A_UV + 64 * 256;         // staging q [64][128] bf16
-constexpr uint32_t A_STK = A_STQ + 64 * 256;        // staging k
-constexpr uint32_t A_STG = A_STK + 64 * 256;        // staging log_alpha [64][128] f32
-constexpr uint32_t A_AS = A_STQ;                    // A [64][65] f32 (aliases staging)
-constexpr uint32_t A_XS = A_AS + 64 * 65 * 4;       // inverse scratch
-constexpr uint32_t A_TS = A_STG;                    // T [64][65] f32
-constexpr uint32_t A_USED = A_STG + 64 * 512;
+constexpr uint32_t A_QK = 0;                        // [Q G | K G]   128 x 128 row tile
+constexpr uint32_t A_KH = A_QK + 128 * 256;         // K e^{-g} 64 x 128 (then A [64][65] f32)
+constexpr uint32_t A_TB = A_KH + 17 * 1024;         // [T_b | 0]     128 x 64 row tile
+constexpr uint32_t A_V = A_TB + 128 * 128;          // V  64 rows x 2 blocks of 64
+constexpr uint32_t A_TS = A_V + 64 * 256;           // T  [64][65] f32
+constexpr uint32_t A_XS = A_TS + 64 * 65 * 4;       // inverse scratch (3 warps x 16 x 17)
+constexpr uint32_t A_USED = A_XS + 3 * 16 * 17 * 4;
 constexpr uint32_t A_SMEM = A_USED + 1024;
-static_assert(A_XS + 8 * 16 * 17 * 4 <= A_STG, "scratch fits the q/k staging");
-constexpr uint32_t A_TM_G = 0, A_TM_W = 64, A_TM_UV = 128, A_TM_COLS = 256;
-constexpr uint32_t kStageBytesA = 64 * 256 * 2 + 64 * 512 + 2 * 64 * 128;   // q, k, log_alpha, V
+static_assert(A_TB % 1024 == 0 && A_V % 1024 == 0 && A_KH % 1024 == 0, "swizzled tiles are 1024-aligned");
+static_assert(64 * 65 * 4 <= A_TB - A_KH, "A fits the K e^{-g} region");
+constexpr uint32_t A_TM_GW = 0, A_TM_UV = 128, A_TM_COLS = 256;
 
 __device__ __forceinline__ bool row_ok(const PrefillParams &p, const SeqSpan &sp, int pos) {
   return pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
 }
 
-__global__ void __launch_bounds__(kThreadsA, 1)
-intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqSpan *spans,
+__global__ void __launch_bounds__(kThreadsA, 2)
+intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const SeqSpan *spans,
              const int *cbase, unsigned char *items) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
-  __shared__ __align__(8) uint64_t stage_bar;
+  __shared__ __align__(8) uint64_t v_bar;
   __shared__ uint32_t valid_sh[2];
-  __shared__ __align__(16) float decay_sh[kDK];
+  __shared__ float decay_sh[kDK];
   __shared__ float beta_sh[kC];
-  __shared__ float beta_st[kC];
   __shared__ float part_sh[4][kDK];
 
   if (device_error_latched(p.err)) return;
@@ -138,8 +130,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   const int gchunk = blockIdx.x / H, h = blockIdx.x % H;
   const int nchunks = cbase[p.num_seqs];
   if (gchunk >= nchunks) return;
-  // sequence of this chunk: the last b with cbase[b] <= gchunk
-  int lo = 0, hi = p.num_seqs - 1;
+  int lo = 0, hi = p.num_seqs - 1;   // the sequence: last b with cbase[b] <= gchunk
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
@@ -147,6 +138,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   const int b = lo;
   const SeqSpan sp = spans[b];
   const int c0 = sp.begin + (gchunk - cbase[b]) * kC;
+  unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
 
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
@@ -156,17 +148,17 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   if (warp == 0) tmem_alloc(&tmem_base_sh, A_TM_COLS);
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
-    mbar_init(&stage_bar, 1);
+    mbar_init(&v_bar, 1);
   }
-  for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0 | M] = 0
+  for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0
     const int r = 64 + (e >> 3), ch = e & 7;
-    *reinterpret_cast<uint4 *>(base + A_TBM + row_tile_chunk(r, 0, ch, 192)) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(base + A_TB + row_tile_chunk(r, 0, ch, 128)) = make_uint4(0, 0, 0, 0);
   }
   if (tid < kC) {
     const bool ok = row_ok(p, sp, c0 + tid);
     const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
     if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
-    beta_st[tid] = ok ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    beta_sh[tid] = ok ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
   }
   fence_before_sync();
   __syncthreads();
@@ -174,15 +166,69 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   const uint32_t tm = tmem_base_sh;
   const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
   if (tid == 0) {
-    mbar_arrive_expect_tx(&stage_bar, kStageBytesA);
-    tma_load_3d(smem_u32(base + A_STQ), &maps.q, 0, h, c0, &stage_bar);
-    tma_load_3d(smem_u32(base + A_STK), &maps.k, 0, h, c0, &stage_bar);
-    tma_load_3d(smem_u32(base + A_STG), &maps.la, 0, h, c0, &stage_bar);
-    tma_load_3d(smem_u32(base + A_V), &maps.v, 0, h, c0, &stage_bar);
-    tma_load_3d(smem_u32(base + A_V + 64 * 128), &maps.v, 64, h, c0, &stage_bar);
+    mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+    tma_load_3d(smem_u32(base + A_V), &vmap, 0, h, c0, &v_bar);
+    tma_load_3d(smem_u32(base + A_V + 64 * 128), &vmap, 64, h, c0, &v_bar);
   }
-  bool ok = __syncthreads_and(mbar_wait(&stage_bar, 0, kWaitCycles));
+  // ---- decay products and operand tiles (global loads overlap the V copy)
+  {
+    prep::PrepTiles t;
+    t.qg = base + A_QK; t.qg_R = 128; t.qg_row0 = 0;
+    t.kg = base + A_QK; t.kg_R = 128; t.kg_row0 = 64;
+    t.kh = base + A_KH;
+    t.kt = nullptr;
+    prep::decay_and_tiles_global(reinterpret_cast<const uint16_t *>(p.q),
+                                 reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
+                                 valid_sh, t, it + IT_WQ, it + IT_KT,
+                                 reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, tid);
+  }
+  fence_async_smem();
+  __syncthreads();
   uint32_t phase = 0;
+  bool ok = true;
+  // ---- Gram: [Q G ; K G] (K e^{-g})^T  -> M (lanes 0-63), A / beta (lanes 64-127)
+  if (tid == 0) {
+    fence_after_sync();
+    const uint32_t id = idesc_bf16(128, 64, 0, 0);
+    const uint32_t sQK = smem_u32(base + A_QK), sKH = smem_u32(base + A_KH);
+    for (int s = 0; s < 8; ++s)
+      mma_bf16(tm + A_TM_GW, desc_kmajor(sQK, 128, 0, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
+    mma_commit(&mma_bar);
+  }
+  ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+  phase++;
+  if (ok) {
+    fence_after_sync();
+    float *As = reinterpret_cast<float *>(base + A_KH);     // K e^{-g} is no longer needed
+    float *Ts = reinterpret_cast<float *>(base + A_TS);
+    float *Xs = reinterpret_cast<float *>(base + A_XS);
+    {
+      float v[32];
+      tmem_ld32(tm + my_cols + A_TM_GW, v);
+      if (lr < kC) {      // M row -> item (64 x 64 row tile), columns 32 wg .. 32 wg + 31
+        const int r = lr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (wg * 32 + j <= r) ? v[j] : 0.f;
+        prep::store_row32(it + IT_M, 64, r, wg * 4, v);
+      }
+      __syncthreads();    // every lane has read the Gram before A overwrites K e^{-g}
+      if (lr >= kC) {
+        const int r = lr - kC;
+        const float br = beta_sh[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int i = wg * 32 + j;
+          As[r * 65 + i] = (i < r) ? br * v[j] : 0.f;
+        }
+      }
+    }
+    __syncthreads();
+    tri::unit_lower_inverse_64(As, Ts, Xs, tid);
+    prep::pack_tb(Ts, beta_sh, base + A_TB, 128, tid);
+    fence_async_smem();
+    __syncthreads();
+    ok = __syncthreads_and(mbar_wait(&v_bar, 0, kWaitCycles));
+  }
   if (ok) {
     // zero V rows of invalid positions (tail of the sequence, pads)
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
@@ -191,96 +237,41 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
         if (!((valid_sh[r >> 5] >> (r & 31)) & 1u))
           *reinterpret_cast<uint4 *>(base + A_V + row_tile_chunk(r, blk, ch, kC)) = make_uint4(0, 0, 0, 0);
       }
+      fence_async_smem();
+      __syncthreads();
     }
-    prep::PrepTiles t;
-    t.qg = base + A_QKW; t.qg_R = 192; t.qg_row0 = 64;
-    t.kg = base + A_QKW; t.kg_R = 192; t.kg_row0 = 128;
-    t.kh = base + A_KH;
-    t.kt = base + A_KT;
-    prep::decay_and_tiles(reinterpret_cast<const uint16_t *>(base + A_STQ),
-                          reinterpret_cast<const uint16_t *>(base + A_STK),
-                          reinterpret_cast<const float *>(base + A_STG), valid_sh, t, part_sh,
-                          decay_sh, beta_st, beta_sh, tid);
-    fence_async_smem();
-    __syncthreads();
-    // ---- Gram: [Q G ; K G] (K e^{-g})^T
+    // ---- [W ; 0] = [T_b ; 0] (K G) ;  [U_v ; 0] = [T_b ; 0] V   (N = 128 each)
     if (tid == 0) {
       fence_after_sync();
-      const uint32_t id = idesc_bf16(128, 64, 0, 0);
-      const uint32_t sQKW = smem_u32(base + A_QKW), sKH = smem_u32(base + A_KH);
-      for (int s = 0; s < 8; ++s)
-        mma_bf16(tm + A_TM_G, desc_kmajor(sQKW, 192, 64, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
-      mma_commit(&mma_bar);
-    }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
-    phase++;
-  }
-  if (ok) {
-    fence_after_sync();
-    float *As = reinterpret_cast<float *>(base + A_AS);
-    float *Ts = reinterpret_cast<float *>(base + A_TS);
-    float *Xs = reinterpret_cast<float *>(base + A_XS);
-    prep::extract_gram(tm + my_cols + A_TM_G, base + A_TBM, 192, 128, As, beta_sh, tid);
-    __syncthreads();
-    tri::unit_lower_inverse_64(As, Ts, Xs, tid);
-    prep::pack_tb(Ts, beta_sh, base + A_TBM, 192, tid);
-    fence_async_smem();
-    __syncthreads();
-    // ---- W^T = (K G)^T T_b^T ;  [U_v ; 0] = [T_b ; 0] V   (N = 128: all of d_v)
-    if (tid == 0) {
-      fence_after_sync();
-      const uint32_t sQKW = smem_u32(base + A_QKW), sTBM = smem_u32(base + A_TBM);
+      const uint32_t sQK = smem_u32(base + A_QK), sTB = smem_u32(base + A_TB);
       const uint32_t sV = smem_u32(base + A_V);
-      const uint32_t idw = idesc_bf16(128, 64, 1, 0);
+      const uint32_t id = idesc_bf16(128, 128, 0, 1);
       for (int s = 0; s < 4; ++s)
-        mma_bf16(tm + A_TM_W, desc_mnmajor(sQKW, 192, 128, s), desc_kmajor(sTBM, 192, 0, s), idw, s > 0);
-      const uint32_t idu = idesc_bf16(128, 128, 0, 1);
+        mma_bf16(tm + A_TM_GW, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sQK, 128, 64, s), id, s > 0);
       for (int s = 0; s < 4; ++s)
-        mma_bf16(tm + A_TM_UV, desc_kmajor(sTBM, 192, 0, s), desc_mnmajor(sV, 64, 0, s), idu, s > 0);
+        mma_bf16(tm + A_TM_UV, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sV, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
     }
     ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
     phase++;
   }
-  if (ok) {
+  if (ok && (warp & 3) < 2) {
+    // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> item rows 0..63, U_v -> item
     fence_after_sync();
-    // -W into rows 0..63 of the [-W | Q G | K G] tile (lane = key channel)
-    {
-      float v[32];
-      tmem_ld32(tm + my_cols + A_TM_W, v);
+    const int r = lr;
+    float v[32];
+    for (int q2 = 0; q2 < 2; ++q2) {
+      tmem_ld32(tm + lane_base + A_TM_GW + (uint32_t)(wg * 64 + q2 * 32), v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        *reinterpret_cast<__nv_bfloat16 *>(base + A_QKW + row_tile_off(wg * 32 + j, lr, 192)) =
-            __float2bfloat16_rn(-v[j]);
-    }
-    // U_v rows (lanes 0-63): columns 64 wg .. 64 wg + 63 -> block wg of the U_v tile
-    if ((warp & 3) < 2) {
-      float v[32];
-      const uint32_t col = lane_base + A_TM_UV + (uint32_t)(wg * 64);
-      tmem_ld32(tm + col, v);
-      prep::store_row32(base + A_UV + wg * 64 * 128, 64, lr, 0, v);
-      tmem_ld32(tm + col + 32, v);
-      prep::store_row32(base + A_UV + wg * 64 * 128, 64, lr, 4, v);
-    }
-    fence_async_smem();
-    __syncthreads();
-    // ---- bulk stores of the item
-    if (tid == 0) {
-      unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
-      bulk_store(it + IT_WQ, base + A_QKW, 128 * 128);                       // block 0 rows 0..127
-      bulk_store(it + IT_WQ + 128 * 128, base + A_QKW + 192 * 128, 128 * 128);  // block 1 rows 0..127
-      bulk_store(it + IT_KT, base + A_KT, 64 * 256);
-      bulk_store(it + IT_UV, base + A_UV, 64 * 256);
-      bulk_store(it + IT_M, base + A_TBM + 128 * 128, 64 * 128);
-      bulk_store(it + IT_GC, decay_sh, kDK * 4);
-      bulk_commit();
-      bulk_wait_read();
+      for (int j = 0; j < 32; ++j) v[j] = -v[j];
+      prep::store_row32(it + IT_WQ + wg * 128 * 128, 128, r, q2 * 4, v);
+      tmem_ld32(tm + lane_base + A_TM_UV + (uint32_t)(wg * 64 + q2 * 32), v);
+      prep::store_row32(it + IT_UV + wg * 64 * 128, 64, r, q2 * 4, v);
     }
   }
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
-    // let whatever timed out (the staging loads or a product) finish, bounded
-    mbar_wait(&stage_bar, 0, kWaitCycles);
+    mbar_wait(&v_bar, 0, kWaitCycles);
     if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
   }
   fence_before_sync();
@@ -292,7 +283,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
 }
 
 // ============================================================ state pass (B)
-constexpr int kThreadsB = 128;
+constexpr int kThreadsB = 256;
 constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
 constexpr uint32_t BUF_BYTES = 66560;
 constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
@@ -331,8 +322,9 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
 
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int tid = threadIdx.x, warp = tid >> 5, lr = tid & 127, wg = tid >> 7;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
 
   if (warp == 0) tmem_alloc(&tmem_base_sh, B_TM_COLS);
   if (tid == 0) {
@@ -344,14 +336,12 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = tmem_base_sh;
-  {   // initial state: thread owns state row tid (64 columns)
+  {   // initial state: thread owns state row lr, columns 32 wg .. 32 wg + 31
     float v[32];
-    for (int half = 0; half < 2; ++half) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32 + j] : 0.f;
-      tmem_st32(tm + lane_base + B_TM_S + half * 32, v);
-    }
+    for (int j = 0; j < 32; ++j)
+      v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32 + j] : 0.f;
+    tmem_st32(tm + my_cols + B_TM_S, v);
     tmem_st_wait();
   }
   if (tid == 0) {
@@ -374,15 +364,13 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     loads_waited = j + 1;
     // ---- S -> bf16 operand; S *= e^{g_C}
     {
-      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[tid];
+      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + B_TM_S + half * 32, v);
-        prep::store_row32(base + B_SB, 128, tid, half * 4, v);
+      tmem_ld32(tm + my_cols + B_TM_S, v);
+      prep::store_row32(base + B_SB, 128, lr, wg * 4, v);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
-        tmem_st32(tm + lane_base + B_TM_S + half * 32, v);
-      }
+      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
+      tmem_st32(tm + my_cols + B_TM_S, v);
       tmem_st_wait();
     }
     fence_async_smem();
@@ -401,23 +389,21 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     if (!ok) break;
     fence_after_sync();
     // ---- U = U_v - W S (lanes 0-63) -> bf16 operand
-    if (warp < 2) {
-      const int r = tid;
+    if ((warp & 3) < 2) {
+      const int r = lr;
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + B_TM_D1 + half * 32, v);
+      tmem_ld32(tm + my_cols + B_TM_D1, v);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, half * 4 + q, kC));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int q = 0; q < 4; ++q) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, wg * 4 + q, kC));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
-            v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-          }
+        for (int e = 0; e < 4; ++e) {
+          v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
+          v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
         }
-        prep::store_row32(base + B_UB, 64, r, half * 4, v);
       }
+      prep::store_row32(base + B_UB, 64, r, wg * 4, v);
     }
     fence_async_smem();
     fence_before_sync();
@@ -438,24 +424,22 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     if (!ok) break;
     fence_after_sync();
     // ---- O (lanes 64-127) -> global
-    if (warp >= 2) {
-      const int r = tid - kC;
+    if ((warp & 3) >= 2) {
+      const int r = lr - kC;
       const int pos = c0 + r;
       float v[32];
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tm + lane_base + B_TM_D1 + half * 32, v);
-        if (pos < sp.end) {
-          const bool valid = p.mask == nullptr || p.mask[pos] != 0;
-          uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + half * 32;
+      tmem_ld32(tm + my_cols + B_TM_D1, v);
+      if (pos < sp.end) {
+        const bool valid = p.mask == nullptr || p.mask[pos] != 0;
+        uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * 32;
 #pragma unroll
-          for (int jj = 0; jj < 32; jj += 8) {
-            uint4 pk;
-            pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
-            pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
-            pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
-            pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
-            *reinterpret_cast<uint4 *>(orow + jj) = pk;
-          }
+        for (int jj = 0; jj < 32; jj += 8) {
+          uint4 pk;
+          pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
+          pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
+          pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
+          pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
+          *reinterpret_cast<uint4 *>(orow + jj) = pk;
         }
       }
     }
@@ -474,13 +458,11 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
   } else if (p.final_state) {
     float v[32];
-    for (int half = 0; half < 2; ++half) {
-      tmem_ld32(tm + lane_base + B_TM_S + half * 32, v);
-      float *dst = p.final_state + (((size_t)b * H + h) * kDK + tid) * DV + dv0 + half * 32;
+    tmem_ld32(tm + my_cols + B_TM_S, v);
+    float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32;
 #pragma unroll
-      for (int jj = 0; jj < 32; jj += 4)
-        *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
-    }
+    for (int jj = 0; jj < 32; jj += 4)
+      *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
   }
   // item loads still in flight after a timeout land (bounded) before the CTA exits
   for (int jj = loads_waited; jj < loads_issued; ++jj)
@@ -535,17 +517,14 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   chunk_index_kernel<<<1, 1024, 0, s>>>(p, spans, cbase);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  IntraMaps maps;
-  if (!encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV, CU_TENSOR_MAP_SWIZZLE_128B))
+  CUtensorMap vmap;
+  if (!encode_3d(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
   const size_t gridA = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
   if (gridA > 0x7FFFFFFFull) return cudaErrorInvalidValue;
-  intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, maps, spans, cbase, items);
+  intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
