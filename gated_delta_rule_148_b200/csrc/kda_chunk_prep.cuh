@@ -117,10 +117,12 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
 // Q G into rows 64.. of the 128-row output tile `gq` and K e^{g_C - g} into the
 // 64-row output tile `gkt` (global memory, same swizzled layout), and e^{g_C} into
 // `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
+// beta_val (threads 0..63: beta of row tid, already in a register) is stored to
+// beta_out after the row loads are issued, so its latency overlaps theirs.
 __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
-    float *gdecay, float (*part)[kDK], float *decay, int tid) {
+    float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out, int tid) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -150,6 +152,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
   }
   part[qt][c] = t0;
   part[qt][c + 1] = t1;
+  if (tid < kC) beta_out[tid] = beta_val;
   __syncthreads();
   float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
 #pragma unroll

@@ -19,6 +19,7 @@
 //   [65536, 73728)  M            64 x 64 bf16 row tile
 //   [73728, 74240)  e^{g_C}      128 fp32
 #include <climits>
+#include <mutex>
 
 #include <cudaTypedefs.h>
 
@@ -115,7 +116,7 @@ __device__ __forceinline__ bool row_ok(const PrefillParams &p, const SeqSpan &sp
 
 __global__ void __launch_bounds__(kThreadsA, 2)
 intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const SeqSpan *spans,
-             const int *cbase, unsigned char *items) {
+             const int *cbase, unsigned char *items, int h0, int Hg) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
@@ -127,7 +128,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 
   if (device_error_latched(p.err)) return;
   const int H = p.H;
-  const int gchunk = blockIdx.x / H, h = blockIdx.x % H;
+  const int gchunk = blockIdx.x / Hg, h = h0 + blockIdx.x % Hg;
   const int nchunks = cbase[p.num_seqs];
   if (gchunk >= nchunks) return;
   int lo = 0, hi = p.num_seqs - 1;   // the sequence: last b with cbase[b] <= gchunk
@@ -154,11 +155,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     const int r = 64 + (e >> 3), ch = e & 7;
     *reinterpret_cast<uint4 *>(base + A_TB + row_tile_chunk(r, 0, ch, 128)) = make_uint4(0, 0, 0, 0);
   }
+  float beta_val = 0.f;      // stored to shared memory inside the prep, after its loads
   if (tid < kC) {
     const bool ok = row_ok(p, sp, c0 + tid);
     const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
     if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
-    beta_sh[tid] = ok ? p.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    if (ok) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
   }
   fence_before_sync();
   __syncthreads();
@@ -180,7 +182,8 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     prep::decay_and_tiles_global(reinterpret_cast<const uint16_t *>(p.q),
                                  reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
                                  valid_sh, t, it + IT_WQ, it + IT_KT,
-                                 reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, tid);
+                                 reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, beta_val,
+                                 beta_sh, tid);
   }
   fence_async_smem();
   __syncthreads();
@@ -283,14 +286,21 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 }
 
 // ============================================================ state pass (B)
-constexpr int kThreadsB = 256;
+// 8 compute warps + 1 producer warp.  The producer streams each chunk's item
+// into one of two buffers as soon as the products that read the buffer are
+// done; the compute warps run the chain and synchronise among themselves on a
+// named barrier.  The output accumulator is double-buffered in TMEM, so a
+// chunk's output epilogue runs while the next chunk's first product is in
+// flight.
+constexpr int kComputeThreadsB = 256;
+constexpr int kThreadsB = kComputeThreadsB + 32;
 constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
 constexpr uint32_t BUF_BYTES = 66560;
 constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
 constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES, B_UB = B_SB + 128 * 128;
 constexpr uint32_t B_USED = B_UB + 64 * 128;
 constexpr uint32_t B_SMEM = B_USED + 1024;
-constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 128;
+constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 256;   // D1 buffers at 64 and 128
 
 __device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int tile,
                                           uint64_t *bar) {
@@ -302,18 +312,28 @@ __device__ __forceinline__ void load_item(unsigned char *buf, const unsigned cha
   bulk_load(buf + BUF_GC, it + IT_GC, 512, bar);
 }
 
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, %0;" :: "n"(kComputeThreadsB) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreadsB, 1)
-state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsigned char *items) {
+state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsigned char *items,
+             int h0, int Hg) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t load_bar[2];
+  __shared__ __align__(8) uint64_t free_bar[2];
+  __shared__ int err_sh;
 
   if (device_error_latched(p.err)) return;
   const int tiles = p.dv / kNV;
   const int tile = blockIdx.x % tiles;
-  const int h = (blockIdx.x / tiles) % p.H;
-  const int b = blockIdx.x / (tiles * p.H);
+  const int h = h0 + (blockIdx.x / tiles) % Hg;
+  const int b = blockIdx.x / (tiles * Hg);
   const int dv0 = tile * kNV;
   const int H = p.H, DV = p.dv;
   const SeqSpan sp = spans[b];
@@ -322,7 +342,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
 
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
-  const int tid = threadIdx.x, warp = tid >> 5, lr = tid & 127, wg = tid >> 7;
+  const int tid = threadIdx.x, warp = tid >> 5, lr = tid & 127, wg = (tid >> 7) & 1;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
 
@@ -331,39 +351,46 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     mbar_init(&mma_bar, 1);
     mbar_init(&load_bar[0], 1);
     mbar_init(&load_bar[1], 1);
+    mbar_init(&free_bar[0], 1);
+    mbar_init(&free_bar[1], 1);
+    err_sh = 0;
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = tmem_base_sh;
-  {   // initial state: thread owns state row lr, columns 32 wg .. 32 wg + 31
-    float v[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32 + j] : 0.f;
-    tmem_st32(tm + my_cols + B_TM_S, v);
-    tmem_st_wait();
-  }
-  if (tid == 0) {
-    for (int j = 0; j < 2 && j < nch; ++j)
-      load_item(base + (j ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES, tile,
-                &load_bar[j]);
-  }
-  const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
-  uint32_t phase = 0;
-  bool ok = true;
-  int loads_issued = nch < 2 ? nch : 2;   // item loads issued so far (thread 0's view)
-  int loads_waited = 0;
 
-  for (int j = 0; j < nch; ++j) {
-    const int c0 = sp.begin + j * kC;
-    unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
-    const uint32_t sbuf = smem_u32(buf);
-    ok = __syncthreads_and(mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles));
-    if (!ok) break;
-    loads_waited = j + 1;
-    // ---- S -> bf16 operand; S *= e^{g_C}
-    {
+  if (warp == kComputeThreadsB / 32) {
+    // ---------------- producer warp: item loads, two chunks ahead of the chain
+    if ((tid & 31) == 0) {
+      for (int j = 0; j < nch; ++j) {
+        if (j >= 2 && !mbar_wait(&free_bar[j & 1], ((j - 2) >> 1) & 1, kWaitCycles)) {
+          atomicOr(p.err, ERR_BIT_TIMEOUT);
+          break;
+        }
+        if (*reinterpret_cast<volatile int *>(&err_sh)) break;
+        load_item(base + ((j & 1) ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES,
+                  tile, &load_bar[j & 1]);
+      }
+    }
+  } else {
+    // ---------------- compute warps
+    {   // initial state: thread owns state row lr, columns 32 wg .. 32 wg + 31
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32 + j] : 0.f;
+      tmem_st32(tm + my_cols + B_TM_S, v);
+      tmem_st_wait();
+    }
+    const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
+    uint32_t phase = 0;
+    bool ok = true;
+
+    // Chunk j: S -> bf16 operand, S *= e^{g_C}; then [-W ; Q G] S into D1[j & 1].
+    auto begin_chunk = [&](int j) {
+      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
+      if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles)) err_sh = 1;
       const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
       float v[32];
       tmem_ld32(tm + my_cols + B_TM_S, v);
@@ -372,101 +399,117 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
       tmem_st32(tm + my_cols + B_TM_S, v);
       tmem_st_wait();
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    // ---- [-W S ; (Q G) S] = [-W ; Q G] S
-    if (tid == 0) {
-      fence_after_sync();
-      const uint32_t id = idesc_bf16(128, 64, 0, 1);
-      for (int s = 0; s < 8; ++s)
-        mma_bf16(tm + B_TM_D1, desc_kmajor(sbuf + BUF_WQ, 128, 0, s), desc_mnmajor(sSB, 128, 0, s), id, s > 0);
-      mma_commit(&mma_bar);
-    }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
-    phase++;
-    if (!ok) break;
-    fence_after_sync();
-    // ---- U = U_v - W S (lanes 0-63) -> bf16 operand
-    if ((warp & 3) < 2) {
-      const int r = lr;
-      float v[32];
-      tmem_ld32(tm + my_cols + B_TM_D1, v);
+      fence_async_smem();
+      fence_before_sync();
+      compute_sync();
+      if (tid == 0 && !err_sh) {
+        fence_after_sync();
+        const uint32_t id = idesc_bf16(128, 64, 0, 1);
+        const uint32_t d1 = tm + B_TM_D1 + (uint32_t)((j & 1) * 64);
+        const uint64_t a0 = desc_kmajor(smem_u32(buf) + BUF_WQ, 128, 0, 0);
+        const uint64_t b0 = desc_mnmajor(sSB, 128, 0, 0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, wg * 4 + q, kC));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
-          v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
+        for (int s = 0; s < 8; ++s)
+          mma_bf16(d1, a0 + (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4),
+                   b0 + (uint64_t)((16 * s * 128) >> 4), id, s > 0);
+        mma_commit(&mma_bar);
       }
-      prep::store_row32(base + B_UB, 64, r, wg * 4, v);
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
-    if (tid == 0) {
-      fence_after_sync();
-      const uint32_t ido = idesc_bf16(128, 64, 0, 1);
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tm + B_TM_D1, desc_kmajor(sbuf + BUF_UV, 128, 0, s), desc_mnmajor(sUB, 64, 0, s), ido, 1);
-      const uint32_t ids = idesc_bf16(128, 64, 1, 1);
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tm + B_TM_S, desc_mnmajor(sbuf + BUF_KT, 64, 0, s), desc_mnmajor(sUB, 64, 0, s), ids, 1);
-      mma_commit(&mma_bar);
-    }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
-    phase++;
-    if (!ok) break;
-    fence_after_sync();
-    // ---- O (lanes 64-127) -> global
-    if ((warp & 3) >= 2) {
-      const int r = lr - kC;
-      const int pos = c0 + r;
-      float v[32];
-      tmem_ld32(tm + my_cols + B_TM_D1, v);
-      if (pos < sp.end) {
-        const bool valid = p.mask == nullptr || p.mask[pos] != 0;
-        uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * 32;
-#pragma unroll
-        for (int jj = 0; jj < 32; jj += 8) {
-          uint4 pk;
-          pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
-          pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
-          pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
-          pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
-          *reinterpret_cast<uint4 *>(orow + jj) = pk;
-        }
-      }
-    }
-    fence_before_sync();
-    __syncthreads();
-    // this buffer is free: stream chunk j + 2 into it
-    if (j + 2 < nch) {
-      if (tid == 0)
-        load_item(buf, items + ((size_t)(cb + j + 2) * H + h) * ITEM_BYTES, tile, &load_bar[j & 1]);
-      loads_issued = j + 3;
-    }
-  }
+    };
 
-  if (!ok) {
-    if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
-    mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
-  } else if (p.final_state) {
-    float v[32];
-    tmem_ld32(tm + my_cols + B_TM_S, v);
-    float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32;
+    if (nch > 0) begin_chunk(0);
+    for (int j = 0; j < nch; ++j) {
+      const int c0 = sp.begin + j * kC;
+      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
+      const uint32_t sbuf = smem_u32(buf);
+      const uint32_t d1 = B_TM_D1 + (uint32_t)((j & 1) * 64);
+      // ---- wait for [-W S ; (Q G) S]; U = U_v - W S (lanes 0-63) -> bf16 operand
+      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      phase++;
+      fence_after_sync();
+      if ((warp & 3) < 2) {
+        const int r = lr;
+        float v[32];
+        tmem_ld32(tm + my_cols + d1, v);
 #pragma unroll
-    for (int jj = 0; jj < 32; jj += 4)
-      *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+        for (int q = 0; q < 4; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, wg * 4 + q, kC));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
+            v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+          }
+        }
+        prep::store_row32(base + B_UB, 64, r, wg * 4, v);
+      }
+      fence_async_smem();
+      fence_before_sync();
+      compute_sync();
+      if (*reinterpret_cast<volatile int *>(&err_sh)) { ok = false; break; }
+      // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
+      if (tid == 0) {
+        fence_after_sync();
+        const uint32_t ido = idesc_bf16(128, 64, 0, 1);
+        const uint32_t ids = idesc_bf16(128, 64, 1, 1);
+        const uint64_t ao = desc_kmajor(sbuf + BUF_UV, 128, 0, 0);
+        const uint64_t as = desc_mnmajor(sbuf + BUF_KT, 64, 0, 0);
+        const uint64_t bu = desc_mnmajor(sUB, 64, 0, 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
+        mma_commit(&mma_bar);
+      }
+      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      phase++;
+      fence_after_sync();
+      if (tid == 0) mbar_arrive(&free_bar[j & 1]);     // the products that read buffer j & 1 are done
+      // ---- next chunk's first product goes out before this chunk's output epilogue
+      if (j + 1 < nch) begin_chunk(j + 1);
+      // ---- O (lanes 64-127 of D1[j & 1]) -> global
+      if ((warp & 3) >= 2) {
+        const int r = lr - kC;
+        const int pos = c0 + r;
+        float v[32];
+        tmem_ld32(tm + my_cols + d1, v);
+        if (pos < sp.end) {
+          const bool valid = p.mask == nullptr || p.mask[pos] != 0;
+          uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * 32;
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 8) {
+            uint4 pk;
+            pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
+            pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
+            pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
+            pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
+            *reinterpret_cast<uint4 *>(orow + jj) = pk;
+          }
+        }
+      }
+    }
+    compute_sync();
+    ok = ok && !*reinterpret_cast<volatile int *>(&err_sh);
+    if (!ok) {
+      if (tid == 0) {
+        err_sh = 1;
+        atomicOr(p.err, ERR_BIT_TIMEOUT);
+      }
+      if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+    } else if (p.final_state) {
+      float v[32];
+      tmem_ld32(tm + my_cols + B_TM_S, v);
+      float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32;
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 4)
+        *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+    }
+    if (tid == 0 && !ok) {
+      // item loads the producer issued but the chain never consumed land before exit
+      for (int jj = 0; jj < nch; ++jj) mbar_wait(&load_bar[jj & 1], (jj >> 1) & 1, 20000);
+    }
   }
-  // item loads still in flight after a timeout land (bounded) before the CTA exits
-  for (int jj = loads_waited; jj < loads_issued; ++jj)
-    mbar_wait(&load_bar[jj & 1], (jj >> 1) & 1, kWaitCycles);
   fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -507,6 +550,44 @@ bool prefill_split_supported(const PrefillParams &p, bool bf16) {
 
 size_t prefill_split_workspace(int N, int B, int H) { return split::ws_total(N, B, H); }
 
+namespace {
+
+// Head groups run as a pipeline: the intra kernel of group g+1 (bandwidth-bound,
+// all SMs) overlaps the state pass of group g (latency-bound, few SMs) on its
+// own high-priority stream; everything joins back on the caller's stream.
+constexpr int kGroups = 1;
+constexpr int kMaxDev = 64;
+struct GroupStreams {
+  bool ready = false;
+  cudaStream_t aux[kGroups];
+  cudaEvent_t ev_a[kGroups], ev_b[kGroups];
+};
+GroupStreams g_streams[kMaxDev];
+std::mutex g_streams_mu;
+
+cudaError_t group_streams(GroupStreams **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  GroupStreams &gs = g_streams[dev];
+  if (!gs.ready) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e != cudaSuccess) return e;
+    for (int g = 0; g < kGroups; ++g) {
+      if ((e = cudaStreamCreateWithPriority(&gs.aux[g], cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&gs.ev_a[g], cudaEventDisableTiming)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&gs.ev_b[g], cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    gs.ready = true;
+  }
+  *out = &gs;
+  return cudaSuccess;
+}
+
+}  // namespace
+
 // spans: B entries already written by the pre-pass; ws: workspace base.
 cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s) {
   using namespace split;
@@ -522,15 +603,31 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
     return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
-  const size_t gridA = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
-  if (gridA > 0x7FFFFFFFull) return cudaErrorInvalidValue;
-  intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
   if (e != cudaSuccess) return e;
-  const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / kNV);
-  state_kernel<<<gridB, kThreadsB, B_SMEM, s>>>(p, spans, cbase, items);
+  std::lock_guard<std::mutex> lock(g_streams_mu);
+  GroupStreams *gs = nullptr;
+  if ((e = group_streams(&gs)) != cudaSuccess) return e;
+  const int G = p.H < kGroups ? p.H : kGroups;
+  const int Hg = (p.H + G - 1) / G;
+  int used = 0;
+  for (int g = 0; g < G; ++g) {
+    const int h0 = g * Hg, hg = (p.H - h0) < Hg ? (p.H - h0) : Hg;
+    if (hg <= 0) break;
+    const size_t gridA = max_chunks(p.N, p.num_seqs) * (size_t)hg;
+    if (gridA > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+    intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, h0, hg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(gs->ev_a[g], s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(gs->aux[g], gs->ev_a[g], 0)) != cudaSuccess) return e;
+    const unsigned gridB = (unsigned)p.num_seqs * hg * (p.dv / kNV);
+    state_kernel<<<gridB, kThreadsB, B_SMEM, gs->aux[g]>>>(p, spans, cbase, items, h0, hg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(gs->ev_b[g], gs->aux[g])) != cudaSuccess) return e;
+    ++used;
+  }
+  for (int g = 0; g < used; ++g)
+    if ((e = cudaStreamWaitEvent(s, gs->ev_b[g], 0)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
