@@ -114,9 +114,9 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
 // P1 reading q, k, log_alpha straight from global memory (rows of the chunk at
 // packed positions c0 .. c0+63 of head h; invalid rows count as zero).  Besides the
 // shared tiles (Q G and K G rows of `t.qg/t.kg`, K e^{-g} in `t.kh`), it writes
-// Q G into rows 64.. of the 128-row output tile `gq` and K e^{g_C - g} into the
-// 64-row output tile `gkt` (global memory, same swizzled layout), and e^{g_C} into
-// `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
+// Q G into rows 64.. of the 128-row output tile `gq` (if not null) and K e^{g_C - g}
+// into the 64-row tile `gkt` (global or shared memory, same swizzled layout), and
+// e^{g_C} into `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
 // beta_val (threads 0..63: beta of row tid, already in a register) is stored to
 // beta_out after the row loads are issued, so its latency overlaps theirs.
 __device__ __forceinline__ void decay_and_tiles_global(
@@ -184,7 +184,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
     e1 *= a1[i];
     const uint32_t qgv = pack_bf16x2(qa * e0, qb * e1);
     *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
-    *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
+    if (gq) *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
     *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
         pack_bf16x2(ka * e0, kb2 * e1);
   }

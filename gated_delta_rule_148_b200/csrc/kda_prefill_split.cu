@@ -93,20 +93,23 @@ __global__ void __launch_bounds__(1024) chunk_index_kernel(PrefillParams p, cons
 }
 
 // ============================================================ intra kernel (A)
-// One CTA per (chunk, head); ~100 KB of shared memory so two CTAs share an SM
-// and hide each other's load and tensor-core latency.  q, k, log_alpha are read
-// straight from global memory; V arrives by TMA; every output goes straight to
-// the workspace item.
+// Persistent: about two CTAs per SM loop over the (chunk, head) items, so the
+// TMEM allocation, barrier set-up and constant tiles are paid once per CTA.
+// ~100 KB of shared memory lets two CTAs share an SM and hide each other's load
+// and tensor-core latency.  q, k, log_alpha are read straight from global
+// memory, V arrives by TMA; the item's tiles leave through shared memory with
+// bulk stores.
 constexpr int kThreadsA = 256;
-constexpr uint32_t A_QK = 0;                        // [Q G | K G]   128 x 128 row tile
-constexpr uint32_t A_KH = A_QK + 128 * 256;         // K e^{-g} 64 x 128 (then A [64][65] f32)
+constexpr uint32_t A_QK = 0;                        // [Q G | K G] 128 x 128 row tile; then [-W | .]
+constexpr uint32_t A_KH = A_QK + 128 * 256;         // K e^{-g} 64 x 128; then A [64][65] f32; then U_v
 constexpr uint32_t A_TB = A_KH + 17 * 1024;         // [T_b | 0]     128 x 64 row tile
 constexpr uint32_t A_V = A_TB + 128 * 128;          // V  64 rows x 2 blocks of 64
-constexpr uint32_t A_TS = A_V + 64 * 256;           // T  [64][65] f32
-constexpr uint32_t A_XS = A_TS + 64 * 65 * 4;       // inverse scratch (3 warps x 16 x 17)
-constexpr uint32_t A_USED = A_XS + 3 * 16 * 17 * 4;
+constexpr uint32_t A_TS = A_V + 64 * 256;           // K e^{g_C-g} 64 x 128 tile; then T [64][65] f32
+constexpr uint32_t A_XS = A_TS + 64 * 65 * 4;       // inverse scratch (32 x 33 f32)
+constexpr uint32_t A_USED = A_XS + 32 * 33 * 4;
 constexpr uint32_t A_SMEM = A_USED + 1024;
-static_assert(A_TB % 1024 == 0 && A_V % 1024 == 0 && A_KH % 1024 == 0, "swizzled tiles are 1024-aligned");
+static_assert(A_TB % 1024 == 0 && A_V % 1024 == 0 && A_KH % 1024 == 0 && A_TS % 1024 == 0,
+              "swizzled tiles are 1024-aligned");
 static_assert(64 * 65 * 4 <= A_TB - A_KH, "A fits the K e^{-g} region");
 constexpr uint32_t A_TM_GW = 0, A_TM_UV = 128, A_TM_COLS = 256;
 
@@ -128,18 +131,8 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 
   if (device_error_latched(p.err)) return;
   const int H = p.H;
-  const int gchunk = blockIdx.x / Hg, h = h0 + blockIdx.x % Hg;
-  const int nchunks = cbase[p.num_seqs];
-  if (gchunk >= nchunks) return;
-  int lo = 0, hi = p.num_seqs - 1;   // the sequence: last b with cbase[b] <= gchunk
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  const SeqSpan sp = spans[b];
-  const int c0 = sp.begin + (gchunk - cbase[b]) * kC;
-  unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
+  const int nitems = cbase[p.num_seqs] * Hg;
+  if ((int)blockIdx.x >= nitems) return;
 
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
@@ -151,56 +144,76 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     mbar_init(&mma_bar, 1);
     mbar_init(&v_bar, 1);
   }
-  for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0
+  for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0, for good
     const int r = 64 + (e >> 3), ch = e & 7;
     *reinterpret_cast<uint4 *>(base + A_TB + row_tile_chunk(r, 0, ch, 128)) = make_uint4(0, 0, 0, 0);
-  }
-  float beta_val = 0.f;      // stored to shared memory inside the prep, after its loads
-  if (tid < kC) {
-    const bool ok = row_ok(p, sp, c0 + tid);
-    const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
-    if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
-    if (ok) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = tmem_base_sh;
   const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
-    tma_load_3d(smem_u32(base + A_V), &vmap, 0, h, c0, &v_bar);
-    tma_load_3d(smem_u32(base + A_V + 64 * 128), &vmap, 64, h, c0, &v_bar);
-  }
-  // ---- decay products and operand tiles (global loads overlap the V copy)
-  {
-    prep::PrepTiles t;
-    t.qg = base + A_QK; t.qg_R = 128; t.qg_row0 = 0;
-    t.kg = base + A_QK; t.kg_R = 128; t.kg_row0 = 64;
-    t.kh = base + A_KH;
-    t.kt = nullptr;
-    prep::decay_and_tiles_global(reinterpret_cast<const uint16_t *>(p.q),
-                                 reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
-                                 valid_sh, t, it + IT_WQ, it + IT_KT,
-                                 reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, beta_val,
-                                 beta_sh, tid);
-  }
-  fence_async_smem();
-  __syncthreads();
-  uint32_t phase = 0;
+  const uint32_t sQK = smem_u32(base + A_QK), sKH = smem_u32(base + A_KH);
+  const uint32_t sTB = smem_u32(base + A_TB), sV = smem_u32(base + A_V);
+  uint32_t phase = 0, vphase = 0;
   bool ok = true;
-  // ---- Gram: [Q G ; K G] (K e^{-g})^T  -> M (lanes 0-63), A / beta (lanes 64-127)
-  if (tid == 0) {
-    fence_after_sync();
-    const uint32_t id = idesc_bf16(128, 64, 0, 0);
-    const uint32_t sQK = smem_u32(base + A_QK), sKH = smem_u32(base + A_KH);
-    for (int s = 0; s < 8; ++s)
-      mma_bf16(tm + A_TM_GW, desc_kmajor(sQK, 128, 0, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
-    mma_commit(&mma_bar);
-  }
-  ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
-  phase++;
-  if (ok) {
+
+  for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+    const int gchunk = item / Hg, h = h0 + item % Hg;
+    int lo = 0, hi = p.num_seqs - 1;   // the sequence: last b with cbase[b] <= gchunk
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const SeqSpan sp = spans[b];
+    const int c0 = sp.begin + (gchunk - cbase[b]) * kC;
+    unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
+
+    float beta_val = 0.f;      // stored to shared memory inside the prep, after its loads
+    if (tid < kC) {
+      const bool vr = row_ok(p, sp, c0 + tid);
+      const unsigned bits = __ballot_sync(0xFFFFFFFFu, vr);
+      if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
+      if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+      tma_load_3d(sV, &vmap, 0, h, c0, &v_bar);
+      tma_load_3d(sV + 64 * 128, &vmap, 64, h, c0, &v_bar);
+    }
+    // ---- decay products and operand tiles (global loads overlap the V copy)
+    {
+      prep::PrepTiles t;
+      t.qg = base + A_QK; t.qg_R = 128; t.qg_row0 = 0;
+      t.kg = base + A_QK; t.kg_R = 128; t.kg_row0 = 64;
+      t.kh = base + A_KH;
+      t.kt = nullptr;
+      prep::decay_and_tiles_global(reinterpret_cast<const uint16_t *>(p.q),
+                                   reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
+                                   valid_sh, t, nullptr, base + A_TS,
+                                   reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, beta_val,
+                                   beta_sh, tid);
+    }
+    fence_async_smem();
+    __syncthreads();
+    // ---- Gram: [Q G ; K G] (K e^{-g})^T  -> M (lanes 0-63), A / beta (lanes 64-127);
+    //      Q G and K e^{g_C-g} leave for the item
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t id = idesc_bf16(128, 64, 0, 0);
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(tm + A_TM_GW, desc_kmajor(sQK, 128, 0, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
+      mma_commit(&mma_bar);
+      bulk_store(it + IT_WQ + 64 * 128, base + A_QK, 64 * 128);                   // Q G, block 0
+      bulk_store(it + IT_WQ + 128 * 128 + 64 * 128, base + A_QK + 128 * 128, 64 * 128);  // block 1
+      bulk_store(it + IT_KT, base + A_TS, 64 * 256);
+      bulk_commit();
+    }
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    phase++;
+    if (!ok) break;
     fence_after_sync();
     float *As = reinterpret_cast<float *>(base + A_KH);     // K e^{-g} is no longer needed
     float *Ts = reinterpret_cast<float *>(base + A_TS);
@@ -213,9 +226,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = (wg * 32 + j <= r) ? v[j] : 0.f;
         prep::store_row32(it + IT_M, 64, r, wg * 4, v);
-      }
-      __syncthreads();    // every lane has read the Gram before A overwrites K e^{-g}
-      if (lr >= kC) {
+      } else {
         const int r = lr - kC;
         const float br = beta_sh[r];
 #pragma unroll
@@ -225,14 +236,14 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
         }
       }
     }
+    if (tid == 0) bulk_wait_read();     // K e^{g_C-g} has left the T region
     __syncthreads();
     tri::unit_lower_inverse_64(As, Ts, Xs, tid);
     prep::pack_tb(Ts, beta_sh, base + A_TB, 128, tid);
     fence_async_smem();
-    __syncthreads();
-    ok = __syncthreads_and(mbar_wait(&v_bar, 0, kWaitCycles));
-  }
-  if (ok) {
+    ok = __syncthreads_and(mbar_wait(&v_bar, vphase & 1, kWaitCycles));
+    vphase++;
+    if (!ok) break;
     // zero V rows of invalid positions (tail of the sequence, pads)
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
       for (int e = tid; e < kC * 16; e += kThreadsA) {
@@ -246,8 +257,6 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     // ---- [W ; 0] = [T_b ; 0] (K G) ;  [U_v ; 0] = [T_b ; 0] V   (N = 128 each)
     if (tid == 0) {
       fence_after_sync();
-      const uint32_t sQK = smem_u32(base + A_QK), sTB = smem_u32(base + A_TB);
-      const uint32_t sV = smem_u32(base + A_V);
       const uint32_t id = idesc_bf16(128, 128, 0, 1);
       for (int s = 0; s < 4; ++s)
         mma_bf16(tm + A_TM_GW, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sQK, 128, 64, s), id, s > 0);
@@ -257,25 +266,42 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     }
     ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
     phase++;
-  }
-  if (ok && (warp & 3) < 2) {
-    // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> item rows 0..63, U_v -> item
+    if (!ok) break;
     fence_after_sync();
-    const int r = lr;
-    float v[32];
-    for (int q2 = 0; q2 < 2; ++q2) {
-      tmem_ld32(tm + lane_base + A_TM_GW + (uint32_t)(wg * 64 + q2 * 32), v);
+    if ((warp & 3) < 2) {
+      // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> rows 0..63 of the Q G | K G
+      // tile (its products are done), U_v -> the K e^{-g} region; both leave by bulk store
+      const int r = lr;
+      float v[32];
+      for (int q2 = 0; q2 < 2; ++q2) {
+        tmem_ld32(tm + lane_base + A_TM_GW + (uint32_t)(wg * 64 + q2 * 32), v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = -v[j];
-      prep::store_row32(it + IT_WQ + wg * 128 * 128, 128, r, q2 * 4, v);
-      tmem_ld32(tm + lane_base + A_TM_UV + (uint32_t)(wg * 64 + q2 * 32), v);
-      prep::store_row32(it + IT_UV + wg * 64 * 128, 64, r, q2 * 4, v);
+        for (int j = 0; j < 32; ++j) v[j] = -v[j];
+        prep::store_row32(base + A_QK + wg * 128 * 128, 128, r, q2 * 4, v);
+        tmem_ld32(tm + lane_base + A_TM_UV + (uint32_t)(wg * 64 + q2 * 32), v);
+        prep::store_row32(base + A_KH + wg * 64 * 128, 64, r, q2 * 4, v);
+      }
     }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store(it + IT_WQ, base + A_QK, 64 * 128);                              // -W, block 0
+      bulk_store(it + IT_WQ + 128 * 128, base + A_QK + 128 * 128, 64 * 128);      // -W, block 1
+      bulk_store(it + IT_UV, base + A_KH, 64 * 256);
+      bulk_commit();
+      bulk_wait_read();      // the tiles are rewritten by the next item
+    }
+    fence_before_sync();
+    __syncthreads();
   }
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
-    mbar_wait(&v_bar, 0, kWaitCycles);
+    mbar_wait(&v_bar, (vphase - 0) & 1, 20000);
     if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+  }
+  if (tid == 0) {
+    bulk_commit();
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // item stores complete
   }
   fence_before_sync();
   __syncthreads();
@@ -565,6 +591,18 @@ struct GroupStreams {
 GroupStreams g_streams[kMaxDev];
 std::mutex g_streams_mu;
 
+int num_sms() {
+  static int n[kMaxDev] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+
 cudaError_t group_streams(GroupStreams **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -614,8 +652,9 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   for (int g = 0; g < G; ++g) {
     const int h0 = g * Hg, hg = (p.H - h0) < Hg ? (p.H - h0) : Hg;
     if (hg <= 0) break;
-    const size_t gridA = max_chunks(p.N, p.num_seqs) * (size_t)hg;
-    if (gridA > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+    const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)hg;
+    if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+    const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
     intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, h0, hg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(gs->ev_a[g], s)) != cudaSuccess) return e;

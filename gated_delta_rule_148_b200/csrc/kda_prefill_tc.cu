@@ -69,11 +69,11 @@ constexpr uint32_t OFF_STB = OFF_STG + 64 * 512;      // staging beta [64] f32
 // The inverse's scratch aliases the staging buffers: the next chunk is staged
 // only after the inverse is done.
 constexpr uint32_t OFF_AS = OFF_STQ;                  // A [64][65] f32
-constexpr uint32_t OFF_XS = OFF_AS + 64 * 65 * 4;     // 8 x 16 x 17 f32 per-warp scratch
+constexpr uint32_t OFF_XS = OFF_AS + 64 * 65 * 4;     // 32 x 33 f32 inverse scratch
 constexpr uint32_t OFF_TS = OFF_STG;                  // T [64][65] f32
 constexpr uint32_t SMEM_USED = OFF_STB + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // + alignment slack
-static_assert(OFF_XS + 8 * 16 * 17 * 4 <= OFF_STG, "inverse scratch must fit the q/k staging");
+static_assert(OFF_XS + 32 * 33 * 4 <= OFF_STG, "inverse scratch must fit the q/k staging");
 static_assert(OFF_TS + 64 * 65 * 4 <= OFF_STB, "T must fit the g staging");
 
 // TMEM columns

@@ -3,19 +3,17 @@
 // dense products; "Kimi Linear's 75% KV cache cut ...", theclarity.today,
 // fourth paragraph).
 //
-// Blocked by 16: the four diagonal blocks D_a = (I + A_aa)^{-1} by forward
-// substitution in registers (one thread per column), then the off-diagonal
-// blocks in order of distance d = a - b:
-//   T_ab = -D_a * sum_{m=b}^{a-1} A_am T_mb
-// with the 16 x 16 x 16 block products on the tensor cores (warp-level
-// mma.sync m16n8k8, TF32 inputs rounded to nearest, fp32 accumulation).  The
-// inverse only feeds bf16 operands, so TF32 inputs (2^-11) are below the
-// final rounding (2^-9).
+// Built from 16 x 16 blocks (the inverse of a block unit-lower-triangular
+// matrix [[L11, 0], [L21, L22]] is [[L11^-1, 0], [-L22^-1 L21 L11^-1, L22^-1]]),
+// with the 16 x 16 x 16 block products on the tensor cores (warp-level mma.sync
+// m16n8k8, TF32 inputs rounded to nearest, fp32 accumulation).  The inverse
+// only feeds bf16 operands, so TF32 inputs (2^-11) are below the final
+// rounding (2^-9).
 //
 // Shared arrays are fp32, row-major with stride 65.  A must be strictly lower
 // (zeros on and above the diagonal).  Only entries on or below the diagonal of
 // T are written with meaningful values; the blocks above the diagonal are not
-// touched.  Needs 256 threads (8 warps) and a 16 x 17 fp32 scratch per warp.
+// touched.
 #pragma once
 
 #include <stdint.h>
@@ -76,14 +74,18 @@ __device__ __forceinline__ void store_acc(float *Z, int ldz, const float (&acc)[
   }
 }
 
-// scratch: 8 warps x 16 x 17 floats.  Must be called by all 256 threads.
+// Scratch: 32 x 33 floats.  Must be called by all 256 threads.
+// Recursive doubling: the four 16 x 16 diagonal inverses D_a (registers, one
+// thread per column); then the two 32 x 32 diagonal inverses
+//   P0 = [[D0, 0], [-D1 A10 D0, D1]],  P1 = [[D2, 0], [-D3 A32 D2, D3]];
+// then the lower-left 32 x 32 block -P1 (A_LL P0), with one warp per 16 x 16
+// output tile.  The block products are tensor-core MMAs.
 __device__ __forceinline__ void unit_lower_inverse_64(const float *__restrict__ As,
                                                       float *__restrict__ Ts,
                                                       float *__restrict__ scratch, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  // ---- diagonal blocks: thread (blk, j) holds column j of D_blk in registers.
-  // Right-looking: once t[i] is known it is folded into every later row, so
-  // the dependency depth is 16 steps rather than 120 sequential FMAs.
+  // ---- 16 x 16 diagonal blocks: thread (blk, j) holds column j of D_blk in registers.
+  // Right-looking: once t[i] is known it is folded into every later row.
   if (tid < 64) {
     const int blk = tid >> 4, j = tid & 15, o = blk * 16;
     float acc[16];
@@ -98,23 +100,38 @@ __device__ __forceinline__ void unit_lower_inverse_64(const float *__restrict__ 
     }
   }
   __syncthreads();
-  // ---- off-diagonal blocks by distance
-#pragma unroll 1
-  for (int d = 1; d <= 3; ++d) {
-    if (warp < 4 - d) {
-      const int b = warp, a = warp + d;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      for (int m = b; m < a; ++m)
-        block_mma(acc, As + (a * 16) * LD + m * 16, LD, Ts + (m * 16) * LD + b * 16, LD, lane);
-      float *X = scratch + warp * 16 * 17;
-      store_acc(X, 17, acc, 1.f, lane);
-      __syncwarp();
-      float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      block_mma(acc2, Ts + (a * 16) * LD + a * 16, LD, X, 17, lane);
-      store_acc(Ts + (a * 16) * LD + b * 16, LD, acc2, -1.f, lane);
-    }
-    __syncthreads();
+  // ---- 32 x 32 diagonal blocks: warp 0 -> T10 = -D1 A10 D0, warp 1 -> T32 = -D3 A32 D2
+  if (warp < 2) {
+    const int a = 2 * warp + 1, b = 2 * warp;      // (1,0) or (3,2)
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    block_mma(acc, As + (a * 16) * LD + b * 16, LD, Ts + (b * 16) * LD + b * 16, LD, lane);
+    float *X = scratch + warp * 16 * 17;
+    store_acc(X, 17, acc, 1.f, lane);
+    __syncwarp();
+    float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    block_mma(acc2, Ts + (a * 16) * LD + a * 16, LD, X, 17, lane);
+    store_acc(Ts + (a * 16) * LD + b * 16, LD, acc2, -1.f, lane);
   }
+  __syncthreads();
+  // ---- lower-left 32 x 32: X = A[32:64, 0:32] P0 (tile (i, j) sums m = j..1), one warp per tile
+  float *X = scratch;                             // 32 x 33
+  if (warp < 4) {
+    const int i = warp >> 1, j = warp & 1;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int m = j; m < 2; ++m)
+      block_mma(acc, As + (32 + i * 16) * LD + m * 16, LD, Ts + (m * 16) * LD + j * 16, LD, lane);
+    store_acc(X + (i * 16) * 33 + j * 16, 33, acc, 1.f, lane);
+  }
+  __syncthreads();
+  // ---- T[32:64, 0:32] = -P1 X (tile (i, j) sums m = 0..i)
+  if (warp < 4) {
+    const int i = warp >> 1, j = warp & 1;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int m = 0; m <= i; ++m)
+      block_mma(acc, Ts + (32 + i * 16) * LD + 32 + m * 16, LD, X + (m * 16) * 33 + j * 16, 33, lane);
+    store_acc(Ts + (32 + i * 16) * LD + j * 16, LD, acc, -1.f, lane);
+  }
+  __syncthreads();
 }
 
 }  // namespace tri
