@@ -46,6 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # kernels one kda_prefill launches at H = 32 on the two-kernel path: pad/cu_seqlens
 # pre-pass, chunk index, the intra kernel and the state pass
 LAUNCHES_PER_PREFILL = 2 + 2 * 1
+PREFILL_TRAFFIC_T = 131072   # token count the recorded prefill traffic is for
 
 
 def parse():
@@ -76,7 +77,7 @@ def peaks():
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's source file is
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's source files are
     unchanged since the capture (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -84,13 +85,22 @@ def recorded_traffic(kernel: str):
             e = json.load(f).get(kernel)
         if not e:
             return None
-        with open(os.path.join(ROOT, e["source"]), "rb") as fh:
-            h = hashlib.sha256(fh.read()).hexdigest()[:16]
-        if h == e.get("source_hash"):
+        hs = hashlib.sha256()
+        for src in e.get("sources") or [e["source"]]:
+            with open(os.path.join(ROOT, src), "rb") as fh:
+                hs.update(fh.read())
+        if hs.hexdigest()[:16] == e.get("source_hash"):
             return e.get("dram_bytes_per_launch")
     except Exception:
         pass
     return None
+
+
+def prefill_traffic(T: int):
+    """Recorded DRAM bytes of one prefill call, scaled from the capture's token count to T
+    (inputs, items and outputs all grow in proportion to the tokens)."""
+    b = recorded_traffic("prefill")
+    return None if b is None else int(round(b * T / PREFILL_TRAFFIC_T))
 
 
 # ---------------------------------------------------------------- clocks
@@ -342,7 +352,7 @@ def main_ours(args, rank, world, device):
     algo_bytes = prefill_bytes(T, H)
     achieved = algo_bytes / (ms_step / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic("prefill"),
+                "frac": achieved / pk["hbm_gbs"], "traffic": prefill_traffic(T),
                 "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
                 "kernel": "kda prefill (whole kda_prefill call: pre-pass, chunk index, intra and state kernels)",
                 "algorithmic_bytes_per_launch": algo_bytes,
@@ -354,7 +364,7 @@ def main_ours(args, rank, world, device):
             "config": {"workload": w.name, "global_batch": 1, "seq_len": T, "heads": H,
                        "d_k": 128, "d_v": 128, "chunk": 64, "state": "fp32",
                        "parallelism": f"replicas{world}" if world > 1 else "none",
-                       "l2": "inputs larger than L2 (6.4 GB per step), no flush"},
+                       "l2": f"inputs larger than L2 ({algo_bytes / 1e9:.2f} GB per step), no flush"},
             "roofline": roofline, "clocks": clk, "gpu_launches": LAUNCHES_PER_PREFILL * K}
 
     # ---- e2e through the public API with host buffers
