@@ -217,6 +217,11 @@ def prefill_bytes(T, H):
     return T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
 
 
+def prefill_bytes_head_gate(T, H):
+    """Same, with one fp32 gate per token and head instead of d_k of them."""
+    return T * H * (PREFILL_BYTES_PER_TOKEN_HEAD - 4 * 128 + 4) + H * STATE_BYTES
+
+
 def time_loop(fn, K, W, flush_buf=None):
     """K timed calls after W warm-ups; returns per-call ms (events on the current stream)."""
     import torch
@@ -419,6 +424,16 @@ def main_ours(args, rank, world, device):
                          "hbm_frac": roofline["frac"], "l2": "inputs larger than L2"}
         line["prefill_sweep"] = sweep
         del flush
+        # ---- head-wise gate (one decay per token and head), same q, k, v, beta
+        devh = dict(dev, log_alpha=torch.from_numpy(gen.head_gates(w.seed, T, H)).to(device))
+        msh = time_loop(lambda: run_prefill(kda, devh), K, W)
+        hb = prefill_bytes_head_gate(T, H)
+        line["prefill_head_gate"] = {
+            "tokens_per_s": aggregate_rate(T, world, msh), "ms": msh,
+            "hbm_frac": hb / (msh / 1e3) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": hb,
+            "log_alpha": "[N, H] fp32", "l2": "inputs larger than L2"}
+        line["gpu_launches"] += LAUNCHES_PER_PREFILL * K
+        del devh
 
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(inp)

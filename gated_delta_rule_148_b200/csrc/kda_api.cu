@@ -58,7 +58,7 @@ using namespace kda;
 
 extern "C" {
 
-int kda_version(void) { return (1 << 16) | 0; }
+int kda_version(void) { return (1 << 16) | 1; }
 
 const char *kda_status_string(kda_status s) {
   switch (s) {
@@ -94,12 +94,14 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   int chunk = a->chunk;
   if (chunk == 0) chunk = (a->dtype == KDA_BF16) ? 64 : 16;
   if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if (a->gate != KDA_GATE_CHANNEL && a->gate != KDA_GATE_HEAD) return KDA_ERR_INVALID_ARG;
+  const bool gate_head = a->gate == KDA_GATE_HEAD;
   if (a->num_seqs == 0) return a->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
   if (!a->cu_seqlens) return KDA_ERR_INVALID_ARG;
   const size_t N = (size_t)a->total_tokens, H = (size_t)a->H;
   const size_t es = elem_bytes(a->dtype);
   const Range q{a->q, N * H * a->dk * es}, k{a->k, N * H * a->dk * es};
-  const Range v{a->v, N * H * a->dv * es}, la{a->log_alpha, N * H * a->dk * 4};
+  const Range v{a->v, N * H * a->dv * es}, la{a->log_alpha, N * H * (gate_head ? 1 : a->dk) * 4};
   const Range be{a->beta, N * H * 4}, cu{a->cu_seqlens, 4 * ((size_t)a->num_seqs + 1)};
   const Range mk{a->pad_mask, a->pad_mask ? N : 0};
   const size_t sbytes = (size_t)a->num_seqs * H * a->dk * a->dv * 4;
@@ -109,11 +111,12 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   const Range ws{a->workspace, a->workspace ? a->workspace_bytes : 0};
   if (N > 0 && (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->o))
     return KDA_ERR_INVALID_ARG;
-  const void *need16[] = {a->q, a->k, a->v, (const void *)a->log_alpha, a->o,
+  const void *need16[] = {a->q, a->k, a->v, gate_head ? nullptr : (const void *)a->log_alpha, a->o,
                           (const void *)a->init_state, (const void *)a->final_state};
   for (const void *p : need16)
     if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
-  if (!aligned(a->beta, 4) || !aligned(a->cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+  if (!aligned(a->beta, 4) || !aligned(a->cu_seqlens, 4) || !aligned(a->log_alpha, 4))
+    return KDA_ERR_INVALID_ARG;
   // A pad mask needs at least the span table; a larger workspace (up to
   // kda_prefill_workspace_size) only selects a faster path.
   if (a->pad_mask && (!a->workspace || a->workspace_bytes < spans_bytes(a->num_seqs)))
@@ -150,6 +153,7 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   p.o = a->o;
   p.final_state = a->final_state;
   p.err = err;
+  p.gate_head = gate_head ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = a->dtype == KDA_BF16;
   p.spans = nullptr;
@@ -171,13 +175,15 @@ kda_status kda_decode(const kda_decode_args *a, void *stream) {
   if (!a) return KDA_ERR_INVALID_ARG;
   if (a->dtype != KDA_F32 && a->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (a->B < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (a->gate != KDA_GATE_CHANNEL && a->gate != KDA_GATE_HEAD) return KDA_ERR_INVALID_ARG;
+  const bool gate_head = a->gate == KDA_GATE_HEAD;
   if (!head_dim_ok(a->dk) || !head_dim_ok(a->dv)) return KDA_ERR_UNSUPPORTED;
   if (a->B == 0) return KDA_OK;
   if (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->state || !a->o)
     return KDA_ERR_INVALID_ARG;
   const size_t B = (size_t)a->B, H = (size_t)a->H, es = elem_bytes(a->dtype);
   const Range q{a->q, B * H * a->dk * es}, k{a->k, B * H * a->dk * es};
-  const Range v{a->v, B * H * a->dv * es}, la{a->log_alpha, B * H * a->dk * 4};
+  const Range v{a->v, B * H * a->dv * es}, la{a->log_alpha, B * H * (gate_head ? 1 : a->dk) * 4};
   const Range be{a->beta, B * H * 4}, mk{a->mask, a->mask ? B : 0};
   const Range st{a->state, B * H * a->dk * a->dv * 4}, o{a->o, B * H * a->dv * es};
   if (!aligned(a->state, 16) || !aligned(a->beta, 4) || !aligned(a->log_alpha, 4))
@@ -204,6 +210,7 @@ kda_status kda_decode(const kda_decode_args *a, void *stream) {
   p.state = a->state;
   p.o = a->o;
   p.err = err;
+  p.gate_head = gate_head ? 1 : 0;
   return launch_decode(p, a->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -112,17 +112,20 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
 }
 
 // P1 reading q, k, log_alpha straight from global memory (rows of the chunk at
-// packed positions c0 .. c0+63 of head h; invalid rows count as zero).  Besides the
+// packed positions c0 .. c0+63 of head h; invalid rows count as zero; with a
+// head-wise gate log_alpha is [N, H] and every channel takes the row's value).  Besides the
 // shared tiles (Q G and K G rows of `t.qg/t.kg`, K e^{-g} in `t.kh`), it writes
 // Q G into rows 64.. of the 128-row output tile `gq` (if not null) and K e^{g_C - g}
 // into the 64-row tile `gkt` (global or shared memory, same swizzled layout), and
 // e^{g_C} into `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
 // beta_val (threads 0..63: beta of row tid, already in a register) is stored to
 // beta_out after the row loads are issued, so its latency overlaps theirs.
+template <bool GATE_HEAD>
 __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
-    float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out, int tid) {
+    float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out, int tid,
+    bool wait_bulk = false) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -135,7 +138,12 @@ __device__ __forceinline__ void decay_and_tiles_global(
     qv[i] = 0u;
     kv[i] = 0u;
     if (vr) {
-      la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
+      if (GATE_HEAD) {
+        const float gv = __ldg(log_alpha + (size_t)(c0 + qt * 16 + i) * H + h);
+        la = make_float2(gv, gv);
+      } else {
+        la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
+      }
       qv[i] = __ldg(reinterpret_cast<const unsigned int *>(q + row));
       kv[i] = __ldg(reinterpret_cast<const unsigned int *>(k + row));
     }
@@ -153,6 +161,9 @@ __device__ __forceinline__ void decay_and_tiles_global(
   part[qt][c] = t0;
   part[qt][c + 1] = t1;
   if (tid < kC) beta_out[tid] = beta_val;
+  // the tiles may still be read by bulk stores thread 0 issued earlier; the tile
+  // writes below come after this barrier
+  if (wait_bulk && tid == 0) tc::bulk_wait_read();
   __syncthreads();
   float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
 #pragma unroll

@@ -59,7 +59,7 @@ decode_kernel(DecodeParams p) {
   for (int c = tid; c < DK; c += kDecodeThreads) {
     s_k[c] = load_elem<BF16>(p.k, (size_t)bh * DK + c);
     s_q[c] = load_elem<BF16>(p.q, (size_t)bh * DK + c);
-    s_a[c] = __expf(p.log_alpha[(size_t)bh * DK + c]);
+    s_a[c] = __expf(p.log_alpha[p.gate_head ? (size_t)bh : (size_t)bh * DK + c]);
   }
   const float beta = p.beta[bh];
   __syncthreads();

@@ -35,6 +35,7 @@ struct PrefillParams {
   float *final_state;
   const SeqSpan *spans;   // NULL: spans are [cu[b], cu[b+1])
   unsigned *err;          // device error word
+  int gate_head;          // 1: log_alpha is [N, H] (one gate per token and head)
 };
 
 struct DecodeParams {
@@ -45,6 +46,7 @@ struct DecodeParams {
   float *state;
   void *o;
   unsigned *err;
+  int gate_head;          // 1: log_alpha is [B, H]
 };
 
 // Launchers (return a CUDA error code; argument checks happen before).
@@ -81,6 +83,12 @@ template <bool BF16>
 __device__ __forceinline__ void store_elem(void *base, size_t idx, float val) {
   if (BF16) reinterpret_cast<uint16_t *>(base)[idx] = f32_to_bf16_rne(val);
   else reinterpret_cast<float *>(base)[idx] = val;
+}
+
+// Offset of log_alpha for (row, head h, channel c): [rows, H, dk] or, with a
+// head-wise gate, [rows, H] (the same value for every channel).
+__device__ __forceinline__ size_t la_index(size_t row, int h, int H, int dk, int c, int gate_head) {
+  return gate_head ? row * H + h : (row * H + h) * dk + c;
 }
 
 __device__ __forceinline__ bool device_error_latched(const unsigned *err) {

@@ -96,7 +96,7 @@ prefill_simt_kernel(PrefillParams p) {
       const size_t gi = ((size_t)pos * H + h) * DK + c;
       Ks[r * KS + c] = ok ? load_elem<BF16>(p.k, gi) : 0.f;
       Qs[r * KS + c] = ok ? load_elem<BF16>(p.q, gi) : 0.f;
-      Gs[r * KS + c] = ok ? p.log_alpha[gi] : 0.f;
+      Gs[r * KS + c] = ok ? p.log_alpha[la_index(pos, h, H, DK, c, p.gate_head)] : 0.f;
     }
     for (int e = tid; e < C * kDvTile; e += kThreads) {
       const int r = e / kDvTile, j = e % kDvTile;

@@ -12,7 +12,7 @@
 // The intra kernel writes each (chunk, head) item to the workspace in the exact
 // 128-byte-swizzled shared-memory tile layout the state pass consumes, with
 // bulk (TMA) stores; the state pass streams items back with bulk loads into
-// two alternating buffers.  Workspace per item (74 752 bytes):
+// three rotating buffers.  Workspace per item (74 752 bytes):
 //   [0, 32768)      [-W ; Q G]  128 x 128 bf16 row tile
 //   [32768, 49152)  K e^{g_C-g}  64 x 128 bf16 row tile
 //   [49152, 65536)  U_v          64 rows x 128 bf16, two 64-column blocks (MN-major tile)
@@ -117,6 +117,29 @@ __device__ __forceinline__ bool row_ok(const PrefillParams &p, const SeqSpan &sp
   return pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
 }
 
+// Item -> (sequence, first row of its chunk, head): the sequence is the last b
+// with cbase[b] <= the item's global chunk index.
+struct ItemPos {
+  int b, c0, h;
+  size_t off;     // byte offset of the item in the workspace
+};
+__device__ __forceinline__ ItemPos locate_item(const PrefillParams &p, const SeqSpan *spans,
+                                               const int *cbase, int item, int h0, int Hg) {
+  const int gchunk = item / Hg;
+  int lo = 0, hi = p.num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
+  }
+  ItemPos ip;
+  ip.b = lo;
+  ip.h = h0 + item % Hg;
+  ip.c0 = spans[lo].begin + (gchunk - cbase[lo]) * kC;
+  ip.off = ((size_t)gchunk * p.H + ip.h) * ITEM_BYTES;
+  return ip;
+}
+
+template <bool GATE_HEAD>     // log_alpha [N, H] (one gate per token and head) instead of [N, H, dk]
 __global__ void __launch_bounds__(kThreadsA, 2)
 intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const SeqSpan *spans,
              const int *cbase, unsigned char *items, int h0, int Hg) {
@@ -158,17 +181,20 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   uint32_t phase = 0, vphase = 0;
   bool ok = true;
 
+  // V of an item is requested as soon as the previous item's products have read
+  // the V tile, so its copy overlaps that item's read-out and stores.
+  if (tid == 0 && (int)blockIdx.x < nitems) {
+    const ItemPos ip = locate_item(p, spans, cbase, blockIdx.x, h0, Hg);
+    mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+    tma_load_3d(sV, &vmap, 0, ip.h, ip.c0, &v_bar);
+    tma_load_3d(sV + 64 * 128, &vmap, 64, ip.h, ip.c0, &v_bar);
+  }
+  bool first = true;
   for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
-    const int gchunk = item / Hg, h = h0 + item % Hg;
-    int lo = 0, hi = p.num_seqs - 1;   // the sequence: last b with cbase[b] <= gchunk
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cbase[mid] <= gchunk) lo = mid; else hi = mid - 1;
-    }
-    const int b = lo;
-    const SeqSpan sp = spans[b];
-    const int c0 = sp.begin + (gchunk - cbase[b]) * kC;
-    unsigned char *it = items + ((size_t)gchunk * H + h) * ITEM_BYTES;
+    const ItemPos ip = locate_item(p, spans, cbase, item, h0, Hg);
+    const int h = ip.h, c0 = ip.c0;
+    const SeqSpan sp = spans[ip.b];
+    unsigned char *it = items + ip.off;
 
     float beta_val = 0.f;      // stored to shared memory inside the prep, after its loads
     if (tid < kC) {
@@ -178,11 +204,6 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
     __syncthreads();
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
-      tma_load_3d(sV, &vmap, 0, h, c0, &v_bar);
-      tma_load_3d(sV + 64 * 128, &vmap, 64, h, c0, &v_bar);
-    }
     // ---- decay products and operand tiles (global loads overlap the V copy)
     {
       prep::PrepTiles t;
@@ -190,11 +211,10 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       t.kg = base + A_QK; t.kg_R = 128; t.kg_row0 = 64;
       t.kh = base + A_KH;
       t.kt = nullptr;
-      prep::decay_and_tiles_global(reinterpret_cast<const uint16_t *>(p.q),
-                                   reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
-                                   valid_sh, t, nullptr, base + A_TS,
-                                   reinterpret_cast<float *>(it + IT_GC), part_sh, decay_sh, beta_val,
-                                   beta_sh, tid);
+      prep::decay_and_tiles_global<GATE_HEAD>(
+          reinterpret_cast<const uint16_t *>(p.q), reinterpret_cast<const uint16_t *>(p.k), p.log_alpha,
+          c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
+          decay_sh, beta_val, beta_sh, tid, !first);
     }
     fence_async_smem();
     __syncthreads();
@@ -203,6 +223,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     if (tid == 0) {
       fence_after_sync();
       const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
       for (int s = 0; s < 8; ++s)
         mma_bf16(tm + A_TM_GW, desc_kmajor(sQK, 128, 0, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
@@ -258,8 +279,10 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     if (tid == 0) {
       fence_after_sync();
       const uint32_t id = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
       for (int s = 0; s < 4; ++s)
         mma_bf16(tm + A_TM_GW, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sQK, 128, 64, s), id, s > 0);
+#pragma unroll
       for (int s = 0; s < 4; ++s)
         mma_bf16(tm + A_TM_UV, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sV, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
@@ -268,6 +291,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     phase++;
     if (!ok) break;
     fence_after_sync();
+    if (tid == 0 && item + (int)gridDim.x < nitems) {   // the V tile is free: next item's V
+      const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
+      mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+      tma_load_3d(sV, &vmap, 0, nx.h, nx.c0, &v_bar);
+      tma_load_3d(sV + 64 * 128, &vmap, 64, nx.h, nx.c0, &v_bar);
+    }
     if ((warp & 3) < 2) {
       // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> rows 0..63 of the Q G | K G
       // tile (its products are done), U_v -> the K e^{-g} region; both leave by bulk store
@@ -283,16 +312,15 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       }
     }
     fence_async_smem();
+    fence_before_sync();
     __syncthreads();
     if (tid == 0) {
       bulk_store(it + IT_WQ, base + A_QK, 64 * 128);                              // -W, block 0
       bulk_store(it + IT_WQ + 128 * 128, base + A_QK + 128 * 128, 64 * 128);      // -W, block 1
       bulk_store(it + IT_UV, base + A_KH, 64 * 256);
-      bulk_commit();
-      bulk_wait_read();      // the tiles are rewritten by the next item
+      bulk_commit();       // the next item's prep waits for these reads before it rewrites the tiles
     }
-    fence_before_sync();
-    __syncthreads();
+    first = false;
   }
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
@@ -313,7 +341,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 
 // ============================================================ state pass (B)
 // 8 compute warps + 1 producer warp.  The producer streams each chunk's item
-// into one of two buffers as soon as the products that read the buffer are
+// into one of three buffers as soon as the products that read the buffer are
 // done; the compute warps run the chain and synchronise among themselves on a
 // named barrier.  The output accumulator is double-buffered in TMEM, so a
 // chunk's output epilogue runs while the next chunk's first product is in
@@ -323,9 +351,11 @@ constexpr int kThreadsB = kComputeThreadsB + 32;
 constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
 constexpr uint32_t BUF_BYTES = 66560;
 constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
-constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES, B_UB = B_SB + 128 * 128;
+constexpr int kNBuf = 3;                 // item buffers: the producer runs up to three chunks ahead
+constexpr uint32_t B_SB = kNBuf * BUF_BYTES, B_UB = B_SB + 128 * 128;
 constexpr uint32_t B_USED = B_UB + 64 * 128;
 constexpr uint32_t B_SMEM = B_USED + 1024;
+static_assert(B_SMEM <= 232448, "state pass fits one SM's shared memory");
 constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 256;   // D1 buffers at 64 and 128
 
 __device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int tile,
@@ -351,8 +381,10 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
-  __shared__ __align__(8) uint64_t load_bar[2];
-  __shared__ __align__(8) uint64_t free_bar[2];
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ __align__(8) uint64_t o_bar;
+  __shared__ __align__(8) uint64_t load_bar[kNBuf];
+  __shared__ __align__(8) uint64_t free_bar[kNBuf];
   __shared__ int err_sh;
 
   if (device_error_latched(p.err)) return;
@@ -375,10 +407,12 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   if (warp == 0) tmem_alloc(&tmem_base_sh, B_TM_COLS);
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
-    mbar_init(&load_bar[0], 1);
-    mbar_init(&load_bar[1], 1);
-    mbar_init(&free_bar[0], 1);
-    mbar_init(&free_bar[1], 1);
+    mbar_init(&s_bar, 1);
+    mbar_init(&o_bar, 1);
+    for (int i = 0; i < kNBuf; ++i) {
+      mbar_init(&load_bar[i], 1);
+      mbar_init(&free_bar[i], 1);
+    }
     err_sh = 0;
   }
   fence_before_sync();
@@ -387,16 +421,17 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   const uint32_t tm = tmem_base_sh;
 
   if (warp == kComputeThreadsB / 32) {
-    // ---------------- producer warp: item loads, two chunks ahead of the chain
+    // ---------------- producer warp: item loads, up to three chunks ahead of the chain
     if ((tid & 31) == 0) {
       for (int j = 0; j < nch; ++j) {
-        if (j >= 2 && !mbar_wait(&free_bar[j & 1], ((j - 2) >> 1) & 1, kWaitCycles)) {
+        const int slot = j % kNBuf, use = j / kNBuf;
+        if (use > 0 && !mbar_wait(&free_bar[slot], (use - 1) & 1, kWaitCycles)) {
           atomicOr(p.err, ERR_BIT_TIMEOUT);
           break;
         }
         if (*reinterpret_cast<volatile int *>(&err_sh)) break;
-        load_item(base + ((j & 1) ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES,
-                  tile, &load_bar[j & 1]);
+        load_item(base + slot * BUF_BYTES, items + ((size_t)(cb + j) * H + h) * ITEM_BYTES, tile,
+                  &load_bar[slot]);
       }
     }
   } else {
@@ -410,23 +445,19 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       tmem_st_wait();
     }
     const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
-    uint32_t phase = 0;
+    uint32_t n_b = 0, n_s = 0, n_o = 0;   // commits issued on mma_bar / s_bar / o_bar (thread 0)
     bool ok = true;
 
-    // Chunk j: S -> bf16 operand, S *= e^{g_C}; then [-W ; Q G] S into D1[j & 1].
+    // Chunk j: S -> bf16 operand, then [-W ; Q G] S into D1[j & 1] goes out; the decayed
+    // state S *= e^{g_C} is written back to TMEM while that product runs (it only has to
+    // land before the state update of chunk j).
     auto begin_chunk = [&](int j) {
-      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
-      if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles)) err_sh = 1;
-      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
+      unsigned char *buf = base + (j % kNBuf) * BUF_BYTES;
+      if (!mbar_wait(&load_bar[j % kNBuf], (j / kNBuf) & 1, kWaitCycles)) err_sh = 1;
       float v[32];
       tmem_ld32(tm + my_cols + B_TM_S, v);
       prep::store_row32(base + B_SB, 128, lr, wg * 4, v);
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
-      tmem_st32(tm + my_cols + B_TM_S, v);
-      tmem_st_wait();
       fence_async_smem();
-      fence_before_sync();
       compute_sync();
       if (tid == 0 && !err_sh) {
         fence_after_sync();
@@ -439,18 +470,24 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
           mma_bf16(d1, a0 + (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4),
                    b0 + (uint64_t)((16 * s * 128) >> 4), id, s > 0);
         mma_commit(&mma_bar);
+        ++n_b;
       }
+      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
+      tmem_st32(tm + my_cols + B_TM_S, v);
+      tmem_st_wait();
+      fence_before_sync();
     };
 
     if (nch > 0) begin_chunk(0);
     for (int j = 0; j < nch; ++j) {
       const int c0 = sp.begin + j * kC;
-      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
+      unsigned char *buf = base + (j % kNBuf) * BUF_BYTES;
       const uint32_t sbuf = smem_u32(buf);
       const uint32_t d1 = B_TM_D1 + (uint32_t)((j & 1) * 64);
       // ---- wait for [-W S ; (Q G) S]; U = U_v - W S (lanes 0-63) -> bf16 operand
-      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
-      phase++;
+      if (!mbar_wait(&mma_bar, j & 1, kWaitCycles)) err_sh = 1;
       fence_after_sync();
       if ((warp & 3) < 2) {
         const int r = lr;
@@ -472,7 +509,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       fence_before_sync();
       compute_sync();
       if (*reinterpret_cast<volatile int *>(&err_sh)) { ok = false; break; }
-      // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
+      // ---- S += (K e^{g_C-g})^T U first (the chain), then O += [x ; M] U (rows 0-63 unused)
       if (tid == 0) {
         fence_after_sync();
         const uint32_t ido = idesc_bf16(128, 64, 0, 1);
@@ -482,18 +519,22 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         const uint64_t bu = desc_mnmajor(sUB, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
+          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
+        mma_commit(&s_bar);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
-        mma_commit(&mma_bar);
+          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
+        mma_commit(&o_bar);
+        ++n_s;
+        ++n_o;
       }
-      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
-      phase++;
+      if (!mbar_wait(&s_bar, j & 1, kWaitCycles)) err_sh = 1;
       fence_after_sync();
-      if (tid == 0) mbar_arrive(&free_bar[j & 1]);     // the products that read buffer j & 1 are done
       // ---- next chunk's first product goes out before this chunk's output epilogue
       if (j + 1 < nch) begin_chunk(j + 1);
+      if (!mbar_wait(&o_bar, j & 1, kWaitCycles)) err_sh = 1;
+      fence_after_sync();
+      if (tid == 0) mbar_arrive(&free_bar[j % kNBuf]);     // the products that read this buffer are done
       // ---- O (lanes 64-127 of D1[j & 1]) -> global
       if ((warp & 3) >= 2) {
         const int r = lr - kC;
@@ -521,8 +562,11 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       if (tid == 0) {
         err_sh = 1;
         atomicOr(p.err, ERR_BIT_TIMEOUT);
+        // every product thread 0 issued has finished before the TMEM is released
+        if (n_b > 0) mbar_wait(&mma_bar, (n_b - 1) & 1, kWaitCycles);
+        if (n_s > 0) mbar_wait(&s_bar, (n_s - 1) & 1, kWaitCycles);
+        if (n_o > 0) mbar_wait(&o_bar, (n_o - 1) & 1, kWaitCycles);
       }
-      if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
     } else if (p.final_state) {
       float v[32];
       tmem_ld32(tm + my_cols + B_TM_S, v);
@@ -533,7 +577,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     }
     if (tid == 0 && !ok) {
       // item loads the producer issued but the chain never consumed land before exit
-      for (int jj = 0; jj < nch; ++jj) mbar_wait(&load_bar[jj & 1], (jj >> 1) & 1, 20000);
+      for (int jj = 0; jj < nch; ++jj) mbar_wait(&load_bar[jj % kNBuf], (jj / kNBuf) & 1, 20000);
     }
   }
   fence_before_sync();
@@ -639,7 +683,8 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   CUtensorMap vmap;
   if (!encode_3d(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
-  e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
+  auto intra = p.gate_head ? intra_kernel<true> : intra_kernel<false>;
+  e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
   if (e != cudaSuccess) return e;
@@ -655,7 +700,7 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
     const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)hg;
     if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
     const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
-    intra_kernel<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, h0, hg);
+    intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, h0, hg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(gs->ev_a[g], s)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(gs->aux[g], gs->ev_a[g], 0)) != cudaSuccess) return e;

@@ -378,7 +378,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
 }  // namespace
 
 bool prefill_tc_supported(const PrefillParams &p, bool bf16) {
-  return bf16 && p.dk == kDK && (p.dv % kNV) == 0 && p.chunk == kC;
+  return bf16 && p.dk == kDK && (p.dv % kNV) == 0 && p.chunk == kC && !p.gate_head;
 }
 
 namespace {

@@ -9,6 +9,7 @@ Distributions (the workloads in the model description the kernels target):
   v ~ N(0, 1);
   beta = sigmoid(N(0, 1)) per (token, head), fp32;
   log_alpha = -softplus(N(-2, 1)) per (token, head, key channel), fp32;
+  head-wise gates (one per token and head): -softplus(N(-2, 1)) per (token, head);
   initial state (where one is used) ~ N(0, 0.1) (standard deviation 0.1), fp32.
 q, k and v are rounded to bf16 (round to nearest even) for bf16 workloads; the
 arrays returned here always hold float32 values, which represent bf16 values
@@ -31,7 +32,8 @@ import numpy as np
 
 SEED_BASE = 1480
 
-_STREAMS = ("q", "k", "v", "log_alpha", "beta", "state", "structure", "decode_mask")
+_STREAMS = ("q", "k", "v", "log_alpha", "beta", "state", "structure", "decode_mask",
+            "log_alpha_head")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -172,6 +174,13 @@ def token_tensors(seed: int, N: int, H: int, dk: int, dv: int, dtype: str) -> Di
     np.negative(log_alpha, out=log_alpha)
     beta = _sigmoid(_normal(seed, "beta", (N, H)))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)
+
+
+def head_gates(seed: int, rows: int, H: int) -> np.ndarray:
+    """log_alpha [rows, H] fp32 for one gate per token (or decode row) and head."""
+    la = _softplus(_normal(seed, "log_alpha_head", (rows, H), loc=-2.0))
+    np.negative(la, out=la)
+    return la
 
 
 def prefill_inputs(w: Workload) -> Dict[str, np.ndarray]:

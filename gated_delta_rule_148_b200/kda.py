@@ -28,6 +28,8 @@ KDA_ERR_DEVICE_TIMEOUT = 4
 KDA_ERR_DEVICE_CHECK = 5
 KDA_F32 = 0
 KDA_BF16 = 1
+KDA_GATE_CHANNEL = 0
+KDA_GATE_HEAD = 1
 
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
             "kda_status_string", "kda_version")
@@ -48,7 +50,7 @@ class PrefillArgs(ctypes.Structure):
                 ("pad_mask", ctypes.c_void_p), ("init_state", ctypes.c_void_p),
                 ("o", ctypes.c_void_p), ("final_state", ctypes.c_void_p),
                 ("chunk", ctypes.c_int), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("gate", ctypes.c_int)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -56,7 +58,8 @@ class DecodeArgs(ctypes.Structure):
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("q", ctypes.c_void_p),
                 ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("log_alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p),
-                ("mask", ctypes.c_void_p), ("state", ctypes.c_void_p), ("o", ctypes.c_void_p)]
+                ("mask", ctypes.c_void_p), ("state", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("gate", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -142,7 +145,14 @@ def prefill_args(q, k, v, log_alpha, beta, cu_seqlens, pad_mask=None, init_state
     a.chunk = int(chunk)
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.gate = gate_layout(log_alpha)
     return a
+
+
+def gate_layout(log_alpha) -> int:
+    """KDA_GATE_HEAD for a [rows, H] log_alpha (one gate per token and head), else
+    KDA_GATE_CHANNEL ([rows, H, dk])."""
+    return KDA_GATE_HEAD if log_alpha is not None and log_alpha.dim() == 2 else KDA_GATE_CHANNEL
 
 
 def prefill_workspace_bytes(num_seqs: int) -> int:
@@ -159,7 +169,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """KDA chunkwise prefill (kda_prefill).  Returns (o, final_state).
 
-    q, k [N,H,dk] and v [N,H,dv] bf16 or fp32; log_alpha [N,H,dk] fp32; beta [N,H] fp32;
+    q, k [N,H,dk] and v [N,H,dv] bf16 or fp32; log_alpha [N,H,dk] fp32 (per-channel gate) or
+    [N,H] fp32 (one gate per token and head); beta [N,H] fp32;
     cu_seqlens [B+1] int32; pad_mask [N] uint8 or None; init_state [B,H,dk,dv] fp32 or None.
     Outputs are allocated here when not given (torch allocates; the library does not).
     """
@@ -170,7 +181,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
     _check_cuda("q", q, shape=(N, H, dk))
     _check_cuda("k", k, dtype=q.dtype, shape=(N, H, dk))
     _check_cuda("v", v, dtype=q.dtype, shape=(N, H, dv))
-    _check_cuda("log_alpha", log_alpha, torch.float32, (N, H, dk))
+    _check_cuda("log_alpha", log_alpha, torch.float32,
+                (N, H) if gate_layout(log_alpha) == KDA_GATE_HEAD else (N, H, dk))
     _check_cuda("beta", beta, torch.float32, (N, H))
     _check_cuda("cu_seqlens", cu_seqlens, torch.int32, (B + 1,))
     _check_cuda("pad_mask", pad_mask, torch.uint8, (N,))
@@ -199,14 +211,16 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
 def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
            beta: torch.Tensor, state: torch.Tensor, mask: Optional[torch.Tensor] = None,
            o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """One KDA decode step (kda_decode); ``state`` [B,H,dk,dv] fp32 is updated in place."""
+    """One KDA decode step (kda_decode); ``state`` [B,H,dk,dv] fp32 is updated in place.
+    log_alpha is [B,H,dk] (per-channel gate) or [B,H] (one gate per row and head)."""
     lib = load()
     B, H, dk = q.shape
     dv = v.shape[2]
     _check_cuda("q", q, shape=(B, H, dk))
     _check_cuda("k", k, q.dtype, (B, H, dk))
     _check_cuda("v", v, q.dtype, (B, H, dv))
-    _check_cuda("log_alpha", log_alpha, torch.float32, (B, H, dk))
+    _check_cuda("log_alpha", log_alpha, torch.float32,
+                (B, H) if gate_layout(log_alpha) == KDA_GATE_HEAD else (B, H, dk))
     _check_cuda("beta", beta, torch.float32, (B, H))
     _check_cuda("mask", mask, torch.uint8, (B,))
     _check_cuda("state", state, torch.float32, (B, H, dk, dv))
@@ -219,6 +233,7 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.T
     a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
     a.log_alpha, a.beta, a.mask = _ptr(log_alpha), _ptr(beta), _ptr(mask)
     a.state, a.o = _ptr(state), _ptr(o)
+    a.gate = gate_layout(log_alpha)
     st = lib.kda_decode(ctypes.byref(a), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode")

@@ -58,6 +58,19 @@ typedef enum {
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
 
 /*
+ * Layout of log_alpha.  KDA_GATE_CHANNEL: one decay per key channel, [.., H, dk]
+ * (Kimi Delta Attention).  KDA_GATE_HEAD: one decay per token and head, [.., H],
+ * applied to every channel of the state: the head-wise gate of Gated DeltaNet,
+ * the coarser special case KDA refines ("Kimi Linear's 75% KV cache cut ...",
+ * theclarity.today, third paragraph; "Kimi Linear wlasnie pokonal ...",
+ * remio.ai, section "Jak Kimi Linear wykorzystuje inteligentniejsza pamiec
+ * rekurencyjna").  The result equals the per-channel operator with the gate
+ * broadcast over d_k; the head-wise layout reads 4 bytes of gate per token and
+ * head instead of 4 * dk.
+ */
+typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1 } kda_gate;
+
+/*
  * Chunkwise prefill over a packed variable-length batch.
  *
  * Fields (all device pointers, caller-owned):
@@ -66,9 +79,10 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  *   num_seqs     B >= 0 sequences; total_tokens N >= 0; H >= 1 heads;
  *   dk, dv       head dimensions, each 64 or 128.
  *   q, k         [N, H, dk]; v [N, H, dv]; 16-byte aligned.
- *   log_alpha    [N, H, dk] fp32, natural log of the forget gate; finite and
- *                <= 0 (values outside that range are not checked and give
- *                unspecified results).  16-byte aligned.
+ *   log_alpha    [N, H, dk] fp32 (gate = KDA_GATE_CHANNEL, 16-byte aligned) or
+ *                [N, H] fp32 (gate = KDA_GATE_HEAD, 4-byte aligned): natural
+ *                log of the forget gate; finite and <= 0 (values outside that
+ *                range are not checked and give unspecified results).
  *   beta         [N, H] fp32, finite.
  *   cu_seqlens   [B+1] int32: cu[0] = 0, non-decreasing, cu[B] = N; sequence b
  *                owns packed rows [cu[b], cu[b+1]).  Checked on the device
@@ -94,6 +108,9 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  *                smaller workspace selects a fused single-kernel path; a pad
  *                mask needs at least 16 bytes per sequence (rounded up to 256).
  *                May be NULL when pad_mask is NULL.
+ *   gate         layout of log_alpha (kda_gate); 0 = per channel.  With
+ *                KDA_GATE_HEAD the single-kernel tensor-core path is not used
+ *                (a small workspace selects the CUDA-core path).
  * Numerics: bf16 inputs take the tensor-core path (bf16 operands, fp32
  * accumulation, fp32 state); fp32 inputs take an fp32 CUDA-core path.  o is
  * rounded once (round to nearest even) to its dtype.
@@ -118,6 +135,7 @@ typedef struct {
   int chunk;
   void *workspace;
   size_t workspace_bytes;
+  kda_gate gate;
 } kda_prefill_args;
 
 /* Bytes of workspace for the fastest path of kda_prefill() with these
@@ -148,8 +166,8 @@ kda_status kda_prefill_noalloc(const kda_prefill_args *args, void *stream);
 
 /*
  * One decode step: one new token for each of B independent rows, all heads.
- *   q, k [B, H, dk]; v [B, H, dv] of dtype; log_alpha [B, H, dk] fp32;
- *   beta [B, H] fp32; mask [B] uint8 (1 = active, NULL = all active);
+ *   q, k [B, H, dk]; v [B, H, dv] of dtype; log_alpha [B, H, dk] fp32, or
+ *   [B, H] fp32 with gate = KDA_GATE_HEAD; beta [B, H] fp32; mask [B] uint8 (1 = active, NULL = all active);
  *   state [B, H, dk, dv] fp32, updated in place, 16-byte aligned;
  *   o [B, H, dv] of dtype, must not overlap any other argument.
  * A masked row's state is neither read nor written and its o is written as 0.
@@ -170,6 +188,7 @@ typedef struct {
   const uint8_t *mask;
   float *state;
   void *o;
+  kda_gate gate;
 } kda_decode_args;
 
 kda_status kda_decode(const kda_decode_args *args, void *stream);

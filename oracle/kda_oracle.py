@@ -34,6 +34,12 @@ Three independent formulations of the same operator:
 Masked (pad) positions: the state is not touched and the output is 0
 ("Transformers Community Reports Kimi Linear Cache Bug", ainews: pads must
 neither decay nor write the recurrent state).
+
+Head-wise gates: a log_alpha of shape [rows, H] is one decay per token and head,
+the gating of Gated DeltaNet that KDA refines per channel ("Kimi Linear's 75% KV
+cache cut ...", third paragraph; remio.ai, same section).  Diag(alpha) is then
+alpha times the identity, i.e. the per-channel operator with that value in every
+channel, which is how :func:`head_gate_channels` writes it out.
 """
 from __future__ import annotations
 
@@ -93,10 +99,21 @@ def _ptr(x):
     return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
 
 
+def head_gate_channels(log_alpha, dk: int):
+    """A head-wise gate [rows, H] as the per-channel gate [rows, H, dk] with the same
+    value in every channel; a per-channel gate is returned unchanged."""
+    la = np.asarray(log_alpha)
+    if la.ndim == 2:
+        return np.repeat(la[:, :, None], dk, axis=2)
+    return la
+
+
 def prefill(q, k, v, log_alpha, beta, cu_seqlens, pad_mask=None, init_state=None,
             nthreads: int = 0):
-    """Token-by-token fp64 prefill.  Returns (o [N,H,dv] f64, final_state [B,H,dk,dv] f64)."""
+    """Token-by-token fp64 prefill.  Returns (o [N,H,dv] f64, final_state [B,H,dk,dv] f64).
+    log_alpha is [N,H,dk] (per channel) or [N,H] (one gate per token and head)."""
     lib = _load()
+    log_alpha = head_gate_channels(log_alpha, np.shape(q)[2])
     q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
     N, H, dk = q.shape
@@ -115,8 +132,10 @@ def prefill(q, k, v, log_alpha, beta, cu_seqlens, pad_mask=None, init_state=None
 
 
 def decode(q, k, v, log_alpha, beta, state, mask=None, nthreads: int = 0):
-    """One fp64 decode step.  ``state`` [B,H,dk,dv] float64 is updated in place; returns o."""
+    """One fp64 decode step.  ``state`` [B,H,dk,dv] float64 is updated in place; returns o.
+    log_alpha is [B,H,dk] or [B,H] (one gate per row and head)."""
     lib = _load()
+    log_alpha = head_gate_channels(log_alpha, np.shape(q)[2])
     q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
     B, H, dk = q.shape
     dv = v.shape[2]

@@ -105,9 +105,14 @@ def _call(a):
     (lambda a: setattr(a, "pad_mask", BASE + 0x200000000), kda.KDA_ERR_INVALID_ARG),  # no ws
     (lambda a: (setattr(a, "final_state", a.q)), kda.KDA_ERR_INVALID_ARG),     # aliases q
     (lambda a: (setattr(a, "num_seqs", 0)), kda.KDA_ERR_INVALID_ARG),          # N>0, no seqs
+    (lambda a: setattr(a, "gate", 2), kda.KDA_ERR_INVALID_ARG),               # unknown layout
+    (lambda a: (setattr(a, "gate", kda.KDA_GATE_HEAD),                        # head gate: 4-B
+                setattr(a, "log_alpha", a.log_alpha + 2)), kda.KDA_ERR_INVALID_ARG),
+    (lambda a: (setattr(a, "gate", kda.KDA_GATE_HEAD),                        # [N, H] gate
+                setattr(a, "o", a.log_alpha + N * H * 4 - 64)), kda.KDA_ERR_INVALID_ARG),
 ], ids=["dtype", "H", "num_seqs", "dk", "dv", "chunk", "null_q", "null_o", "null_cu",
         "misaligned_q", "misaligned_la", "o_overlaps_k", "mask_without_ws", "state_aliases_q",
-        "tokens_without_seqs"])
+        "tokens_without_seqs", "gate_value", "head_gate_misaligned", "o_overlaps_head_gate"])
 def test_prefill_rejects_bad_arguments(mutate, expect):
     a = _good_prefill()
     mutate(a)
@@ -145,7 +150,9 @@ def _good_decode():
     (lambda a: setattr(a, "state", a.state + 4), kda.KDA_ERR_INVALID_ARG),
     (lambda a: setattr(a, "o", a.state + 64), kda.KDA_ERR_INVALID_ARG),
     (lambda a: setattr(a, "o", a.q + 2), kda.KDA_ERR_INVALID_ARG),
-], ids=["dtype", "dk", "null_state", "misaligned_state", "o_in_state", "o_overlaps_q"])
+    (lambda a: setattr(a, "gate", -1), kda.KDA_ERR_INVALID_ARG),
+], ids=["dtype", "dk", "null_state", "misaligned_state", "o_in_state", "o_overlaps_q",
+        "gate_value"])
 def test_decode_rejects_bad_arguments(mutate, expect):
     a = _good_decode()
     mutate(a)

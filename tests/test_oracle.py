@@ -340,3 +340,71 @@ def test_prefix_invariance_with_positive_control(T):
     leak, onset, _ = orc.prefix_audit(lambda w: variant(w, lambda *a: _leaky_chunked(*a, C)[0]),
                                       T, 1)
     assert leak and onset == C
+
+
+# ---------------------------------------------------------------- head-wise gate
+def _run_head(q, k, v, la_head, beta, S0, H=2):
+    """C oracle through its [N, H] gate entry: one sequence, the same inputs on H heads
+    (head h uses la_head * (h + 1), so a broadcast over the wrong axis shows)."""
+    T, dk = q.shape
+    rep = lambda x: np.repeat(x[:, None], H, axis=1)
+    la = np.stack([la_head * (h + 1) for h in range(H)], axis=1).astype(np.float32)
+    o, fs = orc.prefill(rep(q), rep(k), rep(v), la, rep(beta), np.array([0, T], np.int32),
+                        init_state=np.repeat(S0[None, None], H, axis=1))
+    return o, fs[0]
+
+
+def test_head_gate_zero_beta_closed_form():
+    """One gate per token and head, beta = 0: S_T = exp(sum log_alpha) S0 (a scalar per
+    head) and o_t = exp(cumsum_t) S0^T q_t."""
+    T, dk, dv = 29, 10, 7
+    q, k, v, _, _ = _one(21, T, dk, dv)
+    la = -np.abs(np.random.default_rng(22).normal(0.2, 0.1, T)).astype(np.float32)
+    S0 = np.random.default_rng(23).normal(0, 1, (dk, dv)).astype(np.float32)
+    o, S = _run_head(q, k, v, la, np.zeros(T, np.float32), S0)
+    for h in range(2):
+        G = np.cumsum(la.astype(np.float64) * (h + 1))
+        np.testing.assert_allclose(S[h], np.exp(G[-1]) * S0, rtol=1e-12, atol=1e-14)
+        o_ref = np.stack([np.exp(G[t]) * (S0.T.astype(np.float64) @ q[t]) for t in range(T)])
+        np.testing.assert_allclose(o[:, h], o_ref, rtol=1e-12, atol=1e-14)
+
+
+def test_head_gate_brute_force():
+    """Explicit transitions alpha_t (I - beta_t k_t k_t^T) (a scalar gate times the
+    identity) vs the C oracle given the [N, H] gate."""
+    rng = np.random.default_rng(31)
+    T, dk, dv = 9, 4, 3
+    q, k, v = (rng.normal(size=(T, d)).astype(np.float32) for d in (dk, dk, dv))
+    la = -np.abs(rng.normal(size=T)).astype(np.float32)
+    beta = rng.uniform(0, 1, size=T).astype(np.float32)
+    S0 = rng.normal(size=(dk, dv)).astype(np.float32)
+    o, S = _run_head(q, k, v, la, beta, S0, H=1)
+    Sx = S0.astype(np.float64)
+    for t in range(T):
+        kk = k[t].astype(np.float64)
+        A = np.exp(np.float64(la[t])) * (np.eye(dk) - np.float64(beta[t]) * np.outer(kk, kk))
+        Sx = A @ Sx + np.float64(beta[t]) * np.outer(kk, v[t].astype(np.float64))
+        np.testing.assert_allclose(o[t, 0], Sx.T @ q[t].astype(np.float64), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S[0], Sx, rtol=1e-12, atol=1e-12)
+
+
+def test_head_gate_rotation_invariance_with_positive_control():
+    """A gate that is a scalar per head commutes with any rotation R of the key space:
+    (q, k, S0) -> (R q, R k, R S0) gives S_t -> R S_t and the same o_t.  A per-channel
+    gate does not commute with R, so the same check must fail for it."""
+    T, dk, dv = 40, 8, 5
+    q, k, v, la_ch, beta = _one(41, T, dk, dv)
+    la_h = la_ch[:, 0].copy()
+    S0 = np.random.default_rng(42).normal(0, 1, (dk, dv)).astype(np.float32)
+    R, _ = np.linalg.qr(np.random.default_rng(43).normal(size=(dk, dk)))
+    rot = lambda x: (x.astype(np.float64) @ R.T).astype(np.float32)   # rows x -> R x
+    S0r = (R @ S0.astype(np.float64)).astype(np.float32)
+    o1, S1 = _run_head(q, k, v, la_h, beta, S0, H=1)
+    o2, S2 = _run_head(rot(q), rot(k), v, la_h, beta, S0r, H=1)
+    tol = 1e-5 * max(1.0, np.abs(o1).max())        # float32 rounding of the rotated inputs
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=tol)
+    np.testing.assert_allclose(S2[0], R @ S1[0], rtol=0, atol=tol)
+    # positive control: per-channel gates break the invariance
+    p1, _ = _run1(q, k, v, la_ch, beta, S0)
+    p2, _ = _run1(rot(q), rot(k), v, la_ch, beta, S0r)
+    assert np.abs(p2 - p1).max() > 100 * tol
