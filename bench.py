@@ -434,6 +434,27 @@ def main_ours(args, rank, world, device):
             "log_alpha": "[N, H] fp32", "l2": "inputs larger than L2"}
         line["gpu_launches"] += LAUNCHES_PER_PREFILL * K
         del devh
+        # ---- short convolution of q, k and v (D = H * d = 4096 each, W = 4, bf16, carried state)
+        cw = gen.conv_inputs(w.seed, [0], H * 128, 4)
+        cwt, cbias = torch.from_numpy(cw["weight"]).to(device), torch.from_numpy(cw["bias"]).to(device)
+        cst = torch.from_numpy(gen.conv_inputs(w.seed, [0], H * 128, 4)["state"]).to(device)
+        cu1 = torch.tensor([0, T], dtype=torch.int32, device=device)
+        ys = [torch.empty((T, H * 128), dtype=torch.bfloat16, device=device) for _ in range(3)]
+
+        def conv_step():
+            for i, key in enumerate(("q", "k", "v")):
+                kda.short_conv(dev[key].view(T, H * 128), cwt, cu1, bias=cbias, state_in=cst,
+                               state_out=cst, y=ys[i])
+        msc = time_loop(conv_step, K, W)
+        cbytes = 3 * (2 * T * H * 128 * 2 + 2 * 3 * H * 128 * 4 + H * 128 * 5 * 4)
+        line["short_conv"] = {
+            "workload": f"short_conv_qkv_T{T}_D{H * 128}_W4_bf16", "tokens_per_s": aggregate_rate(T, world, msc),
+            "ms": msc, "roofline": {"bound": "hbm", "achieved": cbytes / (msc / 1e3) / 1e9,
+                                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                    "frac": cbytes / (msc / 1e3) / 1e9 / pk["hbm_gbs"],
+                                    "algorithmic_bytes_per_step": cbytes}}
+        line["gpu_launches"] += 2 * 3 * K
+        del ys, cst
 
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(inp)

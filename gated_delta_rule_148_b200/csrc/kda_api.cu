@@ -215,6 +215,50 @@ kda_status kda_decode(const kda_decode_args *a, void *stream) {
              ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status kda_short_conv(const kda_conv_args *a, void *stream) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->dtype != KDA_F32 && a->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (a->num_seqs < 0 || a->total_tokens < 0 || a->D < 8 || a->D % 8 != 0) return KDA_ERR_INVALID_ARG;
+  if (a->width < 1 || a->width > 4) return KDA_ERR_UNSUPPORTED;
+  if (a->num_seqs == 0) return a->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+  if (!a->cu_seqlens || !a->weight) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 && (!a->x || !a->y)) return KDA_ERR_INVALID_ARG;
+  const size_t N = (size_t)a->total_tokens, D = (size_t)a->D, es = elem_bytes(a->dtype);
+  const size_t sbytes = (size_t)a->num_seqs * (a->width - 1) * D * 4;
+  const Range x{a->x, N * D * es}, y{a->y, N * D * es}, w{a->weight, D * a->width * 4};
+  const Range bi{a->bias, a->bias ? D * 4 : 0}, cu{a->cu_seqlens, 4 * ((size_t)a->num_seqs + 1)};
+  const Range mk{a->pad_mask, a->pad_mask ? N : 0};
+  const Range s0{a->state_in, a->state_in ? sbytes : 0}, s1{a->state_out, a->state_out ? sbytes : 0};
+  if ((a->x && !aligned(a->x, 16)) || (a->y && !aligned(a->y, 16)) || !aligned(a->weight, 4) ||
+      !aligned(a->bias, 4) || !aligned(a->cu_seqlens, 4) || !aligned(a->state_in, 16) ||
+      !aligned(a->state_out, 4))
+    return KDA_ERR_INVALID_ARG;
+  const Range inputs[] = {x, w, bi, cu, mk, s0};
+  for (const Range &r : inputs) {
+    if (overlap(y, r)) return KDA_ERR_INVALID_ARG;
+    if (overlap(s1, r) && !(r.p == s0.p && s1.p == s0.p)) return KDA_ERR_INVALID_ARG;
+  }
+  if (overlap(y, s1)) return KDA_ERR_INVALID_ARG;
+  unsigned *err = nullptr;
+  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  ConvParams p;
+  p.num_seqs = a->num_seqs;
+  p.N = a->total_tokens;
+  p.D = a->D;
+  p.W = a->width;
+  p.x = a->x;
+  p.weight = a->weight;
+  p.bias = a->bias;
+  p.cu = a->cu_seqlens;
+  p.mask = a->pad_mask;
+  p.state_in = a->state_in;
+  p.state_out = a->state_out;
+  p.y = a->y;
+  p.err = err;
+  return launch_short_conv(p, a->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_get_device_status(void *stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
   unsigned *err = nullptr;

@@ -49,6 +49,18 @@ struct DecodeParams {
   int gate_head;          // 1: log_alpha is [B, H]
 };
 
+struct ConvParams {
+  int num_seqs, N, D, W;
+  const void *x;
+  const float *weight, *bias;
+  const int32_t *cu;
+  const uint8_t *mask;
+  const float *state_in;
+  float *state_out;
+  void *y;
+  unsigned *err;
+};
+
 // Launchers (return a CUDA error code; argument checks happen before).
 cudaError_t launch_prefill_prepass(const PrefillParams &p, bool bf16, SeqSpan *spans,
                                    cudaStream_t s);
@@ -60,6 +72,7 @@ bool prefill_split_supported(const PrefillParams &p, bool bf16);
 size_t prefill_split_workspace(int N, int B, int H);
 cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
+cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {

@@ -33,7 +33,7 @@ import numpy as np
 SEED_BASE = 1480
 
 _STREAMS = ("q", "k", "v", "log_alpha", "beta", "state", "structure", "decode_mask",
-            "log_alpha_head")
+            "log_alpha_head", "conv_x", "conv_weight")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -181,6 +181,27 @@ def head_gates(seed: int, rows: int, H: int) -> np.ndarray:
     la = _softplus(_normal(seed, "log_alpha_head", (rows, H), loc=-2.0))
     np.negative(la, out=la)
     return la
+
+
+def conv_inputs(seed: int, lengths: Sequence[int], D: int, W: int, dtype: str = "bf16",
+                pad_frac: float = 0.0, state: bool = True) -> Dict[str, np.ndarray]:
+    """Inputs of one short-convolution call: x [N, D] ~ N(0, 1) (bf16-rounded for bf16),
+    weight [D, W] ~ N(0, 1/W), bias [D] ~ N(0, 0.1), cu_seqlens, pad_mask (each position
+    a pad with probability pad_frac, or None), state [B, W-1, D] ~ N(0, 1) or None."""
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    N, B = int(cu[-1]), len(lengths)
+    x = _normal(seed, "conv_x", (N, D))
+    if dtype == "bf16" and N > 0:
+        x = round_bf16(x)
+    wb = _normal(seed, "conv_weight", (D * W + D,))
+    out = dict(x=x, weight=(wb[:D * W].reshape(D, W) / np.sqrt(W)).astype(np.float32),
+               bias=(0.1 * wb[D * W:]).astype(np.float32), cu_seqlens=cu, pad_mask=None,
+               state=_normal(seed, "state", (B, W - 1, D)) if state else None)
+    if pad_frac > 0:
+        rng = _child(seed, "structure", 2)
+        out["pad_mask"] = (rng.uniform(size=N) >= pad_frac).astype(np.uint8)
+    return out
 
 
 def prefill_inputs(w: Workload) -> Dict[str, np.ndarray]:

@@ -32,7 +32,7 @@ KDA_GATE_CHANNEL = 0
 KDA_GATE_HEAD = 1
 
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
-            "kda_status_string", "kda_version")
+            "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_short_conv")
 
 
 class KdaError(RuntimeError):
@@ -60,6 +60,15 @@ class DecodeArgs(ctypes.Structure):
                 ("log_alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p),
                 ("mask", ctypes.c_void_p), ("state", ctypes.c_void_p), ("o", ctypes.c_void_p),
                 ("gate", ctypes.c_int)]
+
+
+class ConvArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("num_seqs", ctypes.c_int),
+                ("total_tokens", ctypes.c_int), ("D", ctypes.c_int), ("width", ctypes.c_int),
+                ("x", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("cu_seqlens", ctypes.c_void_p), ("pad_mask", ctypes.c_void_p),
+                ("state_in", ctypes.c_void_p), ("state_out", ctypes.c_void_p),
+                ("y", ctypes.c_void_p)]
 
 
 def library_path() -> str:
@@ -238,6 +247,39 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.T
     if st != KDA_OK:
         raise KdaError(st, "kda_decode")
     return o
+
+
+def short_conv(x: torch.Tensor, weight: torch.Tensor, cu_seqlens: torch.Tensor,
+               bias: Optional[torch.Tensor] = None, pad_mask: Optional[torch.Tensor] = None,
+               state_in: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+               y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Padding-correct short causal convolution (kda_short_conv).  x [N,D] bf16 or fp32,
+    weight [D,W] fp32, bias [D] fp32, state_in/state_out [B,W-1,D] fp32 (may be the same
+    tensor).  Returns y [N,D] (allocated here when not given)."""
+    lib = load()
+    N, D = x.shape
+    W = weight.shape[1]
+    B = cu_seqlens.numel() - 1
+    _check_cuda("x", x, shape=(N, D))
+    _check_cuda("weight", weight, torch.float32, (D, W))
+    _check_cuda("bias", bias, torch.float32, (D,))
+    _check_cuda("cu_seqlens", cu_seqlens, torch.int32, (B + 1,))
+    _check_cuda("pad_mask", pad_mask, torch.uint8, (N,))
+    _check_cuda("state_in", state_in, torch.float32, (B, W - 1, D))
+    _check_cuda("state_out", state_out, torch.float32, (B, W - 1, D))
+    if y is None:
+        y = torch.empty((N, D), dtype=x.dtype, device=x.device)
+    _check_cuda("y", y, x.dtype, (N, D))
+    a = ConvArgs()
+    a.dtype = _dtype_code(x)
+    a.num_seqs, a.total_tokens, a.D, a.width = B, N, D, W
+    a.x, a.weight, a.bias = _ptr(x), _ptr(weight), _ptr(bias)
+    a.cu_seqlens, a.pad_mask = _ptr(cu_seqlens), _ptr(pad_mask)
+    a.state_in, a.state_out, a.y = _ptr(state_in), _ptr(state_out), _ptr(y)
+    st = lib.kda_short_conv(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_short_conv")
+    return y
 
 
 def get_device_status(stream=None) -> int:

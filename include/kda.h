@@ -193,6 +193,51 @@ typedef struct {
 
 kda_status kda_decode(const kda_decode_args *args, void *stream);
 
+/*
+ * Short causal convolution of the layer's inputs, padding-correct, with a
+ * carried convolution state (the convolution window a cached continuation
+ * keeps besides the recurrent state: "Transformers Community Reports Kimi
+ * Linear Cache Bug", ainews, paragraphs on the reproduction and the follow-up
+ * investigation -- padded entries must neither enter the window nor advance the
+ * convolution state).  Depthwise, per channel c of sequence b, over the
+ * sequence's VALID positions only:
+ *   y_t[c] = bias[c] + sum_{i<W} weight[c*W + i] * u_i[c]
+ * where u_0 .. u_{W-2} are the W-1 valid inputs before t (oldest first) and
+ * u_{W-1} = x_t; before the sequence's first valid inputs the window holds the
+ * incoming state.  A pad position has y = 0 and changes nothing.  No activation
+ * is applied.  Fields (device pointers, caller-owned):
+ *   dtype        type of x and y (KDA_BF16 or KDA_F32); everything else fp32.
+ *   num_seqs     B >= 0; total_tokens N >= 0; D >= 8 channels, a multiple of 8.
+ *   width        W in 1..4.
+ *   x, y         [N, D], 16-byte aligned; y must not overlap any input.
+ *   weight       [D, W]; bias [D] or NULL (zeros).
+ *   cu_seqlens   [B+1] int32, as for kda_prefill (checked on the device).
+ *   pad_mask     [N] uint8 (1 = valid) or NULL.
+ *   state_in     [B, W-1, D] (oldest row first), 16-byte aligned, or NULL (zeros).
+ *   state_out    [B, W-1, D]: the last W-1 valid inputs of each sequence
+ *                (completed from state_in when the sequence has fewer), or
+ *                NULL.  May be the same pointer as state_in (in-place update),
+ *                may not otherwise overlap an input.
+ * A decode step is a call with one token per sequence.  Allocates nothing.
+ */
+typedef struct {
+  kda_dtype dtype;
+  int num_seqs;
+  int total_tokens;
+  int D;
+  int width;
+  const void *x;
+  const float *weight;
+  const float *bias;
+  const int32_t *cu_seqlens;
+  const uint8_t *pad_mask;
+  const float *state_in;
+  float *state_out;
+  void *y;
+} kda_conv_args;
+
+kda_status kda_short_conv(const kda_conv_args *args, void *stream);
+
 /* Synchronise `stream`, then return and clear the error latched on the
  * current device by earlier kernels (KDA_OK if none). */
 kda_status kda_get_device_status(void *stream);

@@ -236,3 +236,68 @@ def prefix_audit(run, T: int, perturb, tol: float = 0.0):
     d = d.reshape(T - 1, -1).max(axis=1)
     bad = np.nonzero(d > tol)[0]
     return (len(bad) > 0, (int(bad[0]) if len(bad) else None), d)
+
+
+# ----------------------------------------------------------------------------
+# Short causal convolution (the layer's convolution window, padding-correct)
+# ----------------------------------------------------------------------------
+def short_conv(x, weight, bias, cu_seqlens, pad_mask=None, state_in=None):
+    """Depthwise causal convolution over each sequence's VALID positions, written as
+    the sliding window it is: the window holds the W-1 previous valid inputs (the
+    incoming state before the sequence's first ones); at a valid position the output
+    is bias + sum_i weight[:, i] * u_i over the window followed by x_t, and x_t then
+    enters the window; a pad position outputs 0 and leaves the window alone
+    ("Transformers Community Reports Kimi Linear Cache Bug", ainews: padded entries
+    must not enter the convolution window nor advance the convolution state).
+    x [N, D]; weight [D, W]; bias [D] or None; state_in [B, W-1, D] or None.
+    Returns (y [N, D] float64, state_out [B, W-1, D] float64)."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64)
+    N, D = x.shape
+    W = w.shape[1]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = len(cu) - 1
+    b0 = np.zeros(D) if bias is None else np.asarray(bias, dtype=np.float64)
+    y = np.zeros((N, D))
+    s_out = np.zeros((B, W - 1, D))
+    for b in range(B):
+        window = [np.zeros(D) if state_in is None else np.asarray(state_in[b, j], dtype=np.float64)
+                  for j in range(W - 1)]
+        for t in range(int(cu[b]), int(cu[b + 1])):
+            if pad_mask is not None and pad_mask[t] == 0:
+                continue
+            u = window + [x[t]]
+            y[t] = b0 + sum(w[:, i] * u[i] for i in range(W))
+            window = u[1:]
+        for j in range(W - 1):
+            s_out[b, j] = window[j]
+    return y, s_out
+
+
+def short_conv_at(x, weight, bias, cu_seqlens, positions, pad_mask=None, state_in=None):
+    """Outputs of short_conv at the given packed positions only (for full-size checks):
+    each one from its own window, found by walking back over the pad mask.
+    Returns y [len(positions), D] float64."""
+    w = np.asarray(weight, dtype=np.float64)
+    D, W = w.shape
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    b0 = np.zeros(D) if bias is None else np.asarray(bias, dtype=np.float64)
+    out = np.zeros((len(positions), D))
+    for n, t in enumerate(positions):
+        t = int(t)
+        if pad_mask is not None and pad_mask[t] == 0:
+            continue
+        b = int(np.searchsorted(cu, t, side="right")) - 1
+        prev = []                      # newest first
+        s = t - 1
+        while s >= cu[b] and len(prev) < W - 1:
+            if pad_mask is None or pad_mask[s] != 0:
+                prev.append(np.asarray(x[s], dtype=np.float64))
+            s -= 1
+        j = W - 2                      # newest state row first
+        while len(prev) < W - 1:
+            prev.append(np.zeros(D) if state_in is None else np.asarray(state_in[b, j], np.float64))
+            j -= 1
+        u = prev[::-1] + [np.asarray(x[t], dtype=np.float64)]
+        out[n] = b0 + sum(w[:, i] * u[i] for i in range(W))
+    return out

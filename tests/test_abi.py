@@ -40,6 +40,7 @@ def test_struct_layout_matches_header(tmp_path):
     prog = tmp_path / "layout.c"
     fields_p = [f[0] for f in kda.PrefillArgs._fields_]
     fields_d = [f[0] for f in kda.DecodeArgs._fields_]
+    fields_c = [f[0] for f in kda.ConvArgs._fields_]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "kda.h"', 'int main(void){']
     lines.append('printf("P %zu\\n", sizeof(kda_prefill_args));')
     for f in fields_p:
@@ -47,6 +48,9 @@ def test_struct_layout_matches_header(tmp_path):
     lines.append('printf("D %zu\\n", sizeof(kda_decode_args));')
     for f in fields_d:
         lines.append(f'printf("D.{f} %zu\\n", offsetof(kda_decode_args, {f}));')
+    lines.append('printf("C %zu\\n", sizeof(kda_conv_args));')
+    for f in fields_c:
+        lines.append(f'printf("C.{f} %zu\\n", offsetof(kda_conv_args, {f}));')
     lines.append("return 0;}")
     prog.write_text("\n".join(lines))
     exe = tmp_path / "layout"
@@ -59,6 +63,9 @@ def test_struct_layout_matches_header(tmp_path):
         assert int(got[f"P.{f}"]) == getattr(kda.PrefillArgs, f).offset, f
     for f in fields_d:
         assert int(got[f"D.{f}"]) == getattr(kda.DecodeArgs, f).offset, f
+    assert int(got["C"]) == ctypes.sizeof(kda.ConvArgs)
+    for f in fields_c:
+        assert int(got[f"C.{f}"]) == getattr(kda.ConvArgs, f).offset, f
 
 
 def test_status_strings():
@@ -164,3 +171,30 @@ def test_binding_refuses_host_tensors():
     x = torch.zeros(4, 1, 64)
     with pytest.raises(TypeError):
         kda.decode(x, x, x, x, torch.zeros(4, 1), torch.zeros(4, 1, 64, 64))
+
+
+def _good_conv():
+    a = kda.ConvArgs()
+    a.dtype, a.num_seqs, a.total_tokens, a.D, a.width = kda.KDA_BF16, 2, 256, 64, 4
+    a.x, a.y = BASE, BASE + 0x100000
+    a.weight, a.bias, a.cu_seqlens = BASE + 0x200000, BASE + 0x210000, BASE + 0x220000
+    a.state_in, a.state_out = BASE + 0x230000, BASE + 0x240000
+    return a
+
+
+@pytest.mark.parametrize("mutate,expect", [
+    (lambda a: setattr(a, "dtype", 5), kda.KDA_ERR_INVALID_ARG),
+    (lambda a: setattr(a, "D", 60), kda.KDA_ERR_INVALID_ARG),           # not a multiple of 8
+    (lambda a: setattr(a, "width", 5), kda.KDA_ERR_UNSUPPORTED),
+    (lambda a: setattr(a, "width", 0), kda.KDA_ERR_UNSUPPORTED),
+    (lambda a: setattr(a, "weight", None), kda.KDA_ERR_INVALID_ARG),
+    (lambda a: setattr(a, "x", BASE + 4), kda.KDA_ERR_INVALID_ARG),      # misaligned
+    (lambda a: setattr(a, "y", a.x + 64), kda.KDA_ERR_INVALID_ARG),      # y overlaps x
+    (lambda a: setattr(a, "state_out", a.x), kda.KDA_ERR_INVALID_ARG),   # state over x
+    (lambda a: setattr(a, "num_seqs", 0), kda.KDA_ERR_INVALID_ARG),      # tokens, no seqs
+], ids=["dtype", "D", "width5", "width0", "null_weight", "misaligned_x", "y_overlaps_x",
+        "state_over_x", "tokens_without_seqs"])
+def test_conv_rejects_bad_arguments(mutate, expect):
+    a = _good_conv()
+    mutate(a)
+    assert kda.load().kda_short_conv(ctypes.byref(a), None) == expect

@@ -408,3 +408,90 @@ def test_head_gate_rotation_invariance_with_positive_control():
     p1, _ = _run1(q, k, v, la_ch, beta, S0)
     p2, _ = _run1(rot(q), rot(k), v, la_ch, beta, S0r)
     assert np.abs(p2 - p1).max() > 100 * tol
+
+
+# ---------------------------------------------------------------- short convolution
+def _conv_case(seed, lengths, D, W, pads=0.0, state=True):
+    rng = np.random.default_rng(seed)
+    cu = np.zeros(len(lengths) + 1, np.int64)
+    cu[1:] = np.cumsum(lengths)
+    N = int(cu[-1])
+    x = rng.normal(size=(N, D)).astype(np.float32)
+    w = rng.normal(size=(D, W)).astype(np.float32)
+    b = rng.normal(size=D).astype(np.float32)
+    m = None if pads == 0 else (rng.uniform(size=N) >= pads).astype(np.uint8)
+    s = rng.normal(size=(len(lengths), W - 1, D)).astype(np.float32) if state else None
+    return x, w, b, cu, m, s
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 4])
+def test_conv_unpadded_equals_numpy_convolve(W):
+    """No pads, zero state: each channel is numpy's full convolution with the reversed
+    weights, truncated to the sequence (the causal window), plus the bias."""
+    x, w, b, cu, _, _ = _conv_case(61, [37, 5, 64], 6, W, state=False)
+    y, s = orc.short_conv(x, w, b, cu)
+    for i in range(len(cu) - 1):
+        a, e = int(cu[i]), int(cu[i + 1])
+        for c in range(6):
+            ref = np.convolve(x[a:e, c].astype(np.float64), w[c, ::-1].astype(np.float64))[:e - a] + b[c]
+            np.testing.assert_allclose(y[a:e, c], ref, rtol=1e-12, atol=1e-12)
+        # final state: the last W-1 inputs (zeros in front when the sequence is short)
+        tail = np.concatenate([np.zeros((W - 1, 6)), x[a:e].astype(np.float64)])[-(W - 1):] if W > 1 else np.zeros((0, 6))
+        np.testing.assert_array_equal(s[i], tail)
+
+
+def test_conv_padding_equals_unpadded_run_with_positive_control():
+    """Pads anywhere (edges and inside) give the unpadded run's outputs at the valid
+    positions, 0 at the pads, and the same final state; a window that lets pads in
+    (the reported bug) does not."""
+    x, w, b, cu, m, s = _conv_case(62, [40, 3, 70], 5, 4, pads=0.3)
+    m[38], m[39] = 0, 1            # a pad inside sequence 0's final window
+    y, so = orc.short_conv(x, w, b, cu, m, s)
+    keep = m.astype(bool)
+    lens = [int(keep[cu[i]:cu[i + 1]].sum()) for i in range(len(cu) - 1)]
+    cu2 = np.concatenate([[0], np.cumsum(lens)])
+    y2, so2 = orc.short_conv(x[keep], w, b, cu2, None, s)
+    np.testing.assert_array_equal(y[keep], y2)
+    assert np.all(y[~keep] == 0.0)
+    np.testing.assert_array_equal(so, so2)
+    # positive control: pads as zero inputs inside the window
+    xz = x.copy()
+    xz[~keep] = 0.0
+    y3, so3 = orc.short_conv(xz, w, b, cu, None, s)
+    assert np.abs(y3[keep] - y2).max() > 1e-3 and np.abs(so3 - so2).max() > 1e-3
+
+
+def test_conv_split_sequence_with_carried_state():
+    """Two calls, the second starting from the first's state, equal one call."""
+    x, w, b, _, m, s = _conv_case(63, [90], 7, 3, pads=0.2)
+    cu = np.array([0, 90])
+    y, so = orc.short_conv(x, w, b, cu, m, s)
+    for cut in (1, 2, 45, 89):
+        ya, sa = orc.short_conv(x[:cut], w, b, [0, cut], m[:cut], s)
+        yb, sb = orc.short_conv(x[cut:], w, b, [0, 90 - cut], m[cut:], sa)
+        np.testing.assert_allclose(np.concatenate([ya, yb]), y, rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(sb, so)
+
+
+def test_conv_short_sequences_shift_the_state():
+    """A sequence with n < W-1 valid inputs: the new state is the old one shifted by n
+    rows with the n inputs appended; with only pads it is unchanged."""
+    W, D = 4, 3
+    rng = np.random.default_rng(64)
+    s = rng.normal(size=(3, W - 1, D))
+    x = rng.normal(size=(4, D))
+    m = np.array([1, 0, 0, 1], np.uint8)         # seq0: 1 valid; seq1: 1 pad; seq2: 1 valid
+    cu = [0, 1, 2, 4]
+    y, so = orc.short_conv(x, np.ones((D, W)), None, cu, m, s)
+    np.testing.assert_array_equal(so[0], np.concatenate([s[0][1:], x[0:1]]))
+    np.testing.assert_array_equal(so[1], s[1])
+    np.testing.assert_array_equal(so[2], np.concatenate([s[2][1:], x[3:4]]))
+    np.testing.assert_allclose(y[0], s[0].sum(0) + x[0], rtol=1e-12)   # all-ones weights
+    assert np.all(y[1] == 0) and np.all(y[2] == 0)
+
+
+def test_conv_sampled_positions_match_window_form():
+    x, w, b, cu, m, s = _conv_case(65, [33, 1, 120], 4, 4, pads=0.25)
+    y, _ = orc.short_conv(x, w, b, cu, m, s)
+    pos = np.array([0, 1, 5, 33, 34, 35, 100, 153])
+    np.testing.assert_allclose(orc.short_conv_at(x, w, b, cu, pos, m, s), y[pos], rtol=0, atol=1e-12)
