@@ -15,8 +15,8 @@
 // conv_state [B, W-1, D] fp32.  The operation is HBM-bound (read x, write y):
 // kernel A gives each CTA 256 packed positions and up to 2048 channels; the pad
 // mask of those positions is compacted once per CTA (warp ballots) into the list
-// of valid rows, and each thread forms outputs for 8 consecutive channels with
-// 16-byte loads (the W-fold re-reads of x hit L1).  Kernel B writes the new
+// of valid rows, and each thread walks those rows for its 8 consecutive channels
+// with the window in registers (one 16-byte load and one store per row).  Kernel B writes the new
 // state after kernel A, one thread per (sequence, channel), so conv_state may be
 // updated in place.
 #include "kda_internal.cuh"
@@ -24,9 +24,9 @@
 namespace kda {
 namespace conv {
 
-constexpr int kSeg = 256;          // packed positions per CTA
-constexpr int kChan = 2048;        // channels per CTA
+constexpr int kSeg = 256;            // packed positions per CTA
 constexpr int kThreads = 256;
+constexpr int kChan = 8 * kThreads;  // channels per CTA (8 per thread)
 constexpr int kMaxW = 4;
 
 // Source of a window entry: a packed position (>= 0) or state row j (encoded -1 - j).
@@ -90,11 +90,11 @@ __device__ __forceinline__ void store8(void *y, size_t row, int D, int c, const 
 
 
 // Kernel A: outputs of packed positions [kSeg*blockIdx.x, +kSeg), channels
-// [kChan*blockIdx.y, +kChan).
+// [kChan*blockIdx.y, +kChan).  Thread t owns channels 8t .. 8t+7 and walks the
+// CTA's valid rows in order with the window in registers, so each x row is read
+// once; the 16-byte loads of one row are coalesced across the CTA's threads.
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
-  __shared__ float w_sh[kMaxW][kChan];
-  __shared__ float b_sh[kChan];
   __shared__ int vpos[kSeg];
   __shared__ int wcnt[kThreads / 32];
   __shared__ Hist hist_sh;
@@ -109,9 +109,16 @@ __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
     if (tid == 0) bad |= p.cu[0] != 0 || p.cu[B] != p.N;
     if (bad) atomicOr(p.err, ERR_BIT_CHECK);
   }
-  for (int e = tid; e < nch; e += kThreads) {
-    for (int i = 0; i < W; ++i) w_sh[i][e] = p.weight[(size_t)(c_lo + e) * W + i];
-    b_sh[e] = p.bias ? p.bias[c_lo + e] : 0.f;
+  // this thread's channels and their taps
+  const int cl = tid * 8, c = c_lo + cl;
+  const bool mine = cl < nch;
+  float wt[kMaxW - 1][8], wx[8], bz[8];      // window taps, the current row's tap, bias
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    bz[j] = (mine && p.bias) ? p.bias[c + j] : 0.f;
+    wx[j] = mine ? p.weight[(size_t)(c + j) * W + (W - 1)] : 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxW - 1; ++i) wt[i][j] = (mine && i < W - 1) ? p.weight[(size_t)(c + j) * W + i] : 0.f;
   }
   // first sequence with cu[b + 1] > s0
   int lo = 0, hi = B - 1;
@@ -119,7 +126,6 @@ __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
     const int mid = (lo + hi) >> 1;
     if (p.cu[mid + 1] <= s0) lo = mid + 1; else hi = mid;
   }
-  const int nchunks = nch / 8;
   for (int b = lo; b < B && p.cu[b] < s1; ++b) {
     const int sb = max(p.cu[b], 0);
     const int a = max(s0, sb), e = min(s1, p.cu[b + 1]);
@@ -139,44 +145,52 @@ __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
     }
     if (ok) vpos[before + __popc(bits & ((1u << lane) - 1u))] = pos;
     __syncthreads();
-    // ---- valid rows: y = bias + sum_i w_i u_i
-    const Hist hs = hist_sh;
-    for (int it = tid; it < nvalid * nchunks; it += kThreads) {
-      const int m = it / nchunks, cl = (it - m * nchunks) * 8;
-      float acc[8];
+    if (mine) {
+      // ---- the window before the first valid row (oldest first)
+      float win[kMaxW - 1][8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = b_sh[cl + j];
+      for (int j = 0; j < kMaxW - 1; ++j) {
 #pragma unroll
-      for (int i = 0; i < kMaxW; ++i) {
-        if (i >= W) break;
-        const int kidx = m + i - (W - 1);        // compacted index of u_i
-        float v[8];
-        bool have = true;
-        if (kidx >= 0) {
-          load8<BF16>(p.x, (size_t)vpos[kidx], D, c_lo + cl, v);
-        } else {
-          const int src = hs.src[W - 1 + kidx];
-          if (src >= 0) {
-            load8<BF16>(p.x, (size_t)src, D, c_lo + cl, v);
-          } else if (p.state_in) {
-            load8<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c_lo + cl, v);
-          } else {
-            have = false;
-          }
-        }
-        if (have) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = fmaf(w_sh[i][cl + j], v[j], acc[j]);
+        for (int q = 0; q < 8; ++q) win[j][q] = 0.f;
+        if (j < W - 1) {
+          const int src = hist_sh.src[j];
+          if (src >= 0) load8<BF16>(p.x, (size_t)src, D, c, win[j]);
+          else if (p.state_in) load8<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c, win[j]);
         }
       }
-      store8<BF16>(p.y, (size_t)vpos[m], D, c_lo + cl, acc);
-    }
-    // ---- pads: y = 0
-    if (p.mask != nullptr && nvalid < e - a) {
-      const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int it = tid; it < (e - a) * nchunks; it += kThreads) {
-        const int r = a + it / nchunks, cl = (it % nchunks) * 8;
-        if (p.mask[r] == 0) store8<BF16>(p.y, (size_t)r, D, c_lo + cl, z);
+      // ---- walk the valid rows
+#pragma unroll 2
+      for (int m = 0; m < nvalid; ++m) {
+        const size_t row = (size_t)vpos[m];
+        float xv[8], acc[8];
+        load8<BF16>(p.x, row, D, c, xv);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(wx[q], xv[q], bz[q]);
+        // taps: u_i = win[i] for i < W-1 (zero taps beyond), u_{W-1} = x_t
+#pragma unroll
+        for (int i = 0; i < kMaxW - 1; ++i)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] = fmaf(wt[i][q], win[i][q], acc[q]);
+        store8<BF16>(p.y, row, D, c, acc);
+        // shift: the newest of the W-1 slots becomes x_t
+#pragma unroll
+        for (int j = 0; j < kMaxW - 2; ++j)
+          if (j + 1 < W - 1) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) win[j][q] = win[j + 1][q];
+          }
+#pragma unroll
+        for (int j = 0; j < kMaxW - 1; ++j)
+          if (j == W - 2) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) win[j][q] = xv[q];
+          }
+      }
+      // ---- pads: y = 0
+      if (p.mask != nullptr && nvalid < e - a) {
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int r = a; r < e; ++r)
+          if (p.mask[r] == 0) store8<BF16>(p.y, (size_t)r, D, c, z);
       }
     }
     __syncthreads();   // vpos, wcnt and hist_sh are rewritten by the next sequence

@@ -12,7 +12,7 @@
 // The intra kernel writes each (chunk, head) item to the workspace in the exact
 // 128-byte-swizzled shared-memory tile layout the state pass consumes, with
 // bulk (TMA) stores; the state pass streams items back with bulk loads into
-// three rotating buffers.  Workspace per item (74 752 bytes):
+// two alternating buffers.  Workspace per item (74 752 bytes):
 //   [0, 32768)      [-W ; Q G]  128 x 128 bf16 row tile
 //   [32768, 49152)  K e^{g_C-g}  64 x 128 bf16 row tile
 //   [49152, 65536)  U_v          64 rows x 128 bf16, two 64-column blocks (MN-major tile)
@@ -341,7 +341,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 
 // ============================================================ state pass (B)
 // 8 compute warps + 1 producer warp.  The producer streams each chunk's item
-// into one of three buffers as soon as the products that read the buffer are
+// into one of two buffers as soon as the products that read the buffer are
 // done; the compute warps run the chain and synchronise among themselves on a
 // named barrier.  The output accumulator is double-buffered in TMEM, so a
 // chunk's output epilogue runs while the next chunk's first product is in
@@ -351,11 +351,9 @@ constexpr int kThreadsB = kComputeThreadsB + 32;
 constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
 constexpr uint32_t BUF_BYTES = 66560;
 constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
-constexpr int kNBuf = 3;                 // item buffers: the producer runs up to three chunks ahead
-constexpr uint32_t B_SB = kNBuf * BUF_BYTES, B_UB = B_SB + 128 * 128;
+constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES, B_UB = B_SB + 128 * 128;
 constexpr uint32_t B_USED = B_UB + 64 * 128;
 constexpr uint32_t B_SMEM = B_USED + 1024;
-static_assert(B_SMEM <= 232448, "state pass fits one SM's shared memory");
 constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 256;   // D1 buffers at 64 and 128
 
 __device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int tile,
@@ -381,10 +379,8 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
-  __shared__ __align__(8) uint64_t s_bar;
-  __shared__ __align__(8) uint64_t o_bar;
-  __shared__ __align__(8) uint64_t load_bar[kNBuf];
-  __shared__ __align__(8) uint64_t free_bar[kNBuf];
+  __shared__ __align__(8) uint64_t load_bar[2];
+  __shared__ __align__(8) uint64_t free_bar[2];
   __shared__ int err_sh;
 
   if (device_error_latched(p.err)) return;
@@ -407,12 +403,10 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   if (warp == 0) tmem_alloc(&tmem_base_sh, B_TM_COLS);
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
-    mbar_init(&s_bar, 1);
-    mbar_init(&o_bar, 1);
-    for (int i = 0; i < kNBuf; ++i) {
-      mbar_init(&load_bar[i], 1);
-      mbar_init(&free_bar[i], 1);
-    }
+    mbar_init(&load_bar[0], 1);
+    mbar_init(&load_bar[1], 1);
+    mbar_init(&free_bar[0], 1);
+    mbar_init(&free_bar[1], 1);
     err_sh = 0;
   }
   fence_before_sync();
@@ -421,17 +415,16 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   const uint32_t tm = tmem_base_sh;
 
   if (warp == kComputeThreadsB / 32) {
-    // ---------------- producer warp: item loads, up to three chunks ahead of the chain
+    // ---------------- producer warp: item loads, two chunks ahead of the chain
     if ((tid & 31) == 0) {
       for (int j = 0; j < nch; ++j) {
-        const int slot = j % kNBuf, use = j / kNBuf;
-        if (use > 0 && !mbar_wait(&free_bar[slot], (use - 1) & 1, kWaitCycles)) {
+        if (j >= 2 && !mbar_wait(&free_bar[j & 1], ((j - 2) >> 1) & 1, kWaitCycles)) {
           atomicOr(p.err, ERR_BIT_TIMEOUT);
           break;
         }
         if (*reinterpret_cast<volatile int *>(&err_sh)) break;
-        load_item(base + slot * BUF_BYTES, items + ((size_t)(cb + j) * H + h) * ITEM_BYTES, tile,
-                  &load_bar[slot]);
+        load_item(base + ((j & 1) ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES,
+                  tile, &load_bar[j & 1]);
       }
     }
   } else {
@@ -445,19 +438,23 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       tmem_st_wait();
     }
     const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
-    uint32_t n_b = 0, n_s = 0, n_o = 0;   // commits issued on mma_bar / s_bar / o_bar (thread 0)
+    uint32_t phase = 0;
     bool ok = true;
 
-    // Chunk j: S -> bf16 operand, then [-W ; Q G] S into D1[j & 1] goes out; the decayed
-    // state S *= e^{g_C} is written back to TMEM while that product runs (it only has to
-    // land before the state update of chunk j).
+    // Chunk j: S -> bf16 operand, S *= e^{g_C}; then [-W ; Q G] S into D1[j & 1].
     auto begin_chunk = [&](int j) {
-      unsigned char *buf = base + (j % kNBuf) * BUF_BYTES;
-      if (!mbar_wait(&load_bar[j % kNBuf], (j / kNBuf) & 1, kWaitCycles)) err_sh = 1;
+      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
+      if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles)) err_sh = 1;
+      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
       float v[32];
       tmem_ld32(tm + my_cols + B_TM_S, v);
       prep::store_row32(base + B_SB, 128, lr, wg * 4, v);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
+      tmem_st32(tm + my_cols + B_TM_S, v);
+      tmem_st_wait();
       fence_async_smem();
+      fence_before_sync();
       compute_sync();
       if (tid == 0 && !err_sh) {
         fence_after_sync();
@@ -470,24 +467,18 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
           mma_bf16(d1, a0 + (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4),
                    b0 + (uint64_t)((16 * s * 128) >> 4), id, s > 0);
         mma_commit(&mma_bar);
-        ++n_b;
       }
-      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
-      tmem_st32(tm + my_cols + B_TM_S, v);
-      tmem_st_wait();
-      fence_before_sync();
     };
 
     if (nch > 0) begin_chunk(0);
     for (int j = 0; j < nch; ++j) {
       const int c0 = sp.begin + j * kC;
-      unsigned char *buf = base + (j % kNBuf) * BUF_BYTES;
+      unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
       const uint32_t sbuf = smem_u32(buf);
       const uint32_t d1 = B_TM_D1 + (uint32_t)((j & 1) * 64);
       // ---- wait for [-W S ; (Q G) S]; U = U_v - W S (lanes 0-63) -> bf16 operand
-      if (!mbar_wait(&mma_bar, j & 1, kWaitCycles)) err_sh = 1;
+      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      phase++;
       fence_after_sync();
       if ((warp & 3) < 2) {
         const int r = lr;
@@ -509,7 +500,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       fence_before_sync();
       compute_sync();
       if (*reinterpret_cast<volatile int *>(&err_sh)) { ok = false; break; }
-      // ---- S += (K e^{g_C-g})^T U first (the chain), then O += [x ; M] U (rows 0-63 unused)
+      // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
       if (tid == 0) {
         fence_after_sync();
         const uint32_t ido = idesc_bf16(128, 64, 0, 1);
@@ -519,22 +510,18 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         const uint64_t bu = desc_mnmajor(sUB, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
-        mma_commit(&s_bar);
+          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
-        mma_commit(&o_bar);
-        ++n_s;
-        ++n_o;
+          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
+        mma_commit(&mma_bar);
       }
-      if (!mbar_wait(&s_bar, j & 1, kWaitCycles)) err_sh = 1;
+      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      phase++;
       fence_after_sync();
+      if (tid == 0) mbar_arrive(&free_bar[j & 1]);     // the products that read buffer j & 1 are done
       // ---- next chunk's first product goes out before this chunk's output epilogue
       if (j + 1 < nch) begin_chunk(j + 1);
-      if (!mbar_wait(&o_bar, j & 1, kWaitCycles)) err_sh = 1;
-      fence_after_sync();
-      if (tid == 0) mbar_arrive(&free_bar[j % kNBuf]);     // the products that read this buffer are done
       // ---- O (lanes 64-127 of D1[j & 1]) -> global
       if ((warp & 3) >= 2) {
         const int r = lr - kC;
@@ -562,11 +549,8 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       if (tid == 0) {
         err_sh = 1;
         atomicOr(p.err, ERR_BIT_TIMEOUT);
-        // every product thread 0 issued has finished before the TMEM is released
-        if (n_b > 0) mbar_wait(&mma_bar, (n_b - 1) & 1, kWaitCycles);
-        if (n_s > 0) mbar_wait(&s_bar, (n_s - 1) & 1, kWaitCycles);
-        if (n_o > 0) mbar_wait(&o_bar, (n_o - 1) & 1, kWaitCycles);
       }
+      if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
     } else if (p.final_state) {
       float v[32];
       tmem_ld32(tm + my_cols + B_TM_S, v);
@@ -577,7 +561,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     }
     if (tid == 0 && !ok) {
       // item loads the producer issued but the chain never consumed land before exit
-      for (int jj = 0; jj < nch; ++jj) mbar_wait(&load_bar[jj % kNBuf], (jj / kNBuf) & 1, 20000);
+      for (int jj = 0; jj < nch; ++jj) mbar_wait(&load_bar[jj & 1], (jj >> 1) & 1, 20000);
     }
   }
   fence_before_sync();

@@ -258,3 +258,17 @@ def test_long_prefill_128k_sampled_heads():
     o, fs = _gpu(inp, "bf16")
     _check(inp, "bf16", o, fs, heads=[0, 21])
     assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("per_token", [-0.5, -1.1])
+def test_strong_decay_within_tensor_core_range(per_token):
+    """The tensor-core path forms e^{-g} inside a 64-token chunk; with a per-token
+    log-decay of -0.5 (-32 per chunk) or -1.1 (-70 per chunk) on a quarter of the
+    channels it must still match the oracle (the path's stated range is a chunk
+    log-decay above about -80)."""
+    inp = gen.random_case(61, [700, 64], 2, 128, 128, "bf16", init_state=True)
+    la = inp["log_alpha"].copy()
+    la[:, :, ::4] = per_token
+    inp["log_alpha"] = la
+    o, fs = _gpu(inp, "bf16")
+    _check(inp, "bf16", o, fs)
