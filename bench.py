@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--T", type=int, default=131072)
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-extras", action="store_true", help="headline prefill line only")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "conv", "backward"], default=None,
                     help="time one workload only (for profiling runs)")
     return ap.parse_args()
 
@@ -253,20 +253,24 @@ def cpu_baseline(inp, budget_s=10.0):
     from oracle import kda_oracle as orc
     H = inp["q"].shape[1]
 
-    def run(Ts):
+    def run(Ts, nthreads=0):
         cu = np.array([0, Ts], np.int32)
         t0 = time.perf_counter()
         orc.prefill(inp["q"][:Ts], inp["k"][:Ts], inp["v"][:Ts], inp["log_alpha"][:Ts],
-                    inp["beta"][:Ts], cu)
+                    inp["beta"][:Ts], cu, nthreads=nthreads)
         return time.perf_counter() - t0
     probe = 512
     dt = run(probe)
     Ts = int(min(inp["q"].shape[0], max(probe, probe * budget_s / max(dt, 1e-3))))
     Ts = max(probe, (Ts // 512) * 512)
     dt = run(Ts)
+    t1 = 256                                   # the same oracle on one core, a short prefix
+    dt1 = run(t1, nthreads=1)
     return {"value": Ts / dt, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
             "sample": f"first {Ts} of {inp['q'].shape[0]} tokens, all {H} heads, fp64 "
-                      f"token-by-token C oracle, {dt:.1f} s"}
+                      f"token-by-token C oracle, {dt:.1f} s",
+            "one_core": {"value": t1 / dt1, "unit": "tokens/s", "cores": 1,
+                         "sample": f"first {t1} tokens, all {H} heads, {dt1:.2f} s"}}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -434,27 +438,13 @@ def main_ours(args, rank, world, device):
             "log_alpha": "[N, H] fp32", "l2": "inputs larger than L2"}
         line["gpu_launches"] += LAUNCHES_PER_PREFILL * K
         del devh
+        # ---- backward pass at T = 4096 (token-serial fp32, reference grade)
+        line["backward"] = bench_backward(K, W, world, device, pk)
+        line["gpu_launches"] += 2 * K
         # ---- short convolution of q, k and v (D = H * d = 4096 each, W = 4, bf16, carried state)
-        cw = gen.conv_inputs(w.seed, [0], H * 128, 4)
-        cwt, cbias = torch.from_numpy(cw["weight"]).to(device), torch.from_numpy(cw["bias"]).to(device)
-        cst = torch.from_numpy(gen.conv_inputs(w.seed, [0], H * 128, 4)["state"]).to(device)
-        cu1 = torch.tensor([0, T], dtype=torch.int32, device=device)
-        ys = [torch.empty((T, H * 128), dtype=torch.bfloat16, device=device) for _ in range(3)]
-
-        def conv_step():
-            for i, key in enumerate(("q", "k", "v")):
-                kda.short_conv(dev[key].view(T, H * 128), cwt, cu1, bias=cbias, state_in=cst,
-                               state_out=cst, y=ys[i])
-        msc = time_loop(conv_step, K, W)
-        cbytes = 3 * (2 * T * H * 128 * 2 + 2 * 3 * H * 128 * 4 + H * 128 * 5 * 4)
-        line["short_conv"] = {
-            "workload": f"short_conv_qkv_T{T}_D{H * 128}_W4_bf16", "tokens_per_s": aggregate_rate(T, world, msc),
-            "ms": msc, "roofline": {"bound": "hbm", "achieved": cbytes / (msc / 1e3) / 1e9,
-                                    "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                    "frac": cbytes / (msc / 1e3) / 1e9 / pk["hbm_gbs"],
-                                    "algorithmic_bytes_per_step": cbytes}}
+        line["short_conv"] = bench_conv(K, W, world, device, pk,
+                                        [dev[key].view(T, H * 128) for key in ("q", "k", "v")], w.seed)
         line["gpu_launches"] += 2 * 3 * K
-        del ys, cst
 
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(inp)
@@ -502,6 +492,78 @@ def bench_decode(args, world, device, pk):
                          "algorithmic_bytes_per_launch": dbytes}}
 
 
+def bench_backward(K, W, world, device, pk, T=4096):
+    """kda_prefill_backward on one sequence of T tokens, H = 32, d = 128, bf16 inputs, fp32
+    gradients (all of them, including the initial state's)."""
+    import torch
+    from gated_delta_rule_148_b200 import inputs as gen
+    from gated_delta_rule_148_b200 import kda
+    w = gen.prefill(T)
+    inp = gen.prefill_inputs(w)
+    H = inp["q"].shape[1]
+    d = {key: torch.from_numpy(inp[key]).to(device) for key in ("log_alpha", "beta", "cu_seqlens")}
+    for key in ("q", "k", "v"):
+        d[key] = torch.from_numpy(inp[key]).to(device).to(torch.bfloat16)
+    go = torch.from_numpy(gen.grad_outputs(w.seed, T, H, 128)).to(device)
+    s0 = torch.zeros((1, H, 128, 128), dtype=torch.float32, device=device)
+    ws = torch.empty(T * H * 128 * 128 * 4, dtype=torch.uint8, device=device)
+
+    def step():
+        kda.prefill_backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"], go,
+                             init_state=s0, workspace=ws)
+    ms = max_over_ranks(time_loop(step, max(1, K // 2), max(1, W // 2)), world, device)
+    if kda.get_device_status() != kda.KDA_OK:
+        raise RuntimeError("device status after the backward pass")
+    # inputs q, k, v (bf16), log_alpha, beta, grad_o; outputs dq, dk, dv, dlog_alpha, dbeta (fp32)
+    per = 3 * 256 + 512 + 4 + 512 + 3 * 512 + 512 + 4
+    nb = T * H * per + 2 * H * 128 * 128 * 4
+    return {"workload": f"prefill_backward_T{T}_H{H}_d128_bf16_inputs", "tokens_per_s": aggregate_rate(T, world, ms),
+            "ms": ms, "algorithmic_bytes": nb,
+            "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+            "note": "token-serial fp32 reference-grade backward; the per-position states it stores "
+                    "(64 KiB per token and head) are not algorithmic bytes"}
+
+
+def bench_conv(K, W, world, device, pk, xs, seed):
+    """One layer's short convolutions: kda_short_conv over each [T, D] input of xs (q, k
+    and v), width 4, bf16, the carried state updated in place; K timed steps after W."""
+    import torch
+    from gated_delta_rule_148_b200 import inputs as gen
+    from gated_delta_rule_148_b200 import kda
+    T, D = xs[0].shape
+    cw = gen.conv_inputs(seed, [0], D, 4)
+    cwt, cbias = torch.from_numpy(cw["weight"]).to(device), torch.from_numpy(cw["bias"]).to(device)
+    cst = torch.from_numpy(cw["state"]).to(device)
+    cu1 = torch.tensor([0, T], dtype=torch.int32, device=device)
+    ys = [torch.empty((T, D), dtype=torch.bfloat16, device=device) for _ in xs]
+
+    def conv_step():
+        for x, y in zip(xs, ys):
+            kda.short_conv(x, cwt, cu1, bias=cbias, state_in=cst, state_out=cst, y=y)
+    ms = max_over_ranks(time_loop(conv_step, K, W), world, device)
+    if kda.get_device_status() != kda.KDA_OK:
+        raise RuntimeError("device status after the short convolution")
+    nb = len(xs) * (2 * T * D * 2 + 2 * 3 * D * 4 + D * 5 * 4)
+    return {"workload": f"short_conv_{len(xs)}x_T{T}_D{D}_W4_bf16",
+            "tokens_per_s": aggregate_rate(T, world, ms), "ms": ms,
+            "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes_per_step": nb}}
+
+
+def main_conv_only(args, rank, world, device):
+    import torch
+    from gated_delta_rule_148_b200 import inputs as gen
+    from gated_delta_rule_148_b200 import kda
+    kda.load()
+    c = gen.conv_inputs(gen.SEED_BASE + 5, [args.T], 4096, 4)
+    x = torch.from_numpy(c["x"]).to(device).to(torch.bfloat16)
+    d = bench_conv(args.steps, args.warmup, world, device, peaks(), [x, x, x], gen.SEED_BASE + 5)
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "short_conv": d}), flush=True)
+
+
 def main_decode_only(args, rank, world, device):
     from gated_delta_rule_148_b200 import kda
     kda.load()
@@ -528,6 +590,14 @@ def main():
     try:
         if args.only == "decode":
             main_decode_only(args, rank, world, device)
+        elif args.only == "conv":
+            main_conv_only(args, rank, world, device)
+        elif args.only == "backward":
+            from gated_delta_rule_148_b200 import kda
+            kda.load()
+            d = bench_backward(args.steps, args.warmup, world, device, peaks(), T=min(args.T, 4096))
+            if rank == 0:
+                print(json.dumps({"metric": METRIC, "backward": d}), flush=True)
         else:
             if args.only == "prefill":
                 args.no_extras = True

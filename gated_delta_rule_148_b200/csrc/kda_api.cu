@@ -259,6 +259,83 @@ kda_status kda_short_conv(const kda_conv_args *a, void *stream) {
              ? KDA_OK : KDA_ERR_CUDA;
 }
 
+size_t kda_prefill_backward_workspace_size(const kda_backward_args *a) {
+  if (!a || a->total_tokens < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0) return 0;
+  return backward_workspace(a->total_tokens, a->H, a->dk, a->dv);
+}
+
+kda_status kda_prefill_backward(const kda_backward_args *a, void *stream) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->dtype != KDA_F32 && a->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (a->num_seqs < 0 || a->total_tokens < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (!head_dim_ok(a->dk) || !head_dim_ok(a->dv)) return KDA_ERR_UNSUPPORTED;
+  if (a->gate != KDA_GATE_CHANNEL && a->gate != KDA_GATE_HEAD) return KDA_ERR_INVALID_ARG;
+  const bool gate_head = a->gate == KDA_GATE_HEAD;
+  if (a->num_seqs == 0) return a->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+  if (!a->cu_seqlens) return KDA_ERR_INVALID_ARG;
+  const size_t N = (size_t)a->total_tokens, H = (size_t)a->H, es = elem_bytes(a->dtype);
+  const size_t dk = a->dk, dv = a->dv, lad = gate_head ? 1 : dk;
+  const size_t sbytes = (size_t)a->num_seqs * H * dk * dv * 4;
+  if (N > 0 && (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->grad_o || !a->grad_q ||
+                !a->grad_k || !a->grad_v || !a->grad_log_alpha || !a->grad_beta))
+    return KDA_ERR_INVALID_ARG;
+  if (N > 0 && (!a->workspace || a->workspace_bytes < backward_workspace(a->total_tokens, a->H, a->dk, a->dv)))
+    return KDA_ERR_INVALID_ARG;
+  const Range q{a->q, N * H * dk * es}, k{a->k, N * H * dk * es}, v{a->v, N * H * dv * es};
+  const Range la{a->log_alpha, N * H * lad * 4}, be{a->beta, N * H * 4};
+  const Range cu{a->cu_seqlens, 4 * ((size_t)a->num_seqs + 1)}, mk{a->pad_mask, a->pad_mask ? N : 0};
+  const Range s0{a->init_state, a->init_state ? sbytes : 0};
+  const Range go{a->grad_o, N * H * dv * 4}, gf{a->grad_final_state, a->grad_final_state ? sbytes : 0};
+  const Range ws{a->workspace, a->workspace ? a->workspace_bytes : 0};
+  const Range outs[] = {{a->grad_q, N * H * dk * 4}, {a->grad_k, N * H * dk * 4}, {a->grad_v, N * H * dv * 4},
+                        {a->grad_log_alpha, N * H * lad * 4}, {a->grad_beta, N * H * 4},
+                        {a->grad_init_state, a->grad_init_state ? sbytes : 0}, ws};
+  const Range ins[] = {q, k, v, la, be, cu, mk, s0, go, gf};
+  for (int i = 0; i < 7; ++i) {
+    for (const Range &r : ins)
+      if (overlap(outs[i], r)) return KDA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 7; ++j)
+      if (overlap(outs[i], outs[j])) return KDA_ERR_INVALID_ARG;
+  }
+  const void *need16[] = {a->q, a->k, a->v, a->grad_o, a->grad_q, a->grad_k, a->grad_v, a->init_state,
+                          a->grad_final_state, a->grad_init_state};
+  for (const void *p : need16)
+    if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+  if (!aligned(a->log_alpha, 4) || !aligned(a->beta, 4) || !aligned(a->grad_log_alpha, 4) ||
+      !aligned(a->grad_beta, 4) || !aligned(a->cu_seqlens, 4) || (a->workspace && !aligned(a->workspace, 256)))
+    return KDA_ERR_INVALID_ARG;
+  unsigned *err = nullptr;
+  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  BackwardParams p;
+  p.num_seqs = a->num_seqs;
+  p.N = a->total_tokens;
+  p.H = a->H;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.log_alpha = a->log_alpha;
+  p.beta = a->beta;
+  p.cu = a->cu_seqlens;
+  p.mask = a->pad_mask;
+  p.init_state = a->init_state;
+  p.d_o = a->grad_o;
+  p.d_final_state = a->grad_final_state;
+  p.gq = a->grad_q;
+  p.gk = a->grad_k;
+  p.gv = a->grad_v;
+  p.gla = a->grad_log_alpha;
+  p.gbeta = a->grad_beta;
+  p.g_init_state = a->grad_init_state;
+  p.ws = static_cast<float *>(a->workspace);
+  p.err = err;
+  p.gate_head = gate_head ? 1 : 0;
+  return launch_backward(p, a->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_get_device_status(void *stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
   unsigned *err = nullptr;

@@ -61,6 +61,20 @@ struct ConvParams {
   unsigned *err;
 };
 
+struct BackwardParams {
+  int num_seqs, N, H, dk, dv;
+  const void *q, *k, *v;
+  const float *log_alpha, *beta;
+  const int32_t *cu;
+  const uint8_t *mask;
+  const float *init_state;
+  const float *d_o, *d_final_state;
+  float *gq, *gk, *gv, *gla, *gbeta, *g_init_state;
+  float *ws;              // [N, H, dk, dv]: the state before every position
+  unsigned *err;
+  int gate_head;
+};
+
 // Launchers (return a CUDA error code; argument checks happen before).
 cudaError_t launch_prefill_prepass(const PrefillParams &p, bool bf16, SeqSpan *spans,
                                    cudaStream_t s);
@@ -73,6 +87,8 @@ size_t prefill_split_workspace(int N, int B, int H);
 cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s);
+size_t backward_workspace(int N, int H, int dk, int dv);
+cudaError_t launch_backward(const BackwardParams &p, bool bf16, cudaStream_t s);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {

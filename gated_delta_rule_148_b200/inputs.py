@@ -33,7 +33,7 @@ import numpy as np
 SEED_BASE = 1480
 
 _STREAMS = ("q", "k", "v", "log_alpha", "beta", "state", "structure", "decode_mask",
-            "log_alpha_head", "conv_x", "conv_weight")
+            "log_alpha_head", "conv_x", "conv_weight", "grad_o")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -202,6 +202,11 @@ def conv_inputs(seed: int, lengths: Sequence[int], D: int, W: int, dtype: str = 
         rng = _child(seed, "structure", 2)
         out["pad_mask"] = (rng.uniform(size=N) >= pad_frac).astype(np.uint8)
     return out
+
+
+def grad_outputs(seed: int, N: int, H: int, dv: int) -> np.ndarray:
+    """Upstream gradient of o for a backward pass: [N, H, dv] ~ N(0, 1), fp32."""
+    return _normal(seed, "grad_o", (N, H, dv))
 
 
 def prefill_inputs(w: Workload) -> Dict[str, np.ndarray]:

@@ -32,7 +32,8 @@ KDA_GATE_CHANNEL = 0
 KDA_GATE_HEAD = 1
 
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
-            "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_short_conv")
+            "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_short_conv",
+            "kda_prefill_backward", "kda_prefill_backward_workspace_size")
 
 
 class KdaError(RuntimeError):
@@ -71,6 +72,21 @@ class ConvArgs(ctypes.Structure):
                 ("y", ctypes.c_void_p)]
 
 
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("num_seqs", ctypes.c_int),
+                ("total_tokens", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("log_alpha", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
+                ("pad_mask", ctypes.c_void_p), ("init_state", ctypes.c_void_p),
+                ("gate", ctypes.c_int), ("grad_o", ctypes.c_void_p),
+                ("grad_final_state", ctypes.c_void_p), ("grad_q", ctypes.c_void_p),
+                ("grad_k", ctypes.c_void_p), ("grad_v", ctypes.c_void_p),
+                ("grad_log_alpha", ctypes.c_void_p), ("grad_beta", ctypes.c_void_p),
+                ("grad_init_state", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -92,6 +108,12 @@ def load(build_if_stale: bool = True) -> ctypes.CDLL:
             lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
             lib.kda_decode.argtypes = [ctypes.POINTER(DecodeArgs), ctypes.c_void_p]
             lib.kda_decode.restype = ctypes.c_int
+            lib.kda_short_conv.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
+            lib.kda_short_conv.restype = ctypes.c_int
+            lib.kda_prefill_backward.argtypes = [ctypes.POINTER(BackwardArgs), ctypes.c_void_p]
+            lib.kda_prefill_backward.restype = ctypes.c_int
+            lib.kda_prefill_backward_workspace_size.argtypes = [ctypes.POINTER(BackwardArgs)]
+            lib.kda_prefill_backward_workspace_size.restype = ctypes.c_size_t
             lib.kda_get_device_status.argtypes = [ctypes.c_void_p]
             lib.kda_get_device_status.restype = ctypes.c_int
             lib.kda_status_string.argtypes = [ctypes.c_int]
@@ -280,6 +302,52 @@ def short_conv(x: torch.Tensor, weight: torch.Tensor, cu_seqlens: torch.Tensor,
     if st != KDA_OK:
         raise KdaError(st, "kda_short_conv")
     return y
+
+
+def prefill_backward(q, k, v, log_alpha, beta, cu_seqlens, grad_o, grad_final_state=None,
+                     pad_mask=None, init_state=None, want_grad_init_state: bool = True,
+                     workspace=None, stream=None):
+    """Backward of the prefill (kda_prefill_backward).  Returns a dict of fp32 CUDA
+    tensors dq, dk, dv, dlog_alpha (log_alpha's layout), dbeta and dS0 (None unless
+    wanted).  grad_o [N,H,dv] and grad_final_state [B,H,dk,dv] are fp32."""
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    B = cu_seqlens.numel() - 1
+    gate = gate_layout(log_alpha)
+    _check_cuda("q", q, shape=(N, H, dk))
+    _check_cuda("k", k, q.dtype, (N, H, dk))
+    _check_cuda("v", v, q.dtype, (N, H, dv))
+    _check_cuda("log_alpha", log_alpha, torch.float32, (N, H) if gate == KDA_GATE_HEAD else (N, H, dk))
+    _check_cuda("beta", beta, torch.float32, (N, H))
+    _check_cuda("cu_seqlens", cu_seqlens, torch.int32, (B + 1,))
+    _check_cuda("pad_mask", pad_mask, torch.uint8, (N,))
+    _check_cuda("init_state", init_state, torch.float32, (B, H, dk, dv))
+    _check_cuda("grad_o", grad_o, torch.float32, (N, H, dv))
+    _check_cuda("grad_final_state", grad_final_state, torch.float32, (B, H, dk, dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((N, H, dk), **f32), "dk": torch.empty((N, H, dk), **f32),
+         "dv": torch.empty((N, H, dv), **f32), "dlog_alpha": torch.empty(tuple(log_alpha.shape), **f32),
+         "dbeta": torch.empty((N, H), **f32),
+         "dS0": torch.empty((B, H, dk, dv), **f32) if want_grad_init_state else None}
+    a = BackwardArgs()
+    a.dtype = _dtype_code(q)
+    a.num_seqs, a.total_tokens, a.H, a.dk, a.dv = B, N, H, dk, dv
+    a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
+    a.log_alpha, a.beta, a.cu_seqlens = _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens)
+    a.pad_mask, a.init_state, a.gate = _ptr(pad_mask), _ptr(init_state), gate
+    a.grad_o, a.grad_final_state = _ptr(grad_o), _ptr(grad_final_state)
+    a.grad_q, a.grad_k, a.grad_v = _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"])
+    a.grad_log_alpha, a.grad_beta, a.grad_init_state = _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"])
+    if workspace is None:
+        nbytes = int(lib.kda_prefill_backward_workspace_size(ctypes.byref(a)))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    a.workspace = _ptr(workspace)
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib.kda_prefill_backward(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill_backward")
+    return g
 
 
 def get_device_status(stream=None) -> int:

@@ -238,6 +238,59 @@ typedef struct {
 
 kda_status kda_short_conv(const kda_conv_args *args, void *stream);
 
+/*
+ * Backward pass of kda_prefill (training): the gradients of <o, grad_o> +
+ * <final_state, grad_final_state> with respect to q, k, v, log_alpha, beta and
+ * init_state, by reverse-mode differentiation of the recurrence (the blockwise
+ * algorithm serves training as well as inference: "Kimi Linear wlasnie
+ * pokonal ...", remio.ai, section "Jak Kimi Linear wykorzystuje inteligentniejsza
+ * pamiec rekurencyjna").  Token-serial fp32 on CUDA cores, one CTA per
+ * (sequence, head): a reference-grade backward, not a tuned one.
+ * Fields (device pointers, caller-owned):
+ *   dtype, num_seqs, total_tokens, H, dk, dv, q, k, v, log_alpha, beta,
+ *   cu_seqlens, pad_mask, init_state, gate   as for kda_prefill (chunk is not
+ *                used; the result does not depend on it).
+ *   grad_o           [N, H, dv] fp32.
+ *   grad_final_state [B, H, dk, dv] fp32 or NULL (zero).
+ *   grad_q, grad_k   [N, H, dk] fp32; grad_v [N, H, dv] fp32;
+ *   grad_log_alpha   fp32, the layout of log_alpha; grad_beta [N, H] fp32;
+ *   grad_init_state  [B, H, dk, dv] fp32 or NULL (not written).
+ *                All outputs 16-byte aligned and not overlapping any input or
+ *                each other; pad positions get zero gradients.
+ *   workspace    kda_prefill_backward_workspace_size() bytes, 256-byte aligned
+ *                (the state before every position: N * H * dk * dv * 4 bytes).
+ */
+typedef struct {
+  kda_dtype dtype;
+  int num_seqs;
+  int total_tokens;
+  int H;
+  int dk;
+  int dv;
+  const void *q;
+  const void *k;
+  const void *v;
+  const float *log_alpha;
+  const float *beta;
+  const int32_t *cu_seqlens;
+  const uint8_t *pad_mask;
+  const float *init_state;
+  kda_gate gate;
+  const float *grad_o;
+  const float *grad_final_state;
+  float *grad_q;
+  float *grad_k;
+  float *grad_v;
+  float *grad_log_alpha;
+  float *grad_beta;
+  float *grad_init_state;
+  void *workspace;
+  size_t workspace_bytes;
+} kda_backward_args;
+
+size_t kda_prefill_backward_workspace_size(const kda_backward_args *args);
+kda_status kda_prefill_backward(const kda_backward_args *args, void *stream);
+
 /* Synchronise `stream`, then return and clear the error latched on the
  * current device by earlier kernels (KDA_OK if none). */
 kda_status kda_get_device_status(void *stream);

@@ -301,3 +301,78 @@ def short_conv_at(x, weight, bias, cu_seqlens, positions, pad_mask=None, state_i
         u = prev[::-1] + [np.asarray(x[t], dtype=np.float64)]
         out[n] = b0 + sum(w[:, i] * u[i] for i in range(W))
     return out
+
+
+# ----------------------------------------------------------------------------
+# Backward pass (reverse-mode derivative of the recurrence, token by token)
+# ----------------------------------------------------------------------------
+def prefill_backward(q, k, v, log_alpha, beta, cu_seqlens, do, dS_final=None, pad_mask=None,
+                     init_state=None):
+    """Gradients of the prefill's outputs (o and the final state) with respect to every
+    input, for upstream gradients ``do`` [N,H,dv] and ``dS_final`` [B,H,dk,dv] (None = 0).
+    The forward step is taken apart into its four operations -- decay S' = Diag(a) S,
+    read p = S'^T k, correction u = beta (v - p), write S = S' + k u^T, output o = S^T q --
+    and each one's adjoint is applied in reverse order (chain rule), in fp64, with the
+    states recomputed forward.  Pads are identity steps: zero gradients there, the state
+    gradient passes through.  Returns a dict with dq, dk, dv, dlog_alpha (the gate's
+    layout), dbeta and dS0."""
+    head_gate = np.asarray(log_alpha).ndim == 2
+    dkk = np.shape(q)[2]
+    la_full = np.asarray(head_gate_channels(log_alpha, dkk), dtype=np.float64)
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    be = np.asarray(beta, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = len(cu) - 1
+    g = {name: np.zeros_like(x) for name, x in (("dq", q), ("dk", k), ("dv", v))}
+    g["dlog_alpha"] = np.zeros((N, H, dk))
+    g["dbeta"] = np.zeros((N, H))
+    g["dS0"] = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if init_state is None else np.asarray(init_state[b, h], np.float64)
+            states = []                      # S_{t-1} before each position
+            for t in range(int(cu[b]), int(cu[b + 1])):
+                states.append(S.copy())
+                if pad_mask is not None and pad_mask[t] == 0:
+                    continue
+                a = np.exp(la_full[t, h])
+                Sp = a[:, None] * S
+                p = Sp.T @ k[t, h]
+                u = be[t, h] * (v[t, h] - p)
+                S = Sp + np.outer(k[t, h], u)
+            G = np.zeros((dk, dv)) if dS_final is None else np.asarray(dS_final[b, h], np.float64).copy()
+            for idx in range(int(cu[b + 1]) - 1, int(cu[b]) - 1, -1):
+                if pad_mask is not None and pad_mask[idx] == 0:
+                    continue
+                Sprev = states[idx - int(cu[b])]
+                a = np.exp(la_full[idx, h])
+                kt, qt, vt, bt, dot = k[idx, h], q[idx, h], v[idx, h], be[idx, h], do[idx, h]
+                Sp = a[:, None] * Sprev
+                p = Sp.T @ kt
+                u = bt * (v[idx, h] - p)
+                St = Sp + np.outer(kt, u)
+                # o = S_t^T q
+                g["dq"][idx, h] = St @ dot
+                G = G + np.outer(qt, dot)
+                # S_t = S' + k u^T
+                dk_ = G @ u
+                du = G.T @ kt
+                Gp = G.copy()
+                # u = beta (v - p)
+                g["dv"][idx, h] = bt * du
+                g["dbeta"][idx, h] = du @ (vt - p)
+                dp = -bt * du
+                # p = S'^T k
+                Gp += np.outer(kt, dp)
+                dk_ += Sp @ dp
+                g["dk"][idx, h] = dk_
+                # S' = Diag(a) S_{t-1}, a = exp(log_alpha)
+                g["dlog_alpha"][idx, h] = (Gp * Sp).sum(axis=1)
+                G = a[:, None] * Gp
+            g["dS0"][b, h] = G
+    if head_gate:
+        g["dlog_alpha"] = g["dlog_alpha"].sum(axis=2)
+    return g

@@ -41,6 +41,7 @@ def test_struct_layout_matches_header(tmp_path):
     fields_p = [f[0] for f in kda.PrefillArgs._fields_]
     fields_d = [f[0] for f in kda.DecodeArgs._fields_]
     fields_c = [f[0] for f in kda.ConvArgs._fields_]
+    fields_b = [f[0] for f in kda.BackwardArgs._fields_]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "kda.h"', 'int main(void){']
     lines.append('printf("P %zu\\n", sizeof(kda_prefill_args));')
     for f in fields_p:
@@ -51,6 +52,9 @@ def test_struct_layout_matches_header(tmp_path):
     lines.append('printf("C %zu\\n", sizeof(kda_conv_args));')
     for f in fields_c:
         lines.append(f'printf("C.{f} %zu\\n", offsetof(kda_conv_args, {f}));')
+    lines.append('printf("B %zu\\n", sizeof(kda_backward_args));')
+    for f in fields_b:
+        lines.append(f'printf("B.{f} %zu\\n", offsetof(kda_backward_args, {f}));')
     lines.append("return 0;}")
     prog.write_text("\n".join(lines))
     exe = tmp_path / "layout"
@@ -66,6 +70,9 @@ def test_struct_layout_matches_header(tmp_path):
     assert int(got["C"]) == ctypes.sizeof(kda.ConvArgs)
     for f in fields_c:
         assert int(got[f"C.{f}"]) == getattr(kda.ConvArgs, f).offset, f
+    assert int(got["B"]) == ctypes.sizeof(kda.BackwardArgs)
+    for f in fields_b:
+        assert int(got[f"B.{f}"]) == getattr(kda.BackwardArgs, f).offset, f
 
 
 def test_status_strings():

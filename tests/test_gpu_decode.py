@@ -91,3 +91,36 @@ def test_batched_decode_full_size_1000_steps():
     assert worst <= TOL["bf16"]
     assert norm_err(to_np(state[track]), ref) <= TOL["bf16"]
     assert kda.get_device_status() == kda.KDA_OK
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_prefill_to_decode_handoff(dtype):
+    """Prefill hands its final state to decode with no conversion (same [B,H,dk,dv] fp32
+    layout, updated in place): prefill of T tokens then 5 decode steps equals the oracle's
+    prefill of the T + 5 tokens, for the outputs of the decoded tokens and the final state."""
+    H, d, T, steps = 2, 128, 300, 5
+    lens = [T + steps, T + steps]
+    c = gen.random_case(55, lens, H, d, d, dtype, init_state=True)
+    B = len(lens)
+    cu = c["cu_seqlens"]
+    first = np.concatenate([np.arange(cu[b], cu[b] + T) for b in range(B)])
+    pre = {k: c[k][first] for k in ("q", "k", "v", "log_alpha", "beta")}
+    pre["cu_seqlens"] = np.array([0, T, 2 * T], np.int32)
+    pre["init_state"] = c["init_state"]
+    dd = dev_inputs(pre, dtype)
+    _, state = kda.prefill(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], dd["cu_seqlens"],
+                           init_state=dd["init_state"])
+    outs = []
+    for s in range(steps):
+        rows = np.array([cu[b] + T + s for b in range(B)])
+        tok = {k: c[k][rows] for k in ("q", "k", "v", "log_alpha", "beta")}
+        dt = dev_inputs(tok, dtype)
+        outs.append(to_np(kda.decode(dt["q"], dt["k"], dt["v"], dt["log_alpha"], dt["beta"], state)))
+    torch.cuda.synchronize()
+    o_ref, s_ref = orc.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], cu,
+                               init_state=c["init_state"])
+    for s in range(steps):
+        rows = np.array([cu[b] + T + s for b in range(B)])
+        assert norm_err(outs[s], o_ref[rows]) <= TOL[dtype]
+    assert norm_err(to_np(state), s_ref) <= TOL[dtype]
+    assert kda.get_device_status() == kda.KDA_OK

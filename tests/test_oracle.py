@@ -495,3 +495,72 @@ def test_conv_sampled_positions_match_window_form():
     y, _ = orc.short_conv(x, w, b, cu, m, s)
     pos = np.array([0, 1, 5, 33, 34, 35, 100, 153])
     np.testing.assert_allclose(orc.short_conv_at(x, w, b, cu, pos, m, s), y[pos], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward pass
+def _loss_bf(q, k, v, la, be, S0, cu, m, do, dSf):
+    """<o, do> + <S_final, dSf> through the fp64 brute force (explicit transitions),
+    per sequence and head; la may be [N, H] (head-wise gate)."""
+    tot = 0.0
+    la_full = orc.head_gate_channels(la, q.shape[2])
+    for b in range(len(cu) - 1):
+        a, e = int(cu[b]), int(cu[b + 1])
+        for h in range(q.shape[1]):
+            o, S = orc.brute_force(q[a:e, h], k[a:e, h], v[a:e, h], la_full[a:e, h], be[a:e, h],
+                                   S0[b, h], None if m is None else m[a:e])
+            tot += (o * do[a:e, h]).sum() + (S * dSf[b, h]).sum()
+    return tot
+
+
+@pytest.mark.parametrize("head_gate", [False, True])
+def test_backward_matches_central_differences(head_gate):
+    """Every gradient of prefill_backward equals the central difference of the fp64
+    brute-force loss <o, dO> + <S_T, dS_T> (step 1e-6), on two sequences with pads."""
+    rng = np.random.default_rng(71)
+    N, H, dk, dv = 9, 2, 3, 2
+    q, k = rng.normal(size=(N, H, dk)), rng.normal(size=(N, H, dk))
+    v = rng.normal(size=(N, H, dv))
+    la = -np.abs(rng.normal(size=(N, H) if head_gate else (N, H, dk)))
+    be = rng.uniform(-0.3, 1.2, (N, H))
+    S0 = rng.normal(size=(2, H, dk, dv))
+    cu = np.array([0, 4, 9])
+    m = np.array([1, 1, 0, 1, 1, 0, 1, 1, 1], np.uint8)
+    do, dSf = rng.normal(size=(N, H, dv)), rng.normal(size=(2, H, dk, dv))
+    g = orc.prefill_backward(q, k, v, la, be, cu, do, dSf, m, S0)
+    args = dict(q=q, k=k, v=v, la=la, be=be, S0=S0)
+    keys = dict(q="dq", k="dk", v="dv", la="dlog_alpha", be="dbeta", S0="dS0")
+    eps = 1e-6
+    for name, x in list(args.items()):
+        fd = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            for sgn in (1, -1):
+                xx = x.copy()
+                xx[i] += sgn * eps
+                fd[i] += sgn * _loss_bf(**dict(args, **{name: xx}), cu=cu, m=m, do=do, dSf=dSf)
+        fd /= 2 * eps
+        np.testing.assert_allclose(g[keys[name]], fd, rtol=1e-6, atol=1e-7, err_msg=name)
+    # pads: zero input gradients
+    for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        assert np.all(g[key][m == 0] == 0.0)
+
+
+def test_backward_zero_upstream_and_state_only():
+    """dO = 0 and dS_T = 0 give all-zero gradients; with beta = 0 and dO = 0 the state
+    gradient is the closed form dS0 = Diag(exp(sum log_alpha)) dS_T and
+    dlog_alpha_t = rowsum(dS_T * S_T) for every t (each decay scales the final state)."""
+    rng = np.random.default_rng(72)
+    N, dk, dv = 6, 4, 3
+    q, k, v = rng.normal(size=(N, 1, dk)), rng.normal(size=(N, 1, dk)), rng.normal(size=(N, 1, dv))
+    la = -np.abs(rng.normal(size=(N, 1, dk)))
+    S0 = rng.normal(size=(1, 1, dk, dv))
+    cu = np.array([0, N])
+    g = orc.prefill_backward(q, k, v, la, rng.uniform(size=(N, 1)), cu, np.zeros((N, 1, dv)),
+                             None, None, S0)
+    assert all(np.all(g[key] == 0) for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"))
+    dSf = rng.normal(size=(1, 1, dk, dv))
+    g = orc.prefill_backward(q, k, v, la, np.zeros((N, 1)), cu, np.zeros((N, 1, dv)), dSf, None, S0)
+    decay = np.exp(la[:, 0].sum(axis=0))
+    np.testing.assert_allclose(g["dS0"][0, 0], decay[:, None] * dSf[0, 0], rtol=1e-12)
+    ST = decay[:, None] * S0[0, 0]
+    for t in range(N):
+        np.testing.assert_allclose(g["dlog_alpha"][t, 0], (dSf[0, 0] * ST).sum(axis=1), rtol=1e-12)
