@@ -272,3 +272,20 @@ def test_strong_decay_within_tensor_core_range(per_token):
     inp["log_alpha"] = la
     o, fs = _gpu(inp, "bf16")
     _check(inp, "bf16", o, fs)
+
+
+def test_many_short_sequences_two_kernel_path():
+    """3000 sequences of 1-40 tokens (most shorter than one chunk), H = 2, bf16, d = 128,
+    pads, nonzero states: the chunk index over thousands of sequences and the many
+    partial chunks of the two-kernel path."""
+    rng = np.random.default_rng(77)
+    lengths = [int(x) for x in rng.integers(1, 41, size=3000)]
+    inp = gen.random_case(78, lengths, 2, 128, 128, "bf16", init_state=True)
+    N = int(inp["cu_seqlens"][-1])
+    m = (rng.uniform(size=N) > 0.1).astype(np.uint8)
+    for key in ("q", "k", "v"):
+        inp[key][m == 0] = 0.0
+    inp["pad_mask"] = m
+    o, fs = _gpu(inp, "bf16")
+    _check(inp, "bf16", o, fs)
+    assert np.all(to_np(o)[m == 0] == 0.0)
