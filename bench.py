@@ -252,6 +252,7 @@ def cpu_baseline(inp, budget_s=10.0):
     """The fp64 oracle on the first T_s tokens (all heads) of the workload."""
     from oracle import kda_oracle as orc
     H = inp["q"].shape[1]
+    cores = orc.max_threads()
 
     def run(Ts, nthreads=0):
         cu = np.array([0, Ts], np.int32)
@@ -266,7 +267,7 @@ def cpu_baseline(inp, budget_s=10.0):
     dt = run(Ts)
     t1 = 256                                   # the same oracle on one core, a short prefix
     dt1 = run(t1, nthreads=1)
-    return {"value": Ts / dt, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+    return {"value": Ts / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"first {Ts} of {inp['q'].shape[0]} tokens, all {H} heads, fp64 "
                       f"token-by-token C oracle, {dt:.1f} s",
             "one_core": {"value": t1 / dt1, "unit": "tokens/s", "cores": 1,

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
   extern __shared__ __align__(16) float smem[];
   __shared__ float sk[128], sq[128], sv[128], sa[128], sdo[128];
   __shared__ float sp[128], su[128], sdp[128], sc2[128], sr1[128], sr4[128];
+  __shared__ float sr2[2][128], sr3[2][128];
   __shared__ float red[kThreads / 32];
   if (device_error_latched(p.err)) return;
   const int b = blockIdx.x / p.H, h = blockIdx.x % p.H, tid = threadIdx.x;
@@ -260,21 +261,29 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
     }
     const float db = block_sum(x3, red);      // its barriers also publish sdp
     if (tid == 0) p.gbeta[bh] = db;
-    // ---- pass 2: R2 = G u, R3 = S dp (rows); dq, dk, dlog_alpha
+    // ---- pass 2: R2 = G u, R3 = S dp (rows; two threads per row, half the columns each)
+    {
+      const int i = tid & 127, half = tid >> 7, w = DV / 2;
+      if (i < DK) {
+        float r2v[4] = {0.f, 0.f, 0.f, 0.f}, r3v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int jj = 0; jj < w; jj += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = (i + half * w + jj + u) & (DV - 1);   // rotated: conflict-free banks
+            r2v[u] = fmaf(G[i * DV + j], su[j], r2v[u]);
+            r3v[u] = fmaf(S[i * DV + j], sdp[j], r3v[u]);
+          }
+        }
+        sr2[half][i] = (r2v[0] + r2v[1]) + (r2v[2] + r2v[3]);
+        sr3[half][i] = (r3v[0] + r3v[1]) + (r3v[2] + r3v[3]);
+      }
+    }
+    __syncthreads();
+    // ---- dq, dk, dlog_alpha
     float xla = 0.f;
     for (int i = tid; i < DK; i += kThreads) {
-      float r2v[4] = {0.f, 0.f, 0.f, 0.f}, r3v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int jj = 0; jj < DV; jj += 4) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = (i + jj + u) & (DV - 1);
-          r2v[u] = fmaf(G[i * DV + j], su[j], r2v[u]);
-          r3v[u] = fmaf(S[i * DV + j], sdp[j], r3v[u]);
-        }
-      }
-      const float r2 = (r2v[0] + r2v[1]) + (r2v[2] + r2v[3]);
-      const float r3 = (r3v[0] + r3v[1]) + (r3v[2] + r3v[3]);
+      const float r2 = sr2[0][i] + sr2[1][i], r3 = sr3[0][i] + sr3[1][i];
       const float ai = sa[i];
       p.gq[bh * DK + i] = ai * sr1[i] + sk[i] * udo;
       p.gk[bh * DK + i] = r2 + sq[i] * udo + ai * r3;

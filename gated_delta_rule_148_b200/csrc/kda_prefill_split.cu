@@ -19,7 +19,6 @@
 //   [65536, 73728)  M            64 x 64 bf16 row tile
 //   [73728, 74240)  e^{g_C}      128 fp32
 #include <climits>
-#include <mutex>
 
 #include <cudaTypedefs.h>
 
@@ -606,18 +605,7 @@ size_t prefill_split_workspace(int N, int B, int H) { return split::ws_total(N, 
 
 namespace {
 
-// Head groups run as a pipeline: the intra kernel of group g+1 (bandwidth-bound,
-// all SMs) overlaps the state pass of group g (latency-bound, few SMs) on its
-// own high-priority stream; everything joins back on the caller's stream.
-constexpr int kGroups = 1;
 constexpr int kMaxDev = 64;
-struct GroupStreams {
-  bool ready = false;
-  cudaStream_t aux[kGroups];
-  cudaEvent_t ev_a[kGroups], ev_b[kGroups];
-};
-GroupStreams g_streams[kMaxDev];
-std::mutex g_streams_mu;
 
 int num_sms() {
   static int n[kMaxDev] = {0};
@@ -629,27 +617,6 @@ int num_sms() {
     n[dev] = v;
   }
   return n[dev];
-}
-
-cudaError_t group_streams(GroupStreams **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  GroupStreams &gs = g_streams[dev];
-  if (!gs.ready) {
-    int least = 0, greatest = 0;
-    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
-    if (e != cudaSuccess) return e;
-    for (int g = 0; g < kGroups; ++g) {
-      if ((e = cudaStreamCreateWithPriority(&gs.aux[g], cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
-      if ((e = cudaEventCreateWithFlags(&gs.ev_a[g], cudaEventDisableTiming)) != cudaSuccess) return e;
-      if ((e = cudaEventCreateWithFlags(&gs.ev_b[g], cudaEventDisableTiming)) != cudaSuccess) return e;
-    }
-    gs.ready = true;
-  }
-  *out = &gs;
-  return cudaSuccess;
 }
 
 }  // namespace
@@ -672,30 +639,13 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_streams_mu);
-  GroupStreams *gs = nullptr;
-  if ((e = group_streams(&gs)) != cudaSuccess) return e;
-  const int G = p.H < kGroups ? p.H : kGroups;
-  const int Hg = (p.H + G - 1) / G;
-  int used = 0;
-  for (int g = 0; g < G; ++g) {
-    const int h0 = g * Hg, hg = (p.H - h0) < Hg ? (p.H - h0) : Hg;
-    if (hg <= 0) break;
-    const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)hg;
-    if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
-    const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
-    intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, h0, hg);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(gs->ev_a[g], s)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(gs->aux[g], gs->ev_a[g], 0)) != cudaSuccess) return e;
-    const unsigned gridB = (unsigned)p.num_seqs * hg * (p.dv / kNV);
-    state_kernel<<<gridB, kThreadsB, B_SMEM, gs->aux[g]>>>(p, spans, cbase, items, h0, hg);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(gs->ev_b[g], gs->aux[g])) != cudaSuccess) return e;
-    ++used;
-  }
-  for (int g = 0; g < used; ++g)
-    if ((e = cudaStreamWaitEvent(s, gs->ev_b[g], 0)) != cudaSuccess) return e;
+  const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
+  if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+  const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
+  intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, 0, p.H);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / kNV);
+  state_kernel<<<gridB, kThreadsB, B_SMEM, s>>>(p, spans, cbase, items, 0, p.H);
   return cudaGetLastError();
 }
 

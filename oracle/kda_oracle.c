@@ -97,8 +97,9 @@ int kda_oracle_prefill(int num_seqs, const int32_t *cu_seqlens, int H, int dk,
   for (b = 0; b < num_seqs; ++b)
     if (cu_seqlens[b + 1] < cu_seqlens[b]) return -1;
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#pragma omp parallel for schedule(dynamic, 1)
+  /* nthreads > 0 limits this call only; the process-wide default is left alone */
+  const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
 #endif
   for (long w = 0; w < (long)num_seqs * H; ++w) {
     int bb = (int)(w / H), h = (int)(w % H);
@@ -138,8 +139,8 @@ int kda_oracle_decode(int B, int H, int dk, int dv, const float *q,
                       double *o, int nthreads) {
   if (B < 0 || H <= 0 || dk <= 0 || dv <= 0 || !state || !o) return -1;
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#pragma omp parallel for schedule(static)
+  const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel for schedule(static) num_threads(nt)
 #endif
   for (long w = 0; w < (long)B * H; ++w) {
     int b = (int)(w / H);
