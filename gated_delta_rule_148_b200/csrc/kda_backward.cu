@@ -18,7 +18,7 @@
 // du = C2 + (q.k) dO and dlog_alpha = a * (R4 + q*R1 + k*R3).
 //
 // Every column of the state follows its own recursion given the key-side vectors,
-// so the work splits over 32-column d_v slices: u, du, dp, dv and G's columns stay
+// so the work splits over 16-column d_v slices: u, du, dp, dv and G's columns stay
 // in one CTA, while the row sums behind dq, dk, dlog_alpha and dbeta are sums of
 // per-slice shares, added into zeroed outputs.  Two kernels, one CTA per
 // (sequence, head, slice): the first replays the forward and stores the state
@@ -34,7 +34,9 @@ namespace kda {
 namespace bwd {
 
 constexpr int kThreads = 256;
-constexpr int kSW = 32;          // d_v columns per CTA (each column's recursion is independent)
+constexpr int kSW = 16;          // d_v columns per CTA (each column's recursion is independent)
+constexpr int kQ = kSW / 4;      // float4 per row of a slice
+constexpr int kCG = 128 / kSW;   // column-sum row groups in the grad kernel (threads 128..255)
 
 __device__ __forceinline__ float block_sum(float x, float *red) {
   // sum over the CTA's 256 threads (every thread gets the result)
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(kThreads) states_kernel(BackwardParams p) {
   float4 *S4 = reinterpret_cast<float4 *>(S);
   const float *I = p.init_state ? p.init_state + ((size_t)b * p.H + h) * DK * DV : nullptr;
   for (int e = tid; e < n4; e += kThreads) {
-    const int i = e >> 3, c = (e & 7) * 4;
+    const int i = e / kQ, c = (e % kQ) * 4;
     S4[e] = I ? *reinterpret_cast<const float4 *>(I + (size_t)i * DV + j0 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   Vec nxt = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads) states_kernel(BackwardParams p) {
     // finish the previous write, store the state before pos, decay it
     const float *kpv = kbuf[kp];
     for (int e = tid; e < n4; e += kThreads) {
-      const int i = e >> 3, c = (e & 7) * 4;
+      const int i = e / kQ, c = (e % kQ) * 4;
       float4 x = S4[e];
       if (pend) {
         const float ki = kpv[i];
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
   extern __shared__ __align__(16) float dyn[];          // two state buffers + G, [dk][kSW] each
   __shared__ float sk[128], sq[128], sa[128], sr1[128], sr4[128];
   __shared__ float sv[kSW], sdo[kSW], sp[kSW], su[kSW], sdp[kSW], sc2[kSW];
-  __shared__ float partp[4][kSW], partc[4][kSW];
+  __shared__ float partp[kCG][kSW], partc[kCG][kSW];
   __shared__ float red[kThreads / 32];
   if (device_error_latched(p.err)) return;
   const int ns = p.dv / kSW, sl = blockIdx.x % ns, bhi = blockIdx.x / ns;
@@ -174,13 +176,13 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
   float4 *G4 = reinterpret_cast<float4 *>(G);
   const float *F = p.d_final_state ? p.d_final_state + ((size_t)b * H + h) * DK * DV : nullptr;
   for (int e = tid; e < n4; e += kThreads) {
-    const int i = e >> 3, c = (e & 7) * 4;
+    const int i = e / kQ, c = (e % kQ) * 4;
     G4[e] = F ? *reinterpret_cast<const float4 *>(F + (size_t)i * DV + j0 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   auto prefetch = [&](int pos, float *dst) {
     const float *src = p.ws + ((size_t)pos * H + h) * DK * DV + j0;
     for (int e = tid; e < n4; e += kThreads) {
-      const int i = e >> 3, c = (e & 7) * 4;
+      const int i = e / kQ, c = (e % kQ) * 4;
       tc::cp_async16(tc::smem_u32(dst + i * kSW + c), src + (size_t)i * DV + c, 16);
     }
     tc::cp_async_commit();
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
     prefetch(ce - 1, Sbuf[0]);
     nxt = fetch<BF16>(p, (size_t)ce - 1, h, j0, tid, true);
   }
-  const int cc = (tid - 128) & (kSW - 1), cg = (tid - 128) / kSW, crows = DK / 4;
+  const int cc = (tid - 128) & (kSW - 1), cg = (tid - 128) / kSW, crows = DK / kCG;
   for (int pos = ce - 1; pos >= cb; --pos) {
     const size_t bh = (size_t)pos * H + h;
     const bool valid = p.mask == nullptr || p.mask[pos] != 0;
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
     const float *S = Sbuf[cur];
     if (pos > cb) prefetch(pos - 1, Sbuf[cur ^ 1]);   // overlaps the step below
     // ---- pass 1: row sums R1 = S dO, R4 = rowsum(G*S) (threads 0..127), column sums
-    //      p = S^T (a*k), C2 = G^T k over four row groups (threads 128..255)
+    //      p = S^T (a*k), C2 = G^T k over kCG row groups (threads 128..255)
     if (tid < 128) {
       const int i = tid;
       if (i < DK) {
@@ -245,9 +247,14 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
     }
     __syncthreads();
     if (tid < kSW) {
-      const float pj = (partp[0][tid] + partp[1][tid]) + (partp[2][tid] + partp[3][tid]);
+      float pj = 0.f, c2 = 0.f;
+#pragma unroll
+      for (int g = 0; g < kCG; ++g) {
+        pj += partp[g][tid];
+        c2 += partc[g][tid];
+      }
       sp[tid] = pj;
-      sc2[tid] = (partc[0][tid] + partc[1][tid]) + (partc[2][tid] + partc[3][tid]);
+      sc2[tid] = c2;
       su[tid] = beta * (sv[tid] - pj);
     }
     __syncthreads();
@@ -289,7 +296,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
     __syncthreads();      // G is read above and rewritten below
     // ---- pass 3: G <- Diag(a) (G + q dO^T + k dp^T)
     for (int e = tid; e < n4; e += kThreads) {
-      const int i = e >> 3, c = (e & 7) * 4;
+      const int i = e / kQ, c = (e % kQ) * 4;
       const float ai = sa[i], qi = sq[i], ki = sk[i];
       float4 gx = G4[e];
       gx.x = ai * (gx.x + qi * sdo[c] + ki * sdp[c]);
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) grad_kernel(BackwardParams p) {
   if (p.g_init_state) {
     float *O = p.g_init_state + ((size_t)b * H + h) * DK * DV + j0;
     for (int e = tid; e < n4; e += kThreads) {
-      const int i = e >> 3, c = (e & 7) * 4;
+      const int i = e / kQ, c = (e % kQ) * 4;
       *reinterpret_cast<float4 *>(O + (size_t)i * DV + c) = G4[e];
     }
   }
