@@ -192,6 +192,14 @@ def prefill_workspace_bytes(num_seqs: int) -> int:
     return int(load().kda_prefill_workspace_size(ctypes.byref(a)))
 
 
+def prefill_workspace(q, k, v, log_alpha, beta, cu_seqlens, chunk: int = 0) -> torch.Tensor:
+    """A device workspace of the size kda_prefill_workspace_size() states for these
+    arguments (for callers that allocate it once, e.g. before a CUDA graph capture)."""
+    a = prefill_args(q, k, v, log_alpha, beta, cu_seqlens, chunk=chunk)
+    nbytes = int(load().kda_prefill_workspace_size(ctypes.byref(a)))
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
             beta: torch.Tensor, cu_seqlens: torch.Tensor, pad_mask: Optional[torch.Tensor] = None,
             init_state: Optional[torch.Tensor] = None, o: Optional[torch.Tensor] = None,

@@ -33,6 +33,9 @@
  *     kda_get_device_status().  Kernels that follow a failed check on the same
  *     stream return without writing.
  *   - No C++ exception crosses the ABI.
+ *   - Every launch is stream-ordered, so the calls can be captured into a CUDA
+ *     graph; the first call on each device looks up the library's device error
+ *     word (cudaGetSymbolAddress), so make one call before capturing.
  *   - Layouts are row-major and contiguous.  N = total packed tokens,
  *     B = sequences (prefill) or rows (decode), H = heads.
  */
