@@ -1,7 +1,8 @@
 // Two-kernel tensor-core prefill: the state-independent work of every chunk
 // runs fully in parallel, the state pass runs once per (sequence, head, d_v
 // slice).  Same chunk algebra as the fused kernel (kda_prefill_tc.cu):
-//   intra (one CTA per chunk and head, all SMs):  Q G, K e^{g_C-g}, M = tril(Q G (K e^{-g})^T),
+//   intra (persistent CTAs over the (chunk, head) items, all SMs):  Q G, K e^{g_C-g},
+//     M = tril(Q G (K e^{-g})^T),
 //     T_b = (I + beta tril(K G (K e^{-g})^T))^{-1} Diag(beta), W = T_b K G, U_v = T_b V, e^{g_C}
 //   state pass (one CTA per sequence, head, 64 columns of d_v; chunks in order):
 //     U = U_v - W S;  O = (Q G) S + M U;  S <- Diag(e^{g_C}) S + (K e^{g_C-g})^T U
@@ -203,7 +204,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
     __syncthreads();
-    // ---- decay products and operand tiles (global loads overlap the V copy)
+    // ---- decay products and operand tiles (global loads; V is already on its way)
     {
       prep::PrepTiles t;
       t.qg = base + A_QK; t.qg_R = 128; t.qg_row0 = 0;
