@@ -61,3 +61,8 @@ def test_backward_bf16_head_gate_and_without_state():
 def test_backward_longer_sequences():
     """Two sequences of 1500 and 900 tokens, H = 4, d = 128, bf16, pads."""
     _run(104, [1500, 900], 4, 128, 128, "bf16", pads=True)
+
+
+def test_backward_empty_and_one_token_sequences():
+    """An empty sequence passes dS_final straight to dS0; one-token sequences."""
+    _run(105, [0, 1, 5, 0], 2, 64, 128, "f32")

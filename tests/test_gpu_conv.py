@@ -103,3 +103,15 @@ def test_conv_full_size_sampled():
     assert norm_err(to_np(y[torch.from_numpy(pos).cuda()]), ref) <= CTOL["bf16"]
     valid = np.nonzero(c["pad_mask"])[0][-(W - 1):]
     np.testing.assert_array_equal(to_np(so)[0], c["x"][valid])
+
+
+def test_conv_empty_sequences_keep_state():
+    """Zero-length sequences leave their state rows as they were (copied to state_out)."""
+    c = gen.conv_inputs(95, [0, 7, 0, 3], 64, 4, "f32", pad_frac=0.3)
+    d = _dev(c, "f32")
+    so = torch.empty_like(d["state"])
+    y = _run(d, so)
+    y_ref, s_ref = orc.short_conv(c["x"], c["weight"], c["bias"], c["cu_seqlens"], c["pad_mask"], c["state"])
+    assert norm_err(to_np(y), y_ref) <= CTOL["f32"]
+    np.testing.assert_array_equal(to_np(so), s_ref.astype(np.float32))
+    np.testing.assert_array_equal(to_np(so)[0], c["state"][0])
