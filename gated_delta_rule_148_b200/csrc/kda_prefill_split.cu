@@ -346,22 +346,72 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
 // named barrier.  The output accumulator is double-buffered in TMEM, so a
 // chunk's output epilogue runs while the next chunk's first product is in
 // flight.
+//
+// A CTA owns NS columns of d_v (64 or 32).  Columns of the state never mix in
+// the recurrence, so narrower slices give more CTAs independent chains with
+// shorter products and conversions.  The bf16 copies of S and U that feed the
+// products are MN-major tiles of NS columns: 128-byte rows with the 128-byte
+// swizzle for NS = 64, 64-byte rows with the 64-byte swizzle for NS = 32.
 constexpr int kComputeThreadsB = 256;
 constexpr int kThreadsB = kComputeThreadsB + 32;
 constexpr uint32_t BUF_WQ = 0, BUF_KT = 32768, BUF_UV = 49152, BUF_M = 57344, BUF_GC = 65536;
 constexpr uint32_t BUF_BYTES = 66560;
 constexpr uint32_t BUF_TX = 32768 + 16384 + 8192 + 8192 + 512;
-constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES, B_UB = B_SB + 128 * 128;
-constexpr uint32_t B_USED = B_UB + 64 * 128;
-constexpr uint32_t B_SMEM = B_USED + 1024;
-constexpr uint32_t B_TM_S = 0, B_TM_D1 = 64, B_TM_COLS = 256;   // D1 buffers at 64 and 128
+constexpr uint32_t B_BUF0 = 0, B_BUF1 = BUF_BYTES, B_SB = 2 * BUF_BYTES;
 
-__device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int tile,
+template <int NS>
+struct StateTiles {
+  static_assert(NS == 64 || NS == 32, "state slice of 64 or 32 columns");
+  static constexpr int kCols = NS / 2;               // d_v columns per compute thread
+  static constexpr uint32_t kRow = NS * 2;           // bytes per row of the S and U operand tiles
+  static constexpr uint32_t UB = B_SB + 128 * kRow;  // S: 128 rows (d_k), U: 64 rows (chunk)
+  static constexpr uint32_t SMEM = UB + 64 * kRow + 1024;
+  static constexpr uint32_t TM_S = 0, TM_D1 = NS;    // D1 buffers at NS and 2 NS
+  static constexpr uint32_t TM_COLS = NS == 64 ? 256 : 128;
+};
+
+// Row r (a K index) of an MN-major operand tile with NS bf16 columns; this
+// thread's NS/2 values start at 16-byte chunk chunk0.  64-byte rows: chunk c of
+// row r sits at c ^ ((r >> 1) & 3); 128-byte rows: at c ^ (r & 7).
+template <int NS>
+__device__ __forceinline__ void store_operand_row(unsigned char *tile, int r, int chunk0,
+                                                  const float *v) {
+#pragma unroll
+  for (int j = 0; j < NS / 2; j += 8) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
+    pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+    pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+    pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+    const int c = chunk0 + (j >> 3);
+    const uint32_t off = NS == 64 ? (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))
+                                  : (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    *reinterpret_cast<uint4 *>(tile + off) = pk;
+  }
+}
+
+// Descriptor of K-step s (tile rows 16 s .. 16 s + 15) of such a tile with R rows.
+template <int NS>
+__device__ __forceinline__ uint64_t desc_operand(uint32_t base, int R, int s) {
+  if constexpr (NS == 64) return desc_mnmajor(base, R, 0, s);
+  else return sdesc(base + (uint32_t)(16 * s * 64), (uint32_t)(R * 64), 512, 4);
+}
+
+template <int W>
+__device__ __forceinline__ void tmem_ldw(uint32_t taddr, float *v) {
+  if constexpr (W == 32) tmem_ld32(taddr, v); else tmem_ld16(taddr, v);
+}
+template <int W>
+__device__ __forceinline__ void tmem_stw(uint32_t taddr, const float *v) {
+  if constexpr (W == 32) tmem_st32(taddr, v); else tmem_st16(taddr, v);
+}
+
+__device__ __forceinline__ void load_item(unsigned char *buf, const unsigned char *it, int uv_blk,
                                           uint64_t *bar) {
   mbar_arrive_expect_tx(bar, BUF_TX);
   bulk_load(buf + BUF_WQ, it + IT_WQ, 32768, bar);
   bulk_load(buf + BUF_KT, it + IT_KT, 16384, bar);
-  bulk_load(buf + BUF_UV, it + IT_UV + tile * 8192, 8192, bar);
+  bulk_load(buf + BUF_UV, it + IT_UV + uv_blk * 8192, 8192, bar);
   bulk_load(buf + BUF_M, it + IT_M, 8192, bar);
   bulk_load(buf + BUF_GC, it + IT_GC, 512, bar);
 }
@@ -373,9 +423,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
 
+template <int NS>
 __global__ void __launch_bounds__(kThreadsB, 1)
 state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsigned char *items,
              int h0, int Hg) {
+  using T = StateTiles<NS>;
+  constexpr int kW = T::kCols;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
@@ -384,11 +437,11 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   __shared__ int err_sh;
 
   if (device_error_latched(p.err)) return;
-  const int tiles = p.dv / kNV;
+  const int tiles = p.dv / NS;
   const int tile = blockIdx.x % tiles;
   const int h = h0 + (blockIdx.x / tiles) % Hg;
   const int b = blockIdx.x / (tiles * Hg);
-  const int dv0 = tile * kNV;
+  const int dv0 = tile * NS;
   const int H = p.H, DV = p.dv;
   const SeqSpan sp = spans[b];
   const int nch = (sp.end - sp.begin + kC - 1) / kC;
@@ -398,9 +451,12 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   unsigned char *base = smem_raw + pad;
   const int tid = threadIdx.x, warp = tid >> 5, lr = tid & 127, wg = (tid >> 7) & 1;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
+  const uint32_t my_cols = lane_base + (uint32_t)(wg * kW);
+  // the item's U_v comes in 64-column blocks: this slice's block and this thread's first chunk in it
+  const int uv_blk = dv0 >> 6;
+  const int uv_c0 = ((dv0 & 63) >> 3) + wg * (kW / 8);
 
-  if (warp == 0) tmem_alloc(&tmem_base_sh, B_TM_COLS);
+  if (warp == 0) tmem_alloc(&tmem_base_sh, T::TM_COLS);
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
     mbar_init(&load_bar[0], 1);
@@ -424,50 +480,50 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         }
         if (*reinterpret_cast<volatile int *>(&err_sh)) break;
         load_item(base + ((j & 1) ? B_BUF1 : B_BUF0), items + ((size_t)(cb + j) * H + h) * ITEM_BYTES,
-                  tile, &load_bar[j & 1]);
+                  uv_blk, &load_bar[j & 1]);
       }
     }
   } else {
     // ---------------- compute warps
-    {   // initial state: thread owns state row lr, columns 32 wg .. 32 wg + 31
-      float v[32];
+    {   // initial state: thread owns state row lr, columns wg kW .. wg kW + kW - 1 of the slice
+      float v[kW];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32 + j] : 0.f;
-      tmem_st32(tm + my_cols + B_TM_S, v);
+      for (int j = 0; j < kW; ++j)
+        v[j] = p.init_state ? p.init_state[(((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * kW + j] : 0.f;
+      tmem_stw<kW>(tm + my_cols + T::TM_S, v);
       tmem_st_wait();
     }
-    const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + B_UB);
+    const uint32_t sSB = smem_u32(base + B_SB), sUB = smem_u32(base + T::UB);
     uint32_t phase = 0;
     bool ok = true;
 
-    // Chunk j: S -> bf16 operand, S *= e^{g_C}; then [-W ; Q G] S into D1[j & 1].
+    // Chunk j: S -> bf16 operand; [-W ; Q G] S into D1[j & 1]; then S *= e^{g_C}
+    // while that product runs (it reads the bf16 copy, not S).  The TMEM store
+    // is waited for before the product that accumulates into S is issued.
     auto begin_chunk = [&](int j) {
       unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
       if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles)) err_sh = 1;
-      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
-      float v[32];
-      tmem_ld32(tm + my_cols + B_TM_S, v);
-      prep::store_row32(base + B_SB, 128, lr, wg * 4, v);
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) v[jj] *= decay;
-      tmem_st32(tm + my_cols + B_TM_S, v);
-      tmem_st_wait();
+      float v[kW];
+      tmem_ldw<kW>(tm + my_cols + T::TM_S, v);
+      store_operand_row<NS>(base + B_SB, lr, wg * (kW / 8), v);
       fence_async_smem();
       fence_before_sync();
       compute_sync();
       if (tid == 0 && !err_sh) {
         fence_after_sync();
-        const uint32_t id = idesc_bf16(128, 64, 0, 1);
-        const uint32_t d1 = tm + B_TM_D1 + (uint32_t)((j & 1) * 64);
+        const uint32_t id = idesc_bf16(128, NS, 0, 1);
+        const uint32_t d1 = tm + T::TM_D1 + (uint32_t)((j & 1) * NS);
         const uint64_t a0 = desc_kmajor(smem_u32(buf) + BUF_WQ, 128, 0, 0);
-        const uint64_t b0 = desc_mnmajor(sSB, 128, 0, 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           mma_bf16(d1, a0 + (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4),
-                   b0 + (uint64_t)((16 * s * 128) >> 4), id, s > 0);
+                   desc_operand<NS>(sSB, 128, s), id, s > 0);
         mma_commit(&mma_bar);
       }
+      const float decay = reinterpret_cast<const float *>(buf + BUF_GC)[lr];
+#pragma unroll
+      for (int jj = 0; jj < kW; ++jj) v[jj] *= decay;
+      tmem_stw<kW>(tm + my_cols + T::TM_S, v);
     };
 
     if (nch > 0) begin_chunk(0);
@@ -475,27 +531,37 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       const int c0 = sp.begin + j * kC;
       unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
       const uint32_t sbuf = smem_u32(buf);
-      const uint32_t d1 = B_TM_D1 + (uint32_t)((j & 1) * 64);
+      const uint32_t d1 = T::TM_D1 + (uint32_t)((j & 1) * NS);
+      // operands of this chunk's conversions that do not depend on the product
+      uint4 uv[kW / 8];
+      bool o_valid = false;
+      if ((warp & 3) < 2) {
+#pragma unroll
+        for (int q = 0; q < kW / 8; ++q)
+          uv[q] = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(lr, 0, uv_c0 + q, kC));
+      } else {
+        const int pos = c0 + lr - kC;
+        o_valid = pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
+      }
       // ---- wait for [-W S ; (Q G) S]; U = U_v - W S (lanes 0-63) -> bf16 operand
       if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
       phase++;
       fence_after_sync();
       if ((warp & 3) < 2) {
-        const int r = lr;
-        float v[32];
-        tmem_ld32(tm + my_cols + d1, v);
+        float v[kW];
+        tmem_ldw<kW>(tm + my_cols + d1, v);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(buf + BUF_UV + row_tile_chunk(r, 0, wg * 4 + q, kC));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int q = 0; q < kW / 8; ++q) {
+          const uint32_t w[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             v[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
             v[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
           }
         }
-        prep::store_row32(base + B_UB, 64, r, wg * 4, v);
+        store_operand_row<NS>(base + T::UB, lr, wg * (kW / 8), v);
       }
+      tmem_st_wait();      // S *= e^{g_C} has landed
       fence_async_smem();
       fence_before_sync();
       compute_sync();
@@ -503,17 +569,16 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       // ---- O += [x ; M] U (rows 0-63 of the result are not used);  S += (K e^{g_C-g})^T U
       if (tid == 0) {
         fence_after_sync();
-        const uint32_t ido = idesc_bf16(128, 64, 0, 1);
-        const uint32_t ids = idesc_bf16(128, 64, 1, 1);
+        const uint32_t ido = idesc_bf16(128, NS, 0, 1);
+        const uint32_t ids = idesc_bf16(128, NS, 1, 1);
         const uint64_t ao = desc_kmajor(sbuf + BUF_UV, 128, 0, 0);
         const uint64_t as = desc_mnmajor(sbuf + BUF_KT, 64, 0, 0);
-        const uint64_t bu = desc_mnmajor(sUB, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), bu + (uint64_t)((16 * s * 128) >> 4), ido, 1);
+          mma_bf16(tm + d1, ao + (uint64_t)(s * 2), desc_operand<NS>(sUB, 64, s), ido, 1);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-          mma_bf16(tm + B_TM_S, as + (uint64_t)((16 * s * 128) >> 4), bu + (uint64_t)((16 * s * 128) >> 4), ids, 1);
+          mma_bf16(tm + T::TM_S, as + (uint64_t)((16 * s * 128) >> 4), desc_operand<NS>(sUB, 64, s), ids, 1);
         mma_commit(&mma_bar);
       }
       if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
@@ -526,23 +591,23 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       if ((warp & 3) >= 2) {
         const int r = lr - kC;
         const int pos = c0 + r;
-        float v[32];
-        tmem_ld32(tm + my_cols + d1, v);
+        float v[kW];
+        tmem_ldw<kW>(tm + my_cols + d1, v);
         if (pos < sp.end) {
-          const bool valid = p.mask == nullptr || p.mask[pos] != 0;
-          uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * 32;
+          uint16_t *orow = reinterpret_cast<uint16_t *>(p.o) + ((size_t)pos * H + h) * DV + dv0 + wg * kW;
 #pragma unroll
-          for (int jj = 0; jj < 32; jj += 8) {
+          for (int jj = 0; jj < kW; jj += 8) {
             uint4 pk;
-            pk.x = valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
-            pk.y = valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
-            pk.z = valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
-            pk.w = valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
+            pk.x = o_valid ? pack_bf16x2(v[jj + 0], v[jj + 1]) : 0u;
+            pk.y = o_valid ? pack_bf16x2(v[jj + 2], v[jj + 3]) : 0u;
+            pk.z = o_valid ? pack_bf16x2(v[jj + 4], v[jj + 5]) : 0u;
+            pk.w = o_valid ? pack_bf16x2(v[jj + 6], v[jj + 7]) : 0u;
             *reinterpret_cast<uint4 *>(orow + jj) = pk;
           }
         }
       }
     }
+    tmem_st_wait();
     compute_sync();
     ok = ok && !*reinterpret_cast<volatile int *>(&err_sh);
     if (!ok) {
@@ -552,11 +617,11 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       }
       if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
     } else if (p.final_state) {
-      float v[32];
-      tmem_ld32(tm + my_cols + B_TM_S, v);
-      float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * 32;
+      float v[kW];
+      tmem_ldw<kW>(tm + my_cols + T::TM_S, v);
+      float *dst = p.final_state + (((size_t)b * H + h) * kDK + lr) * DV + dv0 + wg * kW;
 #pragma unroll
-      for (int jj = 0; jj < 32; jj += 4)
+      for (int jj = 0; jj < kW; jj += 4)
         *reinterpret_cast<float4 *>(dst + jj) = make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
     }
     if (tid == 0 && !ok) {
@@ -568,7 +633,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   __syncthreads();
   if (warp == 0) {
     fence_after_sync();
-    tmem_dealloc(tm, B_TM_COLS);
+    tmem_dealloc(tm, T::TM_COLS);
   }
 }
 
@@ -638,15 +703,20 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   auto intra = p.gate_head ? intra_kernel<true> : intra_kernel<false>;
   e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)B_SMEM);
+  // 32-column state slices while they fit one wave (more independent chains, shorter products);
+  // 64-column slices once there are more chains than SMs (less work per column in total).
+  const bool narrow = (size_t)p.num_seqs * p.H * (p.dv / 32) <= (size_t)num_sms();
+  auto state = narrow ? state_kernel<32> : state_kernel<64>;
+  const uint32_t smem_b = narrow ? StateTiles<32>::SMEM : StateTiles<64>::SMEM;
+  e = cudaFuncSetAttribute(state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
   if (e != cudaSuccess) return e;
   const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
   if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
   const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
   intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, 0, p.H);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / kNV);
-  state_kernel<<<gridB, kThreadsB, B_SMEM, s>>>(p, spans, cbase, items, 0, p.H);
+  const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / (narrow ? 32 : 64));
+  state<<<gridB, kThreadsB, smem_b, s>>>(p, spans, cbase, items, 0, p.H);
   return cudaGetLastError();
 }
 
