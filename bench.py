@@ -439,6 +439,9 @@ def main_ours(args, rank, world, device):
             "log_alpha": "[N, H] fp32", "l2": "inputs larger than L2"}
         line["gpu_launches"] += LAUNCHES_PER_PREFILL * K
         del devh
+        # ---- chunk-size sweep on the path that takes every chunk size (CUDA cores, fp32 q/k/v)
+        line["prefill_chunk_sweep"] = bench_chunk_sweep(K, W, device)
+        line["gpu_launches"] += 2 * 3 * (K + W)
         # ---- backward pass at T = 4096 (token-serial fp32, reference grade)
         line["backward"] = bench_backward(K, W, world, device, pk)
         line["gpu_launches"] += 2 * K
@@ -451,6 +454,28 @@ def main_ours(args, rank, world, device):
         line["cpu_baseline"] = cpu_baseline(inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def bench_chunk_sweep(K, W, device, T=16384):
+    """kda_prefill with fp32 q, k, v (the CUDA-core path) at chunk 16, 32 and 64: B=1, H=32,
+    d=128, the headline workload's first T tokens.  Per-call ms; the tensor-core path's bf16
+    chunk-64 call at the same T is the prefill_sweep entry."""
+    import torch
+    from gated_delta_rule_148_b200 import kda
+    _, _, _, d = prefill_setup(T, device)
+    for key in ("q", "k", "v"):
+        d[key] = d[key].float()
+    d["o"] = torch.empty(d["o"].shape, dtype=torch.float32, device=device)
+    out = {"workload": f"prefill_T{T}_H32_d128_f32_simt", "path": "CUDA cores (fp32 FMA)"}
+    for c in (16, 32, 64):
+        fn = lambda: kda.prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                 d["cu_seqlens"], o=d["o"], final_state=d["fs"], chunk=c)
+        ms = time_loop(fn, K, W)
+        out[str(c)] = {"ms": ms, "tokens_per_s": T / (ms / 1e3)}
+    st = kda.get_device_status()
+    if st != kda.KDA_OK:
+        raise RuntimeError("device status after the chunk sweep: " + kda.status_string(st))
+    return out
 
 
 def bench_decode(args, world, device, pk):

@@ -4,7 +4,7 @@
 //   intra (persistent CTAs over the (chunk, head) items, all SMs):  Q G, K e^{g_C-g},
 //     M = tril(Q G (K e^{-g})^T),
 //     T_b = (I + beta tril(K G (K e^{-g})^T))^{-1} Diag(beta), W = T_b K G, U_v = T_b V, e^{g_C}
-//   state pass (one CTA per sequence, head, 64 columns of d_v; chunks in order):
+//   state pass (one CTA per sequence, head, 32 or 64 columns of d_v; chunks in order):
 //     U = U_v - W S;  O = (Q G) S + M U;  S <- Diag(e^{g_C}) S + (K e^{g_C-g})^T U
 // ("Kimi Linear's 75% KV cache cut ...", theclarity.today, fourth paragraph:
 // chunks and the WY representation; "Kimi Linear wlasnie pokonal ...",

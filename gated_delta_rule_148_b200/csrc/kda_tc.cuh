@@ -1,15 +1,18 @@
 // sm_100a tensor-core primitives used by the prefill kernel: TMEM allocation,
 // tcgen05.mma (bf16 in, fp32 accumulate), tcgen05.ld/st, shared-memory
-// matrix descriptors for 128-byte-swizzled tiles, mbarriers with bounded
-// waits, and cp.async staging.
+// matrix descriptors for 128- and 64-byte-swizzled tiles, mbarriers with
+// bounded waits, and cp.async staging.
 //
-// Shared-memory tile layouts (bf16, all bases 1024-byte aligned):
+// Shared-memory tile layouts (bf16):
 //   K-major "row tile" R x K: K split in blocks of 64 elements (128 B); block
 //     kb holds R rows of 128 B at kb*R*128; the 16-byte chunk c of row r sits
 //     at chunk position c ^ (r & 7) (the 128-byte swizzle).  As an MMA operand
 //     its rows are the M (or N) index and its columns the K index.
 //   The same bytes read as an MN-major operand: rows are the K index and the
-//     64-element blocks of a row run along M (or N).
+//     64-element blocks of a row run along M (or N).  Bases 1024-byte aligned.
+//   A 32-column MN-major tile: 64-byte rows (the K index); the 16-byte chunk c
+//     of row r sits at chunk position c ^ ((r >> 1) & 3) (the 64-byte swizzle);
+//     8-row groups 512 bytes apart; base 512-byte aligned.
 #pragma once
 
 #include <cuda.h>
