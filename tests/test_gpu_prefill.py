@@ -289,3 +289,20 @@ def test_many_short_sequences_two_kernel_path():
     o, fs = _gpu(inp, "bf16")
     _check(inp, "bf16", o, fs)
     assert np.all(to_np(o)[m == 0] == 0.0)
+
+
+def test_state_slice_width_does_not_change_results():
+    """One sequence of 32 heads runs its state pass in 32-column slices (128 chains fit the
+    SMs); the same sequence next to a second one runs it in 64-column slices (256 chains).
+    Columns of the state never mix, so the shared sequence's outputs and final state are
+    bit-identical between the two."""
+    lengths = [777, 300]
+    inp = gen.random_case(81, lengths, 32, 128, 128, "bf16", init_state=True)
+    o2, fs2 = _gpu(inp, "bf16")
+    solo = {k: inp[k][:lengths[0]] for k in ("q", "k", "v", "log_alpha", "beta")}
+    solo["cu_seqlens"] = np.array([0, lengths[0]], np.int32)
+    solo["init_state"] = inp["init_state"][:1]
+    o1, fs1 = _gpu(solo, "bf16")
+    assert torch.equal(o2[:lengths[0]], o1)
+    assert torch.equal(fs2[:1], fs1)
+    _check(solo, "bf16", o1, fs1)
