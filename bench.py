@@ -441,7 +441,7 @@ def main_ours(args, rank, world, device):
         del devh
         # ---- chunk-size sweep on the path that takes every chunk size (CUDA cores, fp32 q/k/v)
         line["prefill_chunk_sweep"] = bench_chunk_sweep(K, W, device)
-        line["gpu_launches"] += 2 * 3 * (K + W)
+        line["gpu_launches"] += 2 * 3 * K
         # ---- backward pass at T = 4096 (token-serial fp32, reference grade)
         line["backward"] = bench_backward(K, W, world, device, pk)
         line["gpu_launches"] += 2 * K
