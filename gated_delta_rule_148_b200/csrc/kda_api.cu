@@ -2,6 +2,7 @@
 //
 // Every entry point validates on the host first and launches nothing on an
 // argument error.  See include/kda.h for the contract of each call.
+#include <atomic>
 #include <cstring>
 
 #include "kda_internal.cuh"
@@ -14,19 +15,27 @@ __device__ unsigned g_error_word;
 namespace {
 
 constexpr int kMaxDevices = 64;
-unsigned *g_err_ptr[kMaxDevices];   // cached device address, per device
+// Device address of g_error_word, per device.  Threads that make their first call on a
+// device at the same time both look it up and store the same value.
+std::atomic<unsigned *> g_err_ptr[kMaxDevices];
 
 kda_status error_word(unsigned **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
-  if (g_err_ptr[dev] == nullptr) {
+  unsigned *cached = g_err_ptr[dev].load(std::memory_order_acquire);
+  if (cached == nullptr) {
     void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return KDA_ERR_CUDA;
-    g_err_ptr[dev] = static_cast<unsigned *>(ptr);
+    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess || ptr == nullptr) return KDA_ERR_CUDA;
+    cached = static_cast<unsigned *>(ptr);
+    g_err_ptr[dev].store(cached, std::memory_order_release);
   }
-  *out = g_err_ptr[dev];
+  *out = cached;
   return KDA_OK;
 }
+
+// Test faults and the bounded-wait limit (kda_debug_set_fault); process-wide.
+std::atomic<int> g_fault{0};
+std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
 
 struct Range {
   const void *p;
@@ -154,6 +163,8 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   p.final_state = a->final_state;
   p.err = err;
   p.gate_head = gate_head ? 1 : 0;
+  p.wait_cycles = g_wait_cycles.load(std::memory_order_relaxed);
+  p.fault = g_fault.load(std::memory_order_relaxed);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = a->dtype == KDA_BF16;
   p.spans = nullptr;
@@ -334,6 +345,13 @@ kda_status kda_prefill_backward(const kda_backward_args *a, void *stream) {
   p.gate_head = gate_head ? 1 : 0;
   return launch_backward(p, a->dtype == KDA_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_debug_set_fault(int fault, long long wait_cycles) {
+  if (fault & ~FAULT_STARVE_STATE_LOADS) return KDA_ERR_INVALID_ARG;
+  g_fault.store(fault, std::memory_order_relaxed);
+  g_wait_cycles.store(wait_cycles > 0 ? wait_cycles : kDefaultWaitCycles, std::memory_order_relaxed);
+  return KDA_OK;
 }
 
 kda_status kda_get_device_status(void *stream) {

@@ -8,6 +8,15 @@
 // theclarity.today, fourth paragraph, WY form of a chunk):
 //   e^{g_r} = prod_{j<=r} a_j,  e^{g_C - g_r} = prod_{j>r} a_j,  e^{-g_r} = e^{g_C - g_r} / e^{g_C}
 //   Q G = q e^{g},  K G = k e^{g},  K e^{-g},  K e^{g_C - g}  (bf16 operand tiles)
+//
+// Range of the factorised Gram.  The Gram products take e^{g_r - g_i} as
+// e^{g_r} * e^{-g_i}; e^{-g_i} <= e^{-g_C} stays representable (and far from
+// overflow in the products) while a channel's log-decay over the chunk is above
+// ln(kFastMinDecay) ~ -60.  A channel below that ("unsafe") gets a zero column
+// in K e^{-g}, so the tensor-core Gram holds the other channels' terms only,
+// and exact_gram_fixup() adds its terms with running products of alpha on the
+// CUDA cores (every factor <= 1, exact for any log_alpha <= 0).  The other
+// tiles only use factors <= 1 and need no special case.
 #pragma once
 
 #include "kda_internal.cuh"
@@ -20,6 +29,16 @@ using namespace tc;
 
 constexpr int kC = 64;
 constexpr int kDK = 128;
+constexpr float kFastMinDecay = 1e-26f;   // e^{g_C} below this: the channel takes the exact path
+
+// Marks channels c, c + 1 whose chunk decay e^{g_C} is below kFastMinDecay in the
+// 4-word mask `unsafe` (zeroed by the caller before the prep) and returns the
+// factors e^{-g_C} the tiles use (0 for an unsafe channel: its K e^{-g} column is 0).
+__device__ __forceinline__ float2 gram_inv_decay(float GC0, float GC1, int c, uint32_t *unsafe) {
+  const bool u0 = !(GC0 > kFastMinDecay), u1 = !(GC1 > kFastMinDecay);
+  if (u0 | u1) atomicOr(&unsafe[c >> 5], ((u0 ? 1u : 0u) | (u1 ? 2u : 0u)) << (c & 31));
+  return make_float2(u0 ? 0.f : 1.f / GC0, u1 ? 0.f : 1.f / GC1);
+}
 
 struct PrepTiles {
   unsigned char *qg;      // Q G rows (K-major row tile `qg_R` rows, starting row `qg_row0`)
@@ -39,7 +58,7 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
                                                 const float *sg, const uint32_t *valid,
                                                 const PrepTiles &t, float (*part)[kDK],
                                                 float *decay, const float *beta_in,
-                                                float *beta_out, int tid) {
+                                                float *beta_out, uint32_t *unsafe, int tid) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -69,8 +88,9 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
     decay[c] = GC0;
     decay[c + 1] = GC1;
   }
-  // e^{-g_C}, clamped where e^{g_C} underflows (outside the tensor-core path's domain)
-  const float inv0 = GC0 > 1e-35f ? 1.f / GC0 : 1e35f, inv1 = GC1 > 1e-35f ? 1.f / GC1 : 1e35f;
+  // e^{-g_C}; 0 for channels that take the exact path (their K e^{-g} column is zero)
+  const float2 inv = gram_inv_decay(GC0, GC1, c, unsafe);
+  const float inv0 = inv.x, inv1 = inv.y;
   const uint32_t *sq = reinterpret_cast<const uint32_t *>(sq16);
   const uint32_t *sk = reinterpret_cast<const uint32_t *>(sk16);
   const int kb = c >> 6, ch = (c & 63) >> 3;
@@ -124,8 +144,8 @@ template <bool GATE_HEAD>
 __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
-    float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out, int tid,
-    bool wait_bulk = false) {
+    float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out,
+    uint32_t *unsafe, int tid, bool wait_bulk = false) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -178,7 +198,8 @@ __device__ __forceinline__ void decay_and_tiles_global(
     decay[c + 1] = GC1;
     *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
   }
-  const float inv0 = GC0 > 1e-35f ? 1.f / GC0 : 1e35f, inv1 = GC1 > 1e-35f ? 1.f / GC1 : 1e35f;
+  const float2 inv = gram_inv_decay(GC0, GC1, c, unsafe);
+  const float inv0 = inv.x, inv1 = inv.y;
   const int kb = c >> 6, ch = (c & 63) >> 3;
   const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
   const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
@@ -271,6 +292,86 @@ __device__ __forceinline__ void pack_tb(const float *Ts, const float *beta, unsi
     pk.w = pack_bf16x2(t[j + 6], t[j + 7]);
     *reinterpret_cast<uint4 *>(ttile + row_tile_chunk(r, 0, (qq * 16 + j) >> 3, R)) = pk;
   }
+}
+
+// Exact Gram terms of the unsafe channels (see the range note at the top).  The
+// tensor-core Gram in TMEM (lanes 0-63: M rows, lanes 64-127: rows of K K^T before
+// beta; this thread's 32 columns at `tm_acc`) holds every other channel's terms;
+// this adds, for each unsafe channel c and i <= r,
+//   x[r][c] k[i][c] prod_{i < t <= r} alpha[t][c]      (x = q for M rows, k for A rows)
+// with running products of alpha (all factors <= 1, so no overflow for any
+// log_alpha <= 0; a term underflows only where its true value is below 1e-38).
+// Rows outside `valid` count as alpha = 1, q = k = 0 (identity steps).  q, k and
+// log_alpha are read from global memory (rows c0 .. c0 + 63 of head h).
+// `stage`: >= 12800 bytes of shared memory.  All 256 threads; contains
+// __syncthreads().  The caller skips it when the mask is empty.
+template <bool GATE_HEAD>
+__device__ __noinline__ void exact_gram_fixup(uint32_t tm_acc, const uint32_t *unsafe,
+                                              const uint32_t *valid, const uint16_t *q,
+                                              const uint16_t *k, const float *log_alpha, int c0,
+                                              int h, int H, float *stage, int tid) {
+  int *list = reinterpret_cast<int *>(stage);   // unsafe channels, ascending
+  float *sa = stage + 128;                      // [16][64] alpha of a group of channels
+  float *sx = sa + 16 * 64;                     // [16][64] q
+  float *sk = sx + 16 * 64;                     // [16][64] k
+  const int n = __popc(unsafe[0]) + __popc(unsafe[1]) + __popc(unsafe[2]) + __popc(unsafe[3]);
+  if (tid < kDK) {
+    const uint32_t w = unsafe[tid >> 5], bit = 1u << (tid & 31);
+    if (w & bit) {
+      int pos = __popc(w & (bit - 1u));
+      for (int j = 0; j < (tid >> 5); ++j) pos += __popc(unsafe[j]);
+      list[pos] = tid;
+    }
+  }
+  const int L = tid & 127, wg = tid >> 7, r = L & 63;
+  const bool rowA = L >= kC;
+  const int ibase = wg * 32;
+  const int ihi = min(ibase + 31, r);
+  float acc[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u) acc[u] = 0.f;
+  for (int g0 = 0; g0 < n; g0 += 16) {
+    __syncthreads();   // the list is written; the previous group's reads are done
+    for (int e = tid; e < 16 * kC; e += 256) {
+      const int j = e >> 6, rr = e & 63;
+      float a = 1.f, xq = 0.f, xk = 0.f;
+      if (g0 + j < n && ((valid[rr >> 5] >> (rr & 31)) & 1u)) {
+        const int c = list[g0 + j];
+        const size_t row = (size_t)(c0 + rr) * H + h;
+        a = __expf(GATE_HEAD ? log_alpha[row] : log_alpha[row * kDK + c]);
+        xq = bf16_to_f32(q[row * kDK + c]);
+        xk = bf16_to_f32(k[row * kDK + c]);
+      }
+      sa[j * kC + rr] = a;
+      sx[j * kC + rr] = xq;
+      sk[j * kC + rr] = xk;
+    }
+    __syncthreads();
+    const int jn = min(16, n - g0);
+    for (int j = 0; j < jn; ++j) {
+      const float *aj = sa + j * kC, *kj = sk + j * kC;
+      float xP = rowA ? kj[r] : sx[j * kC + r];
+      for (int t = ihi + 1; t <= r; ++t) xP *= aj[t];      // prod over (ihi, r]
+#pragma unroll
+      for (int u = 31; u >= 0; --u) {
+        const int i = ibase + u;
+        if (i <= r) {
+          acc[u] = fmaf(xP, kj[i], acc[u]);
+          xP *= aj[i];
+        }
+      }
+    }
+  }
+  float v[32];
+  tmem_ld32(tm_acc, v);
+#pragma unroll
+  for (int u = 0; u < 32; ++u) v[u] += acc[u];
+  tmem_st32(tm_acc, v);
+  tmem_st_wait();
+}
+
+__device__ __forceinline__ bool any_unsafe(const uint32_t *unsafe) {
+  return (unsafe[0] | unsafe[1] | unsafe[2] | unsafe[3]) != 0u;
 }
 
 }  // namespace prep

@@ -36,7 +36,16 @@ struct PrefillParams {
   const SeqSpan *spans;   // NULL: spans are [cu[b], cu[b+1])
   unsigned *err;          // device error word
   int gate_head;          // 1: log_alpha is [N, H] (one gate per token and head)
+  long long wait_cycles;  // limit of every bounded device wait
+  int fault;              // test faults (FAULT_*), 0 in normal use
 };
+
+// Faults a test can plant with kda_debug_set_fault() to exercise the bounded
+// waits; none of them touches memory out of bounds.
+enum : int {
+  FAULT_STARVE_STATE_LOADS = 1,   // the state pass issues no item loads: its waits run out
+};
+constexpr long long kDefaultWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 
 struct DecodeParams {
   int B, H, dk, dv;

@@ -25,6 +25,8 @@
 //     (cudaGetSymbolAddress, with that device current); make that first call
 //     before any stream capture.
 // No cudaMalloc, cudaFree or allocating library routine is called here.
+#include <atomic>
+
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -36,20 +38,23 @@ static __device__ __align__(256) unsigned char
     g_noalloc_scratch[KDA_NOALLOC_MAX_SEQS * sizeof(SeqSpan)];
 
 // Device address of g_noalloc_scratch, per device (the host-side symbol is only
-// a stand-in and must never be handed to a kernel).
-void *g_noalloc_ptr[kMaxDevicesNoAlloc];
+// a stand-in and must never be handed to a kernel).  Two threads whose first
+// calls on a device overlap both look the address up and store the same value.
+std::atomic<void *> g_noalloc_ptr[kMaxDevicesNoAlloc];
 
 kda_status noalloc_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesNoAlloc)
     return KDA_ERR_CUDA;
-  if (g_noalloc_ptr[dev] == nullptr) {
+  void *cached = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (cached == nullptr) {
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
       return KDA_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
+    g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+    cached = ptr;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = cached;
   return KDA_OK;
 }
 

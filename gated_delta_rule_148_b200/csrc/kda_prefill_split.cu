@@ -34,7 +34,6 @@ namespace split {
 using namespace tc;
 
 constexpr int kC = 64, kDK = 128, kNV = 64;
-constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 
 // ---- item layout
 constexpr uint32_t IT_WQ = 0, IT_KT = 32768, IT_UV = 49152, IT_M = 65536, IT_GC = 73728;
@@ -148,6 +147,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t v_bar;
   __shared__ uint32_t valid_sh[2];
+  __shared__ uint32_t unsafe_sh[4];     // channels whose Gram terms take the exact path
   __shared__ float decay_sh[kDK];
   __shared__ float beta_sh[kC];
   __shared__ float part_sh[4][kDK];
@@ -203,6 +203,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
       if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
+    if (tid < 4) unsafe_sh[tid] = 0u;
     __syncthreads();
     // ---- decay products and operand tiles (global loads; V is already on its way)
     {
@@ -214,7 +215,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       prep::decay_and_tiles_global<GATE_HEAD>(
           reinterpret_cast<const uint16_t *>(p.q), reinterpret_cast<const uint16_t *>(p.k), p.log_alpha,
           c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
-          decay_sh, beta_val, beta_sh, tid, !first);
+          decay_sh, beta_val, beta_sh, unsafe_sh, tid, !first);
     }
     fence_async_smem();
     __syncthreads();
@@ -232,10 +233,15 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       bulk_store(it + IT_KT, base + A_TS, 64 * 256);
       bulk_commit();
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
+    if (prep::any_unsafe(unsafe_sh))     // K e^{-g} is no longer needed: its region stages the fix-up
+      prep::exact_gram_fixup<GATE_HEAD>(tm + my_cols + A_TM_GW, unsafe_sh, valid_sh,
+                                        reinterpret_cast<const uint16_t *>(p.q),
+                                        reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
+                                        reinterpret_cast<float *>(base + A_KH), tid);
     float *As = reinterpret_cast<float *>(base + A_KH);     // K e^{-g} is no longer needed
     float *Ts = reinterpret_cast<float *>(base + A_TS);
     float *Xs = reinterpret_cast<float *>(base + A_XS);
@@ -262,7 +268,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     tri::unit_lower_inverse_64(As, Ts, Xs, tid);
     prep::pack_tb(Ts, beta_sh, base + A_TB, 128, tid);
     fence_async_smem();
-    ok = __syncthreads_and(mbar_wait(&v_bar, vphase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&v_bar, vphase & 1, p.wait_cycles));
     vphase++;
     if (!ok) break;
     // zero V rows of invalid positions (tail of the sequence, pads)
@@ -287,7 +293,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
         mma_bf16(tm + A_TM_UV, desc_kmajor(sTB, 128, 0, s), desc_mnmajor(sV, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -325,7 +331,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
     mbar_wait(&v_bar, (vphase - 0) & 1, 20000);
-    if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+    if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
   }
   if (tid == 0) {
     bulk_commit();
@@ -472,9 +478,9 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
 
   if (warp == kComputeThreadsB / 32) {
     // ---------------- producer warp: item loads, two chunks ahead of the chain
-    if ((tid & 31) == 0) {
+    if ((tid & 31) == 0 && !(p.fault & FAULT_STARVE_STATE_LOADS)) {
       for (int j = 0; j < nch; ++j) {
-        if (j >= 2 && !mbar_wait(&free_bar[j & 1], ((j - 2) >> 1) & 1, kWaitCycles)) {
+        if (j >= 2 && !mbar_wait(&free_bar[j & 1], ((j - 2) >> 1) & 1, p.wait_cycles)) {
           atomicOr(p.err, ERR_BIT_TIMEOUT);
           break;
         }
@@ -502,7 +508,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     // is waited for before the product that accumulates into S is issued.
     auto begin_chunk = [&](int j) {
       unsigned char *buf = base + ((j & 1) ? B_BUF1 : B_BUF0);
-      if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, kWaitCycles)) err_sh = 1;
+      if (!mbar_wait(&load_bar[j & 1], (j >> 1) & 1, p.wait_cycles)) err_sh = 1;
       float v[kW];
       tmem_ldw<kW>(tm + my_cols + T::TM_S, v);
       store_operand_row<NS>(base + B_SB, lr, wg * (kW / 8), v);
@@ -544,7 +550,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         o_valid = pos < sp.end && (p.mask == nullptr || p.mask[pos] != 0);
       }
       // ---- wait for [-W S ; (Q G) S]; U = U_v - W S (lanes 0-63) -> bf16 operand
-      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      if (!mbar_wait(&mma_bar, phase & 1, p.wait_cycles)) err_sh = 1;
       phase++;
       fence_after_sync();
       if ((warp & 3) < 2) {
@@ -581,7 +587,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
           mma_bf16(tm + T::TM_S, as + (uint64_t)((16 * s * 128) >> 4), desc_operand<NS>(sUB, 64, s), ids, 1);
         mma_commit(&mma_bar);
       }
-      if (!mbar_wait(&mma_bar, phase & 1, kWaitCycles)) err_sh = 1;
+      if (!mbar_wait(&mma_bar, phase & 1, p.wait_cycles)) err_sh = 1;
       phase++;
       fence_after_sync();
       if (tid == 0) mbar_arrive(&free_bar[j & 1]);     // the products that read buffer j & 1 are done
@@ -615,7 +621,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         err_sh = 1;
         atomicOr(p.err, ERR_BIT_TIMEOUT);
       }
-      if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+      if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
     } else if (p.final_state) {
       float v[kW];
       tmem_ldw<kW>(tm + my_cols + T::TM_S, v);

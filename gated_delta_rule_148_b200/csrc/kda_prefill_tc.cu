@@ -30,10 +30,10 @@
 // Exactness: masked and tail rows enter as zeros (and identity gates);
 // upper-triangle entries are zeroed by selection before any product uses
 // them, so an output row never depends on a later row's values.
-// Numerical domain of this path: the factorisation e^{g_r - g_i} =
-// e^{g_r} e^{-g_i} needs e^{-g} finite, i.e. a per-channel cumulative
-// log-decay >= -80 within each 64-token chunk (the fp32 CUDA-core path has no
-// such limit).
+// Range: the factorisation e^{g_r - g_i} = e^{g_r} e^{-g_i} is used for the
+// channels whose log-decay over the chunk stays above about -60; the Gram terms
+// of any other channel are computed exactly on the CUDA cores
+// (prep::exact_gram_fixup), so the path holds for every log_alpha <= 0.
 #include <climits>
 
 #include <cudaTypedefs.h>
@@ -52,7 +52,6 @@ constexpr int kC = 64;       // chunk
 constexpr int kDK = 128;     // key dim
 constexpr int kNV = 64;      // d_v columns per CTA
 constexpr int kThreads = 256;
-constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 1.9 GHz
 
 // Shared-memory map (bytes from a 1024-aligned base).
 constexpr uint32_t OFF_QKW = 0;                       // [-W | Q G | K G] 192 x 128 row tile
@@ -139,6 +138,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
   __shared__ __align__(8) uint64_t stage_bar;
   __shared__ __align__(8) uint64_t v_bar;
   __shared__ uint32_t valid_sh[2];      // validity bits of the chunk's 64 rows
+  __shared__ uint32_t unsafe_sh[4];     // channels whose Gram terms take the exact path
   __shared__ float decay_sh[kDK];      // e^{g_C} per key channel
   __shared__ float beta_sh[kC];
   __shared__ float part_sh[4][kDK];
@@ -209,7 +209,8 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
       const unsigned bits = __ballot_sync(0xFFFFFFFFu, row_valid(p, sp, c0 + tid));
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
     }
-    ok = __syncthreads_and(mbar_wait(&stage_bar, chunk_idx & 1, kWaitCycles));
+    if (tid < 4) unsafe_sh[tid] = 0u;
+    ok = __syncthreads_and(mbar_wait(&stage_bar, chunk_idx & 1, p.wait_cycles));
     if (!ok) break;
     // ---- P1: decay products and operand tiles
     {
@@ -221,7 +222,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
       prep::decay_and_tiles(reinterpret_cast<const uint16_t *>(base + OFF_STQ),
                             reinterpret_cast<const uint16_t *>(base + OFF_STK),
                             reinterpret_cast<const float *>(base + OFF_STG), valid_sh, t, part_sh,
-                            decay_sh, stb, beta_sh, tid);
+                            decay_sh, stb, beta_sh, unsafe_sh, tid);
     }
     fence_async_smem();
     __syncthreads();
@@ -233,10 +234,17 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_G, desc_kmajor(sQKW, 192, 64, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
+    // channels whose chunk decay is out of the factorised range: exact terms added
+    // (K e^{-g} has been read by the Gram: its region stages the fix-up)
+    if (prep::any_unsafe(unsafe_sh))
+      prep::exact_gram_fixup<false>(tm + my_cols + TM_G, unsafe_sh, valid_sh,
+                                    reinterpret_cast<const uint16_t *>(p.q),
+                                    reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
+                                    reinterpret_cast<float *>(base + OFF_KH), tid);
     // ---- P3: M rows (lanes 0-63) -> TBM rows 128..191; beta * A rows (lanes 64-127) -> As
     prep::extract_gram(tm + my_cols + TM_G, base + OFF_TBM, 192, 128, As, beta_sh, tid);
     __syncthreads();
@@ -248,7 +256,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     // the staging buffers are free: stream the next chunk's q, k, log_alpha, beta
     if (c0 + kC < sp.end) stage_chunk(p, maps, sp, c0 + kC, h, base, &stage_bar, tid);
     // V of this chunk must have landed; zero its invalid rows
-    ok = __syncthreads_and(mbar_wait(&v_bar, chunk_idx & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&v_bar, chunk_idx & 1, p.wait_cycles));
     if (!ok) break;
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
       for (int e = tid; e < kC * 8; e += kThreads) {
@@ -270,7 +278,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_D1, desc_kmajor(sTBM, 192, 0, s), desc_mnmajor(sV, 64, 0, s), idu, s > 0);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -303,7 +311,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_D1, desc_kmajor(sQKW, 192, 0, s), desc_mnmajor(sSB, 128, 0, s), id, 1);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -327,7 +335,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_S, desc_mnmajor(sKT, 64, 0, s), desc_mnmajor(sUB, 64, 0, s), ids, 1);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, kWaitCycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -358,7 +366,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
     // let the product that timed out finish (bounded) before TMEM is released
-    mbar_wait(&mma_bar, (phase - 1) & 1, kWaitCycles);
+    mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
   } else if (p.final_state) {
     float v[32];
     tmem_ld32(tm + my_cols + TM_S, v);

@@ -33,7 +33,8 @@ KDA_GATE_HEAD = 1
 
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_short_conv",
-            "kda_prefill_backward", "kda_prefill_backward_workspace_size")
+            "kda_prefill_backward", "kda_prefill_backward_workspace_size", "kda_debug_set_fault")
+KDA_FAULT_STARVE_STATE_LOADS = 1
 
 
 class KdaError(RuntimeError):
@@ -121,6 +122,8 @@ def load(build_if_stale: bool = True) -> ctypes.CDLL:
             lib.kda_version.restype = ctypes.c_int
             lib.kda_prefill_noalloc.argtypes = [ctypes.POINTER(PrefillArgs), ctypes.c_void_p]
             lib.kda_prefill_noalloc.restype = ctypes.c_int
+            lib.kda_debug_set_fault.argtypes = [ctypes.c_int, ctypes.c_longlong]
+            lib.kda_debug_set_fault.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -190,6 +193,12 @@ def prefill_workspace_bytes(num_seqs: int) -> int:
     a = PrefillArgs()
     a.num_seqs = int(num_seqs)
     return int(load().kda_prefill_workspace_size(ctypes.byref(a)))
+
+
+def prefill_workspace_size_for(q, k, v, log_alpha, beta, cu_seqlens, chunk: int = 0) -> int:
+    """kda_prefill_workspace_size() for these tensors (at least 1 byte)."""
+    a = prefill_args(q, k, v, log_alpha, beta, cu_seqlens, chunk=chunk)
+    return max(int(load().kda_prefill_workspace_size(ctypes.byref(a))), 1)
 
 
 def prefill_workspace(q, k, v, log_alpha, beta, cu_seqlens, chunk: int = 0) -> torch.Tensor:
@@ -361,6 +370,14 @@ def prefill_backward(q, k, v, log_alpha, beta, cu_seqlens, grad_o, grad_final_st
 def get_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the latched device status."""
     return int(load().kda_get_device_status(_stream_handle(stream)))
+
+
+def debug_set_fault(fault: int, wait_cycles: int = 0) -> None:
+    """kda_debug_set_fault: plant a test fault and set the bounded-wait limit (tests only;
+    ``debug_set_fault(0)`` restores normal operation and the default limit)."""
+    st = load().kda_debug_set_fault(int(fault), int(wait_cycles))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_debug_set_fault")
 
 
 def raw_prefill(args: PrefillArgs, stream=None) -> int:

@@ -35,7 +35,9 @@
  *   - No C++ exception crosses the ABI.
  *   - Every launch is stream-ordered, so the calls can be captured into a CUDA
  *     graph; the first call on each device looks up the library's device error
- *     word (cudaGetSymbolAddress), so make one call before capturing.
+ *     word (cudaGetSymbolAddress), so make one call before capturing.  The
+ *     library keeps those device addresses for the life of the process: after
+ *     a cudaDeviceReset(), unload and reload the library before calling it.
  *   - Layouts are row-major and contiguous.  N = total packed tokens,
  *     B = sequences (prefill) or rows (decode), H = heads.
  */
@@ -154,8 +156,15 @@ kda_status kda_prefill(const kda_prefill_args *args, void *stream);
  * operator (an engine whose device memory is owned up front by a host
  * framework that passes operators only their tensors, or a serving loop in
  * which cudaMalloc/cudaFree are not allowed because they may synchronise the
- * device).  Same arguments and results as kda_prefill; args->workspace and
- * args->workspace_bytes are ignored.  The scratch comes from a fixed device
+ * device).  Same arguments as kda_prefill; args->workspace and
+ * args->workspace_bytes are ignored.  Its 64 KiB of scratch holds the span
+ * table of the pad pre-pass but not the per-chunk items of the two-kernel
+ * tensor-core path, so it runs the single-kernel tensor-core path (bf16,
+ * d_k = 128, d_v a multiple of 64, chunk 64, per-channel gate) or the
+ * CUDA-core path (everything else): its results equal kda_prefill's up to
+ * rounding (within the same tolerances against the exact recurrence), not bit
+ * for bit, and it is slower than kda_prefill with a full workspace.  The
+ * scratch comes from a fixed device
  * array inside the library, sized for KDA_NOALLOC_MAX_SEQS sequences (64 KiB,
  * held by every GPU that loads the library until exit); a batch with more
  * sequences returns KDA_ERR_INVALID_ARG and launches nothing.  All calls on a
@@ -297,6 +306,25 @@ kda_status kda_prefill_backward(const kda_backward_args *args, void *stream);
 /* Synchronise `stream`, then return and clear the error latched on the
  * current device by earlier kernels (KDA_OK if none). */
 kda_status kda_get_device_status(void *stream);
+
+/*
+ * Test hook for failure detection without a GPU fault (the pages have no
+ * counterpart).  Every device-side wait of the prefill kernels is bounded;
+ * when one runs out the kernel drains what it has in flight, releases its
+ * tensor memory, latches KDA_ERR_DEVICE_TIMEOUT and returns, so the context
+ * stays usable.  This hook lets a test make that happen on purpose:
+ *   fault        0 (normal operation) or KDA_FAULT_STARVE_STATE_LOADS: the
+ *                state pass of the workspace-backed tensor-core prefill issues
+ *                none of its item loads, so its waits run out; nothing is read
+ *                or written out of bounds and the call's outputs are left
+ *                unspecified.
+ *   wait_cycles  the limit, in SM clock cycles, of every bounded wait in later
+ *                prefill calls; <= 0 restores the default (about 2 s).
+ * Process-wide and read at each kda_prefill call; meant for tests only.
+ * Returns KDA_ERR_INVALID_ARG for an unknown fault bit.
+ */
+#define KDA_FAULT_STARVE_STATE_LOADS 1
+kda_status kda_debug_set_fault(int fault, long long wait_cycles);
 
 /* Static string for a status code; never NULL. */
 const char *kda_status_string(kda_status status);

@@ -205,3 +205,9 @@ def test_conv_rejects_bad_arguments(mutate, expect):
     a = _good_conv()
     mutate(a)
     assert kda.load().kda_short_conv(ctypes.byref(a), None) == expect
+
+
+def test_debug_fault_hook_rejects_unknown_bits_and_resets():
+    lib = kda.load()
+    assert lib.kda_debug_set_fault(1 << 7, 0) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_debug_set_fault(0, 0) == kda.KDA_OK

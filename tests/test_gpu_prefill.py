@@ -260,18 +260,149 @@ def test_long_prefill_128k_sampled_heads():
     assert torch.isfinite(o.float()).all()
 
 
-@pytest.mark.parametrize("per_token", [-0.5, -1.1])
-def test_strong_decay_within_tensor_core_range(per_token):
-    """The tensor-core path forms e^{-g} inside a 64-token chunk; with a per-token
-    log-decay of -0.5 (-32 per chunk) or -1.1 (-70 per chunk) on a quarter of the
-    channels it must still match the oracle (the path's stated range is a chunk
-    log-decay above about -80)."""
-    inp = gen.random_case(61, [700, 64], 2, 128, 128, "bf16", init_state=True)
+def _run_path(inp, dtype, path, chunk=0):
+    """Run one prefill path on the GPU: "split" (the full workspace: the two-kernel
+    tensor-core path for bf16, d = 128, chunk 64), "fused" (a span-table workspace only:
+    the single-kernel tensor-core path), "noalloc" (kda_prefill_noalloc) or "simt"
+    (fp32 inputs: the CUDA-core path)."""
+    d = dev_inputs(inp, dtype)
+    N, H = d["q"].shape[0], d["q"].shape[1]
+    B = d["cu_seqlens"].numel() - 1
+    dv = d["v"].shape[2]
+    dk = d["q"].shape[2]
+    o = torch.full((N, H, dv), 9.0, dtype=d["q"].dtype, device="cuda")
+    fs = torch.full((B, H, dk, dv), 9.0, dtype=torch.float32, device="cuda")
+    args = (d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"])
+    if path == "noalloc":
+        kda.prefill_noalloc(*args, o, final_state=fs, pad_mask=d.get("pad_mask"),
+                            init_state=d.get("init_state"), chunk=chunk)
+    else:
+        ws = None
+        if path == "fused":
+            ws = torch.empty(max(kda.prefill_workspace_bytes(B), 1), dtype=torch.uint8, device="cuda")
+        kda.prefill(*args, pad_mask=d.get("pad_mask"), init_state=d.get("init_state"), o=o,
+                    final_state=fs, chunk=chunk, workspace=ws)
+    torch.cuda.synchronize()
+    assert kda.get_device_status() == kda.KDA_OK
+    return o, fs
+
+
+_DECAYS = ["per_token_-0.5", "per_token_-1.1", "quarter_channels_-4", "spikes_-200"]
+
+
+def _strong_decay(inp, pattern):
     la = inp["log_alpha"].copy()
-    la[:, :, ::4] = per_token
+    if pattern.startswith("per_token"):
+        la[:, :, ::4] = float(pattern.split("_")[-1])
+    elif pattern == "quarter_channels_-4":
+        la[:, :, ::4] = -4.0          # -256 over a 64-token chunk
+    else:                               # one -200 step mid-chunk: all channels, then half of them
+        la[[30, 100, 357], :, :] = -200.0
+        la[[500, 731], :, ::2] = -200.0
     inp["log_alpha"] = la
-    o, fs = _gpu(inp, "bf16")
+    return inp
+
+
+@pytest.mark.parametrize("path", ["split", "fused"])
+@pytest.mark.parametrize("pattern", _DECAYS)
+def test_strong_decay_tensor_core_paths(path, pattern):
+    """Every finite log_alpha <= 0 is in range: a quarter of the channels at -0.5 or -1.1 per
+    token (inside the factorised range), at -4 per token (-256 per chunk), and single -200
+    steps mid-chunk on all or half of the channels.  Both tensor-core paths match the oracle
+    within the bf16 tolerance (channels beyond the factorised range take the exact Gram)."""
+    inp = _strong_decay(gen.random_case(61, [700, 64, 130], 2, 128, 128, "bf16", init_state=True),
+                        pattern)
+    o, fs = _run_path(inp, "bf16", path)
     _check(inp, "bf16", o, fs)
+
+
+@pytest.mark.parametrize("pattern", ["quarter_channels_-4", "spikes_-200"])
+def test_strong_decay_cuda_core_path(pattern):
+    inp = _strong_decay(gen.random_case(62, [700, 64, 130], 2, 128, 64, "f32", init_state=True),
+                        pattern)
+    o, fs = _run_path(inp, "f32", "simt", chunk=64)
+    _check(inp, "f32", o, fs)
+
+
+def _pad_case(seed, lengths, H, dtype, dv=128, interior=True, edges=True, garbage=True):
+    """Edge and interior pads whose q, k, v, log_alpha and beta are random, large or not
+    finite: none of it may reach the outputs or the state."""
+    inp = gen.random_case(seed, lengths, H, 128, dv, dtype, init_state=True)
+    cu = inp["cu_seqlens"]
+    N = int(cu[-1])
+    rng = np.random.default_rng(seed)
+    mask = np.ones(N, np.uint8)
+    for b in range(len(lengths)):
+        a, e = int(cu[b]), int(cu[b + 1])
+        if e - a < 8:
+            continue
+        if edges:
+            mask[a:a + int(rng.integers(0, 5))] = 0
+            mask[e - int(rng.integers(0, 5)):e] = 0
+        if interior:
+            inner = rng.choice(np.arange(a + 4, e - 4), size=min(9, e - a - 8), replace=False)
+            mask[inner] = 0
+    pads = np.nonzero(mask == 0)[0]
+    if garbage and pads.size:
+        big = lambda shape: gen.round_bf16((rng.normal(size=shape) * 1000.0).astype(np.float32))
+        for key in ("q", "k", "v"):
+            inp[key][pads] = big(inp[key][pads].shape)
+        inp["log_alpha"][pads] = -np.abs(rng.normal(size=inp["log_alpha"][pads].shape) * 50.0)
+        inp["beta"][pads] = (rng.normal(size=inp["beta"][pads].shape) * 10.0).astype(np.float32)
+        inp["q"][pads[0]] = np.nan
+        inp["v"][pads[-1]] = np.inf
+        inp["k"][pads[len(pads) // 2]] = -np.inf
+        inp["beta"][pads[0]] = np.nan
+    inp["pad_mask"] = mask
+    return inp
+
+
+@pytest.mark.parametrize("path,dtype", [("split", "bf16"), ("fused", "bf16"), ("noalloc", "bf16"),
+                                        ("simt", "f32")])
+def test_pads_with_garbage_values_every_path(path, dtype):
+    """Edge and interior pads carrying huge, random and non-finite q, k, v, log_alpha and
+    beta: pad outputs are exactly 0, everything else matches the oracle run without the
+    pads (which never reads the pad values)."""
+    inp = _pad_case(63, [300, 17, 129, 700], 2, dtype)
+    o, fs = _run_path(inp, dtype, path)
+    keep = inp["pad_mask"] == 1
+    assert torch.all(o[torch.from_numpy(~keep).cuda()] == 0)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(fs).all()
+    _check(inp, dtype, o, fs)
+
+
+@pytest.mark.parametrize("path", ["fused", "noalloc"])
+def test_single_kernel_paths_match_oracle_with_pads(path):
+    """The single-kernel tensor-core path (a span-table workspace, or the allocation-free
+    entry point) with edge and interior pads and nonzero initial states, d_v = 128 and 64,
+    against the oracle."""
+    for dv in (128, 64):
+        inp = _pad_case(64, [64, 1, 500, 90, 33, 250], 3, "bf16", dv=dv, garbage=False)
+        o, fs = _run_path(inp, "bf16", path)
+        assert torch.all(o[torch.from_numpy(inp["pad_mask"] == 0).cuda()] == 0)
+        _check(inp, "bf16", o, fs)
+
+
+@pytest.mark.parametrize("T", [64 * 3 + 1, 64 * 4 + 30])
+def test_prefix_invariance_single_kernel_path(T):
+    """The bit-identical prefix audit on the single-kernel tensor-core path."""
+    inp = gen.random_case(38, [T], 4, 128, 128, "bf16", init_state=True)
+    rng = np.random.default_rng(40)
+
+    def run(which):
+        x = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+        if which:
+            x["q"][T - 1] = gen.round_bf16(rng.normal(size=x["q"][T - 1].shape).astype(np.float32))
+            x["k"][T - 1] = gen.round_bf16(rng.normal(size=x["k"][T - 1].shape).astype(np.float32))
+            x["v"][T - 1] = gen.round_bf16(rng.normal(size=x["v"][T - 1].shape).astype(np.float32))
+            x["log_alpha"][T - 1] = -np.abs(rng.normal(size=x["log_alpha"][T - 1].shape)) * 90.0
+            x["beta"][T - 1] = 0.77
+        o, _ = _run_path(x, "bf16", "fused")
+        return to_np(o)
+
+    leak, onset, d = orc.prefix_audit(run, T, 1)
+    assert not leak, f"prefix leak, onset {onset}"
+    assert d.max() == 0.0
 
 
 def test_many_short_sequences_two_kernel_path():
@@ -306,3 +437,23 @@ def test_state_slice_width_does_not_change_results():
     assert torch.equal(o2[:lengths[0]], o1)
     assert torch.equal(fs2[:1], fs1)
     _check(solo, "bf16", o1, fs1)
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """Failure detection without a GPU fault: with a planted fault the state pass issues no
+    item loads, so its bounded waits (set to ~1 ms here) run out.  The call returns, the
+    device status reads KDA_ERR_DEVICE_TIMEOUT, and the next normal call on the same context
+    matches the oracle (the kernel left nothing in flight and released its tensor memory)."""
+    inp = gen.random_case(91, [700, 130], 2, 128, 128, "bf16", init_state=True)
+    d = dev_inputs(inp, "bf16")
+    kda.debug_set_fault(kda.KDA_FAULT_STARVE_STATE_LOADS, 2_000_000)
+    try:
+        kda.prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                    init_state=d["init_state"])
+        st = kda.get_device_status()
+    finally:
+        kda.debug_set_fault(0)
+    assert st == kda.KDA_ERR_DEVICE_TIMEOUT, kda.status_string(st)
+    assert kda.get_device_status() == kda.KDA_OK       # the latch was cleared
+    o, fs = _gpu(inp, "bf16")
+    _check(inp, "bf16", o, fs)

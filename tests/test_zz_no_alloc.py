@@ -1,11 +1,13 @@
-"""kda_prefill_noalloc against kda_prefill (GPU, through the C ABI).
+"""kda_prefill_noalloc against kda_prefill and the fp64 oracle (GPU, through the C ABI).
 
 The allocation-free entry point exists for callers that cannot call
 cudaMalloc where they run the operator (memory owned up front by a host
 framework, or loops where an allocation could synchronise the device).  It
-must give the same results as the workspace entry point, call after call,
-although every call reuses the same fixed scratch array inside the library.
-This file is collected last on purpose.
+must give the same results as the workspace entry point up to rounding (it
+takes the single-kernel tensor-core path or the CUDA-core path, never the
+two-kernel path that needs the large workspace), call after call, although
+every call reuses the same fixed scratch array inside the library; and both
+must match the oracle.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -16,12 +18,15 @@ import torch
 from gated_delta_rule_148_b200 import inputs as gen
 from gated_delta_rule_148_b200 import kda
 from kda_testlib import TOL, dev_inputs, norm_err, to_np
+from oracle import kda_oracle as orc
 
 pytestmark = pytest.mark.gpu
 
 
-def _padded_case(seed, lengths):
-    inp = gen.random_case(seed, lengths, 4, 128, 128, "bf16", init_state=True)
+def _padded_case(seed, lengths, dtype="bf16", pads=True):
+    inp = gen.random_case(seed, lengths, 4, 128, 128, dtype, init_state=True)
+    if not pads:
+        return inp
     cu = inp["cu_seqlens"]
     mask = np.ones(int(cu[-1]), np.uint8)
     rng = np.random.default_rng(seed)
@@ -39,10 +44,10 @@ def _padded_case(seed, lengths):
 
 
 def _call(entry, d, N, B, workspace=None):
-    o = torch.full((N, 4, 128), 5.0, dtype=torch.bfloat16, device="cuda")
+    o = torch.full((N, 4, 128), 5.0, dtype=d["q"].dtype, device="cuda")
     fs = torch.full((B, 4, 128, 128), 5.0, dtype=torch.float32, device="cuda")
     a = kda.prefill_args(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
-                         d["pad_mask"], d["init_state"], o, fs, 0, workspace)
+                         d.get("pad_mask"), d["init_state"], o, fs, 0, workspace)
     st = getattr(kda.load(), entry)(ctypes.byref(a), ctypes.c_void_p(
         torch.cuda.current_stream().cuda_stream))
     assert st == kda.KDA_OK, kda.status_string(st)
@@ -50,19 +55,36 @@ def _call(entry, d, N, B, workspace=None):
     return o, fs
 
 
-def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
+def _oracle_check(inp, dtype, o, fs):
+    o_ref, s_ref = orc.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                               inp["cu_seqlens"], pad_mask=inp.get("pad_mask"),
+                               init_state=inp["init_state"])
+    assert norm_err(to_np(o), o_ref) <= TOL[dtype]
+    assert norm_err(to_np(fs), s_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,pads", [("bf16", True), ("bf16", False), ("f32", True)])
+def test_noalloc_matches_workspace_entry_two_calls_in_a_row(dtype, pads):
+    """Two different batches one after the other through the allocation-free entry point
+    (the second reuses the scratch the first left behind): each equals kda_prefill with a
+    workspace up to rounding and matches the oracle; pad outputs are exactly 0."""
     cases = [(70, [300, 17, 129]), (71, [64, 1, 500, 90, 33, 250])]
     for seed, lengths in cases:
-        inp = _padded_case(seed, lengths)
-        d = dev_inputs(inp, "bf16")
+        inp = _padded_case(seed, lengths, dtype, pads)
+        d = dev_inputs(inp, dtype)
         N, B = int(inp["cu_seqlens"][-1]), len(lengths)
-        ws = torch.empty(kda.prefill_workspace_bytes(B), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(kda.prefill_workspace_size_for(d["q"], d["k"], d["v"], d["log_alpha"],
+                                                        d["beta"], d["cu_seqlens"]),
+                         dtype=torch.uint8, device="cuda")
         o_ref, fs_ref = _call("kda_prefill", d, N, B, ws)
         o, fs = _call("kda_prefill_noalloc", d, N, B)
-        assert norm_err(to_np(o), to_np(o_ref)) <= TOL["bf16"]
-        assert norm_err(to_np(fs), to_np(fs_ref)) <= TOL["bf16"]
-        keep = torch.from_numpy(inp["pad_mask"] == 0).cuda()
-        assert torch.all(o[keep] == 0)
+        assert norm_err(to_np(o), to_np(o_ref)) <= TOL[dtype]
+        assert norm_err(to_np(fs), to_np(fs_ref)) <= TOL[dtype]
+        _oracle_check(inp, dtype, o, fs)
+        _oracle_check(inp, dtype, o_ref, fs_ref)
+        if pads:
+            keep = torch.from_numpy(inp["pad_mask"] == 0).cuda()
+            assert torch.all(o[keep] == 0)
 
 
 def test_noalloc_rejects_more_sequences_than_its_scratch_holds():
