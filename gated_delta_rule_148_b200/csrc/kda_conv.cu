@@ -13,10 +13,12 @@
 //
 // Layout: x, y [N, D] (bf16 or fp32), weight [D, W] fp32, bias [D] fp32,
 // conv_state [B, W-1, D] fp32.  The operation is HBM-bound (read x, write y):
-// kernel A gives each CTA 256 packed positions and up to 2048 channels; the pad
+// kernel A gives each CTA 128 packed positions and up to 1024 channels; the pad
 // mask of those positions is compacted once per CTA (warp ballots) into the list
-// of valid rows, and each thread walks those rows for its 8 consecutive channels
-// with the window in registers (one 16-byte load and one store per row).  Kernel B writes the new
+// of valid rows, and each thread walks those rows for its 4 consecutive channels
+// with the window in registers and the next 8 rows' loads already in flight (a
+// ring of raw 8- or 16-byte loads), so a thread keeps about 8 loads outstanding
+// at a register count that lets several CTAs share an SM.  Kernel B writes the new
 // state after kernel A, one thread per (sequence, channel), so conv_state may be
 // updated in place.
 #include "kda_internal.cuh"
@@ -24,10 +26,13 @@
 namespace kda {
 namespace conv {
 
-constexpr int kSeg = 256;            // packed positions per CTA
+constexpr int kSeg = 128;            // packed positions per CTA
 constexpr int kThreads = 256;
-constexpr int kChan = 8 * kThreads;  // channels per CTA (8 per thread)
+constexpr int kPer = 4;              // channels per thread
+constexpr int kChan = kPer * kThreads;  // channels per CTA
+constexpr int kRing = 8;             // rows whose loads are in flight ahead of the walk
 constexpr int kMaxW = 4;
+static_assert(kSeg <= kThreads, "one compaction ballot per position");
 
 // Source of a window entry: a packed position (>= 0) or state row j (encoded -1 - j).
 struct Hist {
@@ -54,47 +59,50 @@ __device__ __forceinline__ Hist history_before(const uint8_t *mask, int sb, int 
   return hs;
 }
 
+// Raw loads of 4 consecutive channels of one row (8 bytes bf16, 16 bytes fp32),
+// unpacked separately so that several rows' loads can be in flight.
+template <bool BF16> struct Raw4;
+template <> struct Raw4<true> { using T = uint2; };
+template <> struct Raw4<false> { using T = float4; };
+
 template <bool BF16>
-__device__ __forceinline__ void load8(const void *x, size_t row, int D, int c, float *v) {
-  if (BF16) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(x) + row * D + c));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[2 * e] = __uint_as_float(w[e] << 16);
-      v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-    }
-  } else {
-    const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + row * D + c);
-    const float4 a = __ldg(p), b = __ldg(p + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
+__device__ __forceinline__ typename Raw4<BF16>::T load4(const void *x, size_t row, int D, int c) {
+  if constexpr (BF16)
+    return __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(x) + row * D + c));
+  else
+    return __ldg(reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + row * D + c));
+}
+
+__device__ __forceinline__ void unpack4(uint2 u, float *v) {
+  v[0] = __uint_as_float(u.x << 16);
+  v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(u.y << 16);
+  v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void unpack4(float4 u, float *v) {
+  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
 }
 
 template <bool BF16>
-__device__ __forceinline__ void store8(void *y, size_t row, int D, int c, const float *v) {
-  if (BF16) {
-    uint4 u;
+__device__ __forceinline__ void store4(void *y, size_t row, int D, int c, const float *v) {
+  if constexpr (BF16) {
+    uint2 u;
     u.x = (uint32_t)f32_to_bf16_rne(v[0]) | ((uint32_t)f32_to_bf16_rne(v[1]) << 16);
     u.y = (uint32_t)f32_to_bf16_rne(v[2]) | ((uint32_t)f32_to_bf16_rne(v[3]) << 16);
-    u.z = (uint32_t)f32_to_bf16_rne(v[4]) | ((uint32_t)f32_to_bf16_rne(v[5]) << 16);
-    u.w = (uint32_t)f32_to_bf16_rne(v[6]) | ((uint32_t)f32_to_bf16_rne(v[7]) << 16);
-    *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(y) + row * D + c) = u;
+    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(y) + row * D + c) = u;
   } else {
-    float4 *p = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + row * D + c);
-    p[0] = make_float4(v[0], v[1], v[2], v[3]);
-    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + row * D + c) = make_float4(v[0], v[1], v[2], v[3]);
   }
 }
 
-
 // Kernel A: outputs of packed positions [kSeg*blockIdx.x, +kSeg), channels
-// [kChan*blockIdx.y, +kChan).  Thread t owns channels 8t .. 8t+7 and walks the
+// [kChan*blockIdx.y, +kChan).  Thread t owns channels 4t .. 4t+3 and walks the
 // CTA's valid rows in order with the window in registers, so each x row is read
-// once; the 16-byte loads of one row are coalesced across the CTA's threads.
+// once; the loads of one row are coalesced across the CTA's threads, and the
+// ring keeps the loads of the next kRing rows in flight.
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
+__global__ void __launch_bounds__(kThreads, BF16 ? 4 : 2) conv_kernel(ConvParams p) {
+  using Raw = typename Raw4<BF16>::T;
   __shared__ int vpos[kSeg];
   __shared__ int wcnt[kThreads / 32];
   __shared__ Hist hist_sh;
@@ -110,15 +118,16 @@ __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
     if (bad) atomicOr(p.err, ERR_BIT_CHECK);
   }
   // this thread's channels and their taps
-  const int cl = tid * 8, c = c_lo + cl;
+  const int cl = tid * kPer, c = c_lo + cl;
   const bool mine = cl < nch;
-  float wt[kMaxW - 1][8], wx[8], bz[8];      // window taps, the current row's tap, bias
+  float wt[kMaxW - 1][kPer], wx[kPer], bz[kPer];      // window taps, the current row's tap, bias
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < kPer; ++j) {
     bz[j] = (mine && p.bias) ? p.bias[c + j] : 0.f;
     wx[j] = mine ? p.weight[(size_t)(c + j) * W + (W - 1)] : 0.f;
 #pragma unroll
-    for (int i = 0; i < kMaxW - 1; ++i) wt[i][j] = (mine && i < W - 1) ? p.weight[(size_t)(c + j) * W + i] : 0.f;
+    for (int i = 0; i < kMaxW - 1; ++i)
+      wt[i][j] = (mine && i < W - 1) ? p.weight[(size_t)(c + j) * W + i] : 0.f;
   }
   // first sequence with cu[b + 1] > s0
   int lo = 0, hi = B - 1;
@@ -147,50 +156,59 @@ __global__ void __launch_bounds__(kThreads) conv_kernel(ConvParams p) {
     __syncthreads();
     if (mine) {
       // ---- the window before the first valid row (oldest first)
-      float win[kMaxW - 1][8];
+      float win[kMaxW - 1][kPer];
 #pragma unroll
       for (int j = 0; j < kMaxW - 1; ++j) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) win[j][q] = 0.f;
+        for (int q = 0; q < kPer; ++q) win[j][q] = 0.f;
         if (j < W - 1) {
           const int src = hist_sh.src[j];
-          if (src >= 0) load8<BF16>(p.x, (size_t)src, D, c, win[j]);
-          else if (p.state_in) load8<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c, win[j]);
+          if (src >= 0) unpack4(load4<BF16>(p.x, (size_t)src, D, c), win[j]);
+          else if (p.state_in) unpack4(load4<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c), win[j]);
         }
       }
-      // ---- walk the valid rows
-#pragma unroll 2
-      for (int m = 0; m < nvalid; ++m) {
-        const size_t row = (size_t)vpos[m];
-        float xv[8], acc[8];
-        load8<BF16>(p.x, row, D, c, xv);
+      // ---- walk the valid rows; ring[u] holds the raw load of row m0 + u
+      Raw ring[kRing];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = fmaf(wx[q], xv[q], bz[q]);
-        // taps: u_i = win[i] for i < W-1 (zero taps beyond), u_{W-1} = x_t
+      for (int u = 0; u < kRing; ++u)
+        if (u < nvalid) ring[u] = load4<BF16>(p.x, (size_t)vpos[u], D, c);
+      for (int m0 = 0; m0 < nvalid; m0 += kRing) {
 #pragma unroll
-        for (int i = 0; i < kMaxW - 1; ++i)
+        for (int u = 0; u < kRing; ++u) {
+          const int m = m0 + u;
+          if (m < nvalid) {
+            float xv[kPer], acc[kPer];
+            unpack4(ring[u], xv);
+            if (m + kRing < nvalid) ring[u] = load4<BF16>(p.x, (size_t)vpos[m + kRing], D, c);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) acc[q] = fmaf(wt[i][q], win[i][q], acc[q]);
-        store8<BF16>(p.y, row, D, c, acc);
-        // shift: the newest of the W-1 slots becomes x_t
+            for (int q = 0; q < kPer; ++q) acc[q] = fmaf(wx[q], xv[q], bz[q]);
+            // taps: u_i = win[i] for i < W-1 (zero taps beyond), u_{W-1} = x_t
 #pragma unroll
-        for (int j = 0; j < kMaxW - 2; ++j)
-          if (j + 1 < W - 1) {
+            for (int i = 0; i < kMaxW - 1; ++i)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) win[j][q] = win[j + 1][q];
+              for (int q = 0; q < kPer; ++q) acc[q] = fmaf(wt[i][q], win[i][q], acc[q]);
+            store4<BF16>(p.y, (size_t)vpos[m], D, c, acc);
+            // shift: the newest of the W-1 slots becomes x_t
+#pragma unroll
+            for (int j = 0; j < kMaxW - 2; ++j)
+              if (j + 1 < W - 1) {
+#pragma unroll
+                for (int q = 0; q < kPer; ++q) win[j][q] = win[j + 1][q];
+              }
+#pragma unroll
+            for (int j = 0; j < kMaxW - 1; ++j)
+              if (j == W - 2) {
+#pragma unroll
+                for (int q = 0; q < kPer; ++q) win[j][q] = xv[q];
+              }
           }
-#pragma unroll
-        for (int j = 0; j < kMaxW - 1; ++j)
-          if (j == W - 2) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) win[j][q] = xv[q];
-          }
+        }
       }
       // ---- pads: y = 0
       if (p.mask != nullptr && nvalid < e - a) {
-        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float z[kPer] = {0.f, 0.f, 0.f, 0.f};
         for (int r = a; r < e; ++r)
-          if (p.mask[r] == 0) store8<BF16>(p.y, (size_t)r, D, c, z);
+          if (p.mask[r] == 0) store4<BF16>(p.y, (size_t)r, D, c, z);
       }
     }
     __syncthreads();   // vpos, wcnt and hist_sh are rewritten by the next sequence
