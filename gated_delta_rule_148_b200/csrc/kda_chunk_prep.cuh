@@ -196,7 +196,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
   if (qt == 0) {
     decay[c] = GC0;
     decay[c + 1] = GC1;
-    *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
+    if (gdecay) *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
   }
   const float2 inv = gram_inv_decay(GC0, GC1, c, unsafe);
   const float inv0 = inv.x, inv1 = inv.y;

@@ -109,7 +109,7 @@ typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1 } kda_gate;
  *   workspace    device scratch, 256-byte aligned.  kda_prefill_workspace_size()
  *                bytes select the fastest path (for bf16, d_k = d_v = 128,
  *                chunk 64: a two-kernel path that stores each chunk's
- *                intermediate tiles, about 73 KB per 64 tokens and head).  A
+ *                intermediate tiles, 88 KB per 64 tokens and head).  A
  *                smaller workspace selects a fused single-kernel path; a pad
  *                mask needs at least 16 bytes per sequence (rounded up to 256).
  *                May be NULL when pad_mask is NULL.
