@@ -11,6 +11,8 @@ namespace kda {
 
 // Per-device error word (bits of ERR_BIT_*); kernels OR into it.
 __device__ unsigned g_error_word;
+// Per-device code of the first bounded wait that ran out (0: none since the last read).
+__device__ unsigned g_timeout_site;
 
 namespace {
 
@@ -28,6 +30,22 @@ kda_status error_word(unsigned **out) {
     if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess || ptr == nullptr) return KDA_ERR_CUDA;
     cached = static_cast<unsigned *>(ptr);
     g_err_ptr[dev].store(cached, std::memory_order_release);
+  }
+  *out = cached;
+  return KDA_OK;
+}
+
+std::atomic<unsigned *> g_site_ptr[kMaxDevices];
+
+kda_status timeout_site_word(unsigned **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+  unsigned *cached = g_site_ptr[dev].load(std::memory_order_acquire);
+  if (cached == nullptr) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_timeout_site) != cudaSuccess || ptr == nullptr) return KDA_ERR_CUDA;
+    cached = static_cast<unsigned *>(ptr);
+    g_site_ptr[dev].store(cached, std::memory_order_release);
   }
   *out = cached;
   return KDA_OK;
@@ -142,8 +160,8 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
       overlap(ws, cu) || overlap(ws, mk) || overlap(ws, s0))
     return KDA_ERR_INVALID_ARG;
 
-  unsigned *err = nullptr;
-  if (error_word(&err) != KDA_OK) return KDA_ERR_CUDA;
+  unsigned *err = nullptr, *site = nullptr;
+  if (error_word(&err) != KDA_OK || timeout_site_word(&site) != KDA_OK) return KDA_ERR_CUDA;
   PrefillParams p;
   p.num_seqs = a->num_seqs;
   p.N = a->total_tokens;
@@ -165,6 +183,7 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   p.gate_head = gate_head ? 1 : 0;
   p.wait_cycles = g_wait_cycles.load(std::memory_order_relaxed);
   p.fault = g_fault.load(std::memory_order_relaxed);
+  p.site = site;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = a->dtype == KDA_BF16;
   p.spans = nullptr;
@@ -352,6 +371,17 @@ kda_status kda_debug_set_fault(int fault, long long wait_cycles) {
   g_fault.store(fault, std::memory_order_relaxed);
   g_wait_cycles.store(wait_cycles > 0 ? wait_cycles : kDefaultWaitCycles, std::memory_order_relaxed);
   return KDA_OK;
+}
+
+int kda_debug_timeout_site(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return -1;
+  unsigned *site = nullptr;
+  if (timeout_site_word(&site) != KDA_OK) return -1;
+  unsigned code = 0;
+  if (cudaMemcpy(&code, site, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  const unsigned zero = 0;
+  if (code != 0 && cudaMemcpy(site, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return -1;
+  return (int)code;
 }
 
 kda_status kda_get_device_status(void *stream) {

@@ -10,13 +10,16 @@
 //   Q G = q e^{g},  K G = k e^{g},  K e^{-g},  K e^{g_C - g}  (bf16 operand tiles)
 //
 // Range of the factorised Gram.  The Gram products take e^{g_r - g_i} as
-// e^{g_r} * e^{-g_i}; e^{-g_i} <= e^{-g_C} stays representable (and far from
-// overflow in the products) while a channel's log-decay over the chunk is above
-// ln(kFastMinDecay) ~ -60.  A channel below that ("unsafe") gets a zero column
-// in K e^{-g}, so the tensor-core Gram holds the other channels' terms only,
-// and exact_gram_fixup() adds its terms with running products of alpha on the
-// CUDA cores (every factor <= 1, exact for any log_alpha <= 0).  The other
-// tiles only use factors <= 1 and need no special case.
+// e^{g_r} * e^{-g_i}.  The factor e^{-g_i} of key row i and channel c is used
+// only while e^{g_i} > kFastMinDecay (log-decay from the chunk start above about
+// -60), where it is far from overflow; from the first row where it is not (the
+// channel's threshold row t_c), the channel's K e^{-g} entries are 0 and
+// exact_gram_fixup() adds those key rows' terms with running products of alpha
+// on the CUDA cores (every factor <= 1, exact for any log_alpha <= 0).  Whether a
+// key row takes the exact path depends on rows up to it only, so an output row
+// never depends on a later row's values (prefix invariance, bit for bit).  A
+// factor e^{g_r} that underflows multiplies terms below e^{-27} of the largest.
+// The other tiles only use factors <= 1 and need no special case.
 #pragma once
 
 #include "kda_internal.cuh"
@@ -29,15 +32,31 @@ using namespace tc;
 
 constexpr int kC = 64;
 constexpr int kDK = 128;
-constexpr float kFastMinDecay = 1e-26f;   // e^{g_C} below this: the channel takes the exact path
+constexpr float kFastMinDecay = 1e-26f;   // e^{g_r} at or below this: exact path from row r on
 
-// Marks channels c, c + 1 whose chunk decay e^{g_C} is below kFastMinDecay in the
-// 4-word mask `unsafe` (zeroed by the caller before the prep) and returns the
-// factors e^{-g_C} the tiles use (0 for an unsafe channel: its K e^{-g} column is 0).
-__device__ __forceinline__ float2 gram_inv_decay(float GC0, float GC1, int c, uint32_t *unsafe) {
-  const bool u0 = !(GC0 > kFastMinDecay), u1 = !(GC1 > kFastMinDecay);
-  if (u0 | u1) atomicOr(&unsafe[c >> 5], ((u0 ? 1u : 0u) | (u1 ? 2u : 0u)) << (c & 31));
-  return make_float2(u0 ? 0.f : 1.f / GC0, u1 ? 0.f : 1.f / GC1);
+// Per-chunk record of the exact-path key rows, in shared memory: bit c of `unsafe`
+// (4 words, zeroed by the caller before the prep) is set when channel c has a
+// threshold row, tfirst[c] (128 ints, set to 64 by the prep) is that row.
+struct ExactRows {
+  uint32_t *unsafe;
+  int *tfirst;
+};
+
+// K e^{-g} entry of row r, channel c, from k and e^{g_r} (see the range note above);
+// `marked` keeps the thread from recording the channel twice.
+__device__ __forceinline__ float kh_entry(float k, float eg, int r, int c, const ExactRows &x,
+                                          bool &marked) {
+  if (eg > kFastMinDecay) {      // eg is a normal number here; the result is rounded to bf16
+    float inv;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(eg));
+    return k * inv;
+  }
+  if (!marked) {
+    atomicMin(&x.tfirst[c], r);
+    atomicOr(&x.unsafe[c >> 5], 1u << (c & 31));
+    marked = true;
+  }
+  return 0.f;
 }
 
 struct PrepTiles {
@@ -58,7 +77,7 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
                                                 const float *sg, const uint32_t *valid,
                                                 const PrepTiles &t, float (*part)[kDK],
                                                 float *decay, const float *beta_in,
-                                                float *beta_out, uint32_t *unsafe, int tid) {
+                                                float *beta_out, const ExactRows &xr, int tid) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -75,6 +94,7 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
   part[qt][c] = t0;
   part[qt][c + 1] = t1;
   if (tid < kC) beta_out[tid] = beta_in[tid];
+  if (tid < kDK) xr.tfirst[tid] = kC;
   __syncthreads();
   float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
 #pragma unroll
@@ -88,16 +108,14 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
     decay[c] = GC0;
     decay[c + 1] = GC1;
   }
-  // e^{-g_C}; 0 for channels that take the exact path (their K e^{-g} column is zero)
-  const float2 inv = gram_inv_decay(GC0, GC1, c, unsafe);
-  const float inv0 = inv.x, inv1 = inv.y;
+  bool mk0 = false, mk1 = false;
   const uint32_t *sq = reinterpret_cast<const uint32_t *>(sq16);
   const uint32_t *sk = reinterpret_cast<const uint32_t *>(sk16);
   const int kb = c >> 6, ch = (c & 63) >> 3;
   const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
   const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
   const uint32_t col64 = (uint32_t)(kb * 64 * 128 + (c & 7) * 2);
-  // forward: e^{g_r} -> Q G and K G
+  // forward: e^{g_r} -> Q G, K G and K e^{-g}
   float e0 = pre0, e1 = pre1;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -113,8 +131,10 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
         pack_bf16x2(qa * e0, qb * e1);
     *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
         pack_bf16x2(ka * e0, kb2 * e1);
+    *reinterpret_cast<uint32_t *>(t.kh + col64 + (uint32_t)(r * 128) + sw) =
+        pack_bf16x2(kh_entry(ka, e0, r, c, xr, mk0), kh_entry(kb2, e1, r, c + 1, xr, mk1));
   }
-  // backward: e^{g_C - g_r} -> K e^{g_C - g} and K e^{-g}
+  // backward: e^{g_C - g_r} -> K e^{g_C - g}
   float s0 = suf0, s1 = suf1;
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
@@ -125,7 +145,6 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
     const float ka = __uint_as_float(kk << 16), kb2 = __uint_as_float(kk & 0xFFFF0000u);
     const uint32_t rr = (uint32_t)(r * 128) + sw;
     *reinterpret_cast<uint32_t *>(t.kt + col64 + rr) = pack_bf16x2(ka * s0, kb2 * s1);
-    *reinterpret_cast<uint32_t *>(t.kh + col64 + rr) = pack_bf16x2(ka * (s0 * inv0), kb2 * (s1 * inv1));
     s0 *= a0[i];
     s1 *= a1[i];
   }
@@ -145,7 +164,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
     float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out,
-    uint32_t *unsafe, int tid, bool wait_bulk = false) {
+    const ExactRows &xr, int tid, bool wait_bulk = false) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -181,6 +200,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
   part[qt][c] = t0;
   part[qt][c + 1] = t1;
   if (tid < kC) beta_out[tid] = beta_val;
+  if (tid < kDK) xr.tfirst[tid] = kC;
   // the tiles may still be read by bulk stores thread 0 issued earlier; the tile
   // writes below come after this barrier
   if (wait_bulk && tid == 0) tc::bulk_wait_read();
@@ -198,8 +218,7 @@ __device__ __forceinline__ void decay_and_tiles_global(
     decay[c + 1] = GC1;
     if (gdecay) *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
   }
-  const float2 inv = gram_inv_decay(GC0, GC1, c, unsafe);
-  const float inv0 = inv.x, inv1 = inv.y;
+  bool mk0 = false, mk1 = false;
   const int kb = c >> 6, ch = (c & 63) >> 3;
   const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
   const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
@@ -219,6 +238,8 @@ __device__ __forceinline__ void decay_and_tiles_global(
     if (gq) *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
     *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
         pack_bf16x2(ka * e0, kb2 * e1);
+    *reinterpret_cast<uint32_t *>(t.kh + col64 + (uint32_t)(r * 128) + sw) =
+        pack_bf16x2(kh_entry(ka, e0, r, c, xr, mk0), kh_entry(kb2, e1, r, c + 1, xr, mk1));
   }
   float s0 = suf0, s1 = suf1;
 #pragma unroll
@@ -228,7 +249,6 @@ __device__ __forceinline__ void decay_and_tiles_global(
     const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
     const uint32_t rr = (uint32_t)(r * 128) + sw;
     *reinterpret_cast<uint32_t *>(gkt + col64 + rr) = pack_bf16x2(ka * s0, kb2 * s1);
-    *reinterpret_cast<uint32_t *>(t.kh + col64 + rr) = pack_bf16x2(ka * (s0 * inv0), kb2 * (s1 * inv1));
     s0 *= a0[i];
     s1 *= a1[i];
   }
@@ -294,33 +314,38 @@ __device__ __forceinline__ void pack_tb(const float *Ts, const float *beta, unsi
   }
 }
 
-// Exact Gram terms of the unsafe channels (see the range note at the top).  The
+// Exact Gram terms of the exact-path key rows (see the range note at the top).  The
 // tensor-core Gram in TMEM (lanes 0-63: M rows, lanes 64-127: rows of K K^T before
-// beta; this thread's 32 columns at `tm_acc`) holds every other channel's terms;
-// this adds, for each unsafe channel c and i <= r,
+// beta; this thread's 32 columns at `tm_acc`) holds every other term; this adds,
+// for each channel c with a threshold row t_c and each key row i >= t_c, i <= r,
 //   x[r][c] k[i][c] prod_{i < t <= r} alpha[t][c]      (x = q for M rows, k for A rows)
-// with running products of alpha (all factors <= 1, so no overflow for any
-// log_alpha <= 0; a term underflows only where its true value is below 1e-38).
-// Rows outside `valid` count as alpha = 1, q = k = 0 (identity steps).  q, k and
-// log_alpha are read from global memory (rows c0 .. c0 + 63 of head h).
-// `stage`: >= 12800 bytes of shared memory.  All 256 threads; contains
-// __syncthreads().  The caller skips it when the mask is empty.
+// with running products of alpha (all factors <= 1).  Columns left of every
+// threshold are not touched.  Rows outside `valid` count as alpha = 1, q = k = 0
+// (identity steps).  q, k and log_alpha are read from global memory (rows c0 ..
+// c0 + 63 of head h).  `stage`: >= 12816 bytes of shared memory, free again
+// when the function returns.  All 256 threads; contains __syncthreads().  The
+// caller skips it when no channel has a threshold row.
 template <bool GATE_HEAD>
-__device__ __noinline__ void exact_gram_fixup(uint32_t tm_acc, const uint32_t *unsafe,
+__device__ __noinline__ void exact_gram_fixup(uint32_t tm_acc, const ExactRows &xr,
                                               const uint32_t *valid, const uint16_t *q,
                                               const uint16_t *k, const float *log_alpha, int c0,
                                               int h, int H, float *stage, int tid) {
-  int *list = reinterpret_cast<int *>(stage);   // unsafe channels, ascending
-  float *sa = stage + 128;                      // [16][64] alpha of a group of channels
+  int *list = reinterpret_cast<int *>(stage);   // channels with a threshold row, ascending
+  int *tmin = list + kDK;                       // the smallest threshold row
+  float *sa = stage + 132;                      // [16][64] alpha of a group of channels
   float *sx = sa + 16 * 64;                     // [16][64] q
   float *sk = sx + 16 * 64;                     // [16][64] k
+  const uint32_t *unsafe = xr.unsafe;
   const int n = __popc(unsafe[0]) + __popc(unsafe[1]) + __popc(unsafe[2]) + __popc(unsafe[3]);
+  if (tid == 0) *tmin = kC;
+  __syncthreads();
   if (tid < kDK) {
     const uint32_t w = unsafe[tid >> 5], bit = 1u << (tid & 31);
     if (w & bit) {
       int pos = __popc(w & (bit - 1u));
       for (int j = 0; j < (tid >> 5); ++j) pos += __popc(unsafe[j]);
       list[pos] = tid;
+      atomicMin(tmin, xr.tfirst[tid]);
     }
   }
   const int L = tid & 127, wg = tid >> 7, r = L & 63;
@@ -350,24 +375,28 @@ __device__ __noinline__ void exact_gram_fixup(uint32_t tm_acc, const uint32_t *u
     const int jn = min(16, n - g0);
     for (int j = 0; j < jn; ++j) {
       const float *aj = sa + j * kC, *kj = sk + j * kC;
+      const int tc = xr.tfirst[list[g0 + j]];
       float xP = rowA ? kj[r] : sx[j * kC + r];
       for (int t = ihi + 1; t <= r; ++t) xP *= aj[t];      // prod over (ihi, r]
 #pragma unroll
       for (int u = 31; u >= 0; --u) {
         const int i = ibase + u;
         if (i <= r) {
-          acc[u] = fmaf(xP, kj[i], acc[u]);
+          if (i >= tc) acc[u] = fmaf(xP, kj[i], acc[u]);
           xP *= aj[i];
         }
       }
     }
   }
+  const int t0 = *tmin;
   float v[32];
   tmem_ld32(tm_acc, v);
 #pragma unroll
-  for (int u = 0; u < 32; ++u) v[u] += acc[u];
+  for (int u = 0; u < 32; ++u)
+    if (ibase + u >= t0) v[u] += acc[u];
   tmem_st32(tm_acc, v);
   tmem_st_wait();
+  __syncthreads();   // every thread is done with `stage` before the caller reuses it
 }
 
 __device__ __forceinline__ bool any_unsafe(const uint32_t *unsafe) {

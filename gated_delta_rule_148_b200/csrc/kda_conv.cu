@@ -13,12 +13,11 @@
 //
 // Layout: x, y [N, D] (bf16 or fp32), weight [D, W] fp32, bias [D] fp32,
 // conv_state [B, W-1, D] fp32.  The operation is HBM-bound (read x, write y):
-// kernel A gives each CTA 128 packed positions and up to 1024 channels; the pad
+// kernel A gives each CTA 128 packed positions and up to 2048 channels; the pad
 // mask of those positions is compacted once per CTA (warp ballots) into the list
-// of valid rows, and each thread walks those rows for its 4 consecutive channels
+// of valid rows, and each thread walks those rows for its 8 consecutive channels
 // with the window in registers and the next 8 rows' loads already in flight (a
-// ring of raw 8- or 16-byte loads), so a thread keeps about 8 loads outstanding
-// at a register count that lets several CTAs share an SM.  Kernel B writes the new
+// ring of raw 16- or 32-byte loads), so each thread keeps 8 loads outstanding.  Kernel B writes the new
 // state after kernel A, one thread per (sequence, channel), so conv_state may be
 // updated in place.
 #include "kda_internal.cuh"
@@ -28,9 +27,9 @@ namespace conv {
 
 constexpr int kSeg = 128;            // packed positions per CTA
 constexpr int kThreads = 256;
-constexpr int kPer = 4;              // channels per thread
+constexpr int kPer = 8;              // channels per thread
 constexpr int kChan = kPer * kThreads;  // channels per CTA
-constexpr int kRing = 8;             // rows whose loads are in flight ahead of the walk
+constexpr int kRing = 8;             // rows whose loads are in flight ahead of the walk (bf16)
 constexpr int kMaxW = 4;
 static_assert(kSeg <= kThreads, "one compaction ballot per position");
 
@@ -59,56 +58,90 @@ __device__ __forceinline__ Hist history_before(const uint8_t *mask, int sb, int 
   return hs;
 }
 
-// Raw loads of 4 consecutive channels of one row (8 bytes bf16, 16 bytes fp32),
-// unpacked separately so that several rows' loads can be in flight.
-template <bool BF16> struct Raw4;
-template <> struct Raw4<true> { using T = uint2; };
-template <> struct Raw4<false> { using T = float4; };
+// Raw loads of kPer consecutive channels of one row (kPer bf16 = kPer / 2 words, or
+// kPer fp32 words), unpacked separately so that several rows' loads can be in flight.
+template <bool BF16> __host__ __device__ constexpr int raw_words() { return BF16 ? kPer / 2 : kPer; }
+static_assert(kPer == 2 || kPer == 4 || kPer == 8, "row loads of 4 to 32 bytes");
+template <bool BF16> struct RawRow { uint32_t w[raw_words<BF16>()]; };
 
 template <bool BF16>
-__device__ __forceinline__ typename Raw4<BF16>::T load4(const void *x, size_t row, int D, int c) {
-  if constexpr (BF16)
-    return __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(x) + row * D + c));
-  else
-    return __ldg(reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + row * D + c));
-}
-
-__device__ __forceinline__ void unpack4(uint2 u, float *v) {
-  v[0] = __uint_as_float(u.x << 16);
-  v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-  v[2] = __uint_as_float(u.y << 16);
-  v[3] = __uint_as_float(u.y & 0xFFFF0000u);
-}
-__device__ __forceinline__ void unpack4(float4 u, float *v) {
-  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-}
-
-template <bool BF16>
-__device__ __forceinline__ void store4(void *y, size_t row, int D, int c, const float *v) {
-  if constexpr (BF16) {
-    uint2 u;
-    u.x = (uint32_t)f32_to_bf16_rne(v[0]) | ((uint32_t)f32_to_bf16_rne(v[1]) << 16);
-    u.y = (uint32_t)f32_to_bf16_rne(v[2]) | ((uint32_t)f32_to_bf16_rne(v[3]) << 16);
-    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(y) + row * D + c) = u;
+__device__ __forceinline__ RawRow<BF16> load_row(const void *x, size_t row, int D, int c) {
+  constexpr int n = raw_words<BF16>();
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(x) + (row * D + c) * (BF16 ? 1 : 2) / 2;
+  RawRow<BF16> r;
+  if constexpr (n % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < n; e += 4) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src) + e / 4);
+      r.w[e] = u.x; r.w[e + 1] = u.y; r.w[e + 2] = u.z; r.w[e + 3] = u.w;
+    }
+  } else if constexpr (n == 2) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(src));
+    r.w[0] = u.x; r.w[1] = u.y;
   } else {
-    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + row * D + c) = make_float4(v[0], v[1], v[2], v[3]);
+    r.w[0] = __ldg(src);
+  }
+  return r;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void unpack_row(const RawRow<BF16> &r, float *v) {
+  if constexpr (BF16) {
+#pragma unroll
+    for (int e = 0; e < kPer / 2; ++e) {
+      v[2 * e] = __uint_as_float(r.w[e] << 16);
+      v[2 * e + 1] = __uint_as_float(r.w[e] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) v[e] = __uint_as_float(r.w[e]);
+  }
+}
+
+// Two fp32 -> packed bf16x2, round to nearest even; `lo` lands in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_row(void *y, size_t row, int D, int c, const float *v) {
+  RawRow<BF16> r;
+  if constexpr (BF16) {
+#pragma unroll
+    for (int e = 0; e < kPer / 2; ++e) r.w[e] = bf16x2_rn(v[2 * e], v[2 * e + 1]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) r.w[e] = __float_as_uint(v[e]);
+  }
+  constexpr int n = raw_words<BF16>();
+  uint32_t *dst = reinterpret_cast<uint32_t *>(y) + (row * D + c) * (BF16 ? 1 : 2) / 2;
+  if constexpr (n % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < n; e += 4)
+      reinterpret_cast<uint4 *>(dst)[e / 4] = make_uint4(r.w[e], r.w[e + 1], r.w[e + 2], r.w[e + 3]);
+  } else if constexpr (n == 2) {
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(r.w[0], r.w[1]);
+  } else {
+    *dst = r.w[0];
   }
 }
 
 // Kernel A: outputs of packed positions [kSeg*blockIdx.x, +kSeg), channels
-// [kChan*blockIdx.y, +kChan).  Thread t owns channels 4t .. 4t+3 and walks the
+// [kChan*blockIdx.y, +kChan).  Thread t owns channels 8t .. 8t+7 and walks the
 // CTA's valid rows in order with the window in registers, so each x row is read
 // once; the loads of one row are coalesced across the CTA's threads, and the
 // ring keeps the loads of the next kRing rows in flight.
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, BF16 ? 4 : 2) conv_kernel(ConvParams p) {
-  using Raw = typename Raw4<BF16>::T;
+template <bool BF16, int KW>      // KW: the window width W (1..4), fixed at compile time
+__global__ void __launch_bounds__(kThreads, 2) conv_kernel(ConvParams p) {
   __shared__ int vpos[kSeg];
   __shared__ int wcnt[kThreads / 32];
   __shared__ Hist hist_sh;
   if (device_error_latched(p.err)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int W = p.W, D = p.D, B = p.num_seqs;
+  constexpr int W = KW;
+  const int D = p.D, B = p.num_seqs;
   const int s0 = blockIdx.x * kSeg, s1 = min(s0 + kSeg, p.N);
   const int c_lo = blockIdx.y * kChan, nch = min(kChan, D - c_lo);
   if (blockIdx.x == 0 && blockIdx.y == 0) {       // cu_seqlens: 0, non-decreasing, ends at N
@@ -163,23 +196,25 @@ __global__ void __launch_bounds__(kThreads, BF16 ? 4 : 2) conv_kernel(ConvParams
         for (int q = 0; q < kPer; ++q) win[j][q] = 0.f;
         if (j < W - 1) {
           const int src = hist_sh.src[j];
-          if (src >= 0) unpack4(load4<BF16>(p.x, (size_t)src, D, c), win[j]);
-          else if (p.state_in) unpack4(load4<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c), win[j]);
+          if (src >= 0) unpack_row<BF16>(load_row<BF16>(p.x, (size_t)src, D, c), win[j]);
+          else if (p.state_in)
+            unpack_row<false>(load_row<false>(p.state_in, (size_t)b * (W - 1) + (-1 - src), D, c), win[j]);
         }
       }
       // ---- walk the valid rows; ring[u] holds the raw load of row m0 + u
-      Raw ring[kRing];
+      constexpr int ring_n = BF16 ? kRing : kRing / 2;     // fp32 rows are twice as wide
+      RawRow<BF16> ring[ring_n];
 #pragma unroll
-      for (int u = 0; u < kRing; ++u)
-        if (u < nvalid) ring[u] = load4<BF16>(p.x, (size_t)vpos[u], D, c);
-      for (int m0 = 0; m0 < nvalid; m0 += kRing) {
+      for (int u = 0; u < ring_n; ++u)
+        if (u < nvalid) ring[u] = load_row<BF16>(p.x, (size_t)vpos[u], D, c);
+      for (int m0 = 0; m0 < nvalid; m0 += ring_n) {
 #pragma unroll
-        for (int u = 0; u < kRing; ++u) {
+        for (int u = 0; u < ring_n; ++u) {
           const int m = m0 + u;
           if (m < nvalid) {
             float xv[kPer], acc[kPer];
-            unpack4(ring[u], xv);
-            if (m + kRing < nvalid) ring[u] = load4<BF16>(p.x, (size_t)vpos[m + kRing], D, c);
+            unpack_row<BF16>(ring[u], xv);
+            if (m + ring_n < nvalid) ring[u] = load_row<BF16>(p.x, (size_t)vpos[m + ring_n], D, c);
 #pragma unroll
             for (int q = 0; q < kPer; ++q) acc[q] = fmaf(wx[q], xv[q], bz[q]);
             // taps: u_i = win[i] for i < W-1 (zero taps beyond), u_{W-1} = x_t
@@ -187,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, BF16 ? 4 : 2) conv_kernel(ConvParams
             for (int i = 0; i < kMaxW - 1; ++i)
 #pragma unroll
               for (int q = 0; q < kPer; ++q) acc[q] = fmaf(wt[i][q], win[i][q], acc[q]);
-            store4<BF16>(p.y, (size_t)vpos[m], D, c, acc);
+            store_row<BF16>(p.y, (size_t)vpos[m], D, c, acc);
             // shift: the newest of the W-1 slots becomes x_t
 #pragma unroll
             for (int j = 0; j < kMaxW - 2; ++j)
@@ -206,9 +241,11 @@ __global__ void __launch_bounds__(kThreads, BF16 ? 4 : 2) conv_kernel(ConvParams
       }
       // ---- pads: y = 0
       if (p.mask != nullptr && nvalid < e - a) {
-        const float z[kPer] = {0.f, 0.f, 0.f, 0.f};
+        float z[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) z[q] = 0.f;
         for (int r = a; r < e; ++r)
-          if (p.mask[r] == 0) store4<BF16>(p.y, (size_t)r, D, c, z);
+          if (p.mask[r] == 0) store_row<BF16>(p.y, (size_t)r, D, c, z);
       }
     }
     __syncthreads();   // vpos, wcnt and hist_sh are rewritten by the next sequence
@@ -251,8 +288,11 @@ cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s) {
   using namespace conv;
   if (p.N > 0) {
     const dim3 grid((unsigned)((p.N + kSeg - 1) / kSeg), (unsigned)((p.D + kChan - 1) / kChan));
-    if (bf16) conv_kernel<true><<<grid, kThreads, 0, s>>>(p);
-    else conv_kernel<false><<<grid, kThreads, 0, s>>>(p);
+    using Kern = void (*)(ConvParams);
+    static const Kern kerns[2][4] = {
+        {conv_kernel<false, 1>, conv_kernel<false, 2>, conv_kernel<false, 3>, conv_kernel<false, 4>},
+        {conv_kernel<true, 1>, conv_kernel<true, 2>, conv_kernel<true, 3>, conv_kernel<true, 4>}};
+    kerns[bf16 ? 1 : 0][p.W - 1]<<<grid, kThreads, 0, s>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -38,6 +38,7 @@ struct PrefillParams {
   int gate_head;          // 1: log_alpha is [N, H] (one gate per token and head)
   long long wait_cycles;  // limit of every bounded device wait
   int fault;              // test faults (FAULT_*), 0 in normal use
+  unsigned *site;         // device word: code of the first bounded wait that ran out
 };
 
 // Faults a test can plant with kda_debug_set_fault() to exercise the bounded
@@ -127,6 +128,11 @@ __device__ __forceinline__ void store_elem(void *base, size_t idx, float val) {
 // head-wise gate, [rows, H] (the same value for every channel).
 __device__ __forceinline__ size_t la_index(size_t row, int h, int H, int dk, int c, int gate_head) {
   return gate_head ? row * H + h : (row * H + h) * dk + c;
+}
+
+// Records which bounded wait ran out first (codes listed with kda_debug_timeout_site()).
+__device__ __forceinline__ void note_timeout(unsigned *site, unsigned code) {
+  if (site) atomicCAS(site, 0u, code);
 }
 
 __device__ __forceinline__ bool device_error_latched(const unsigned *err) {

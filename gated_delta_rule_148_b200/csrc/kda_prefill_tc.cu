@@ -138,7 +138,9 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
   __shared__ __align__(8) uint64_t stage_bar;
   __shared__ __align__(8) uint64_t v_bar;
   __shared__ uint32_t valid_sh[2];      // validity bits of the chunk's 64 rows
-  __shared__ uint32_t unsafe_sh[4];     // channels whose Gram terms take the exact path
+  __shared__ uint32_t unsafe_sh[4];     // channels with exact-path key rows
+  __shared__ int tfirst_sh[128];        // their first exact-path key row
+  const prep::ExactRows xrows{unsafe_sh, tfirst_sh};
   __shared__ float decay_sh[kDK];      // e^{g_C} per key channel
   __shared__ float beta_sh[kC];
   __shared__ float part_sh[4][kDK];
@@ -210,7 +212,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
     }
     if (tid < 4) unsafe_sh[tid] = 0u;
-    ok = __syncthreads_and(mbar_wait(&stage_bar, chunk_idx & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&stage_bar, chunk_idx & 1, p.wait_cycles) || (note_timeout(p.site, 21), false));
     if (!ok) break;
     // ---- P1: decay products and operand tiles
     {
@@ -222,7 +224,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
       prep::decay_and_tiles(reinterpret_cast<const uint16_t *>(base + OFF_STQ),
                             reinterpret_cast<const uint16_t *>(base + OFF_STK),
                             reinterpret_cast<const float *>(base + OFF_STG), valid_sh, t, part_sh,
-                            decay_sh, stb, beta_sh, unsafe_sh, tid);
+                            decay_sh, stb, beta_sh, xrows, tid);
     }
     fence_async_smem();
     __syncthreads();
@@ -234,14 +236,14 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_G, desc_kmajor(sQKW, 192, 64, s), desc_kmajor(sKH, 64, 0, s), id, s > 0);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles) || (note_timeout(p.site, 22), false));
     phase++;
     if (!ok) break;
     fence_after_sync();
     // channels whose chunk decay is out of the factorised range: exact terms added
     // (K e^{-g} has been read by the Gram: its region stages the fix-up)
     if (prep::any_unsafe(unsafe_sh))
-      prep::exact_gram_fixup<false>(tm + my_cols + TM_G, unsafe_sh, valid_sh,
+      prep::exact_gram_fixup<false>(tm + my_cols + TM_G, xrows, valid_sh,
                                     reinterpret_cast<const uint16_t *>(p.q),
                                     reinterpret_cast<const uint16_t *>(p.k), p.log_alpha, c0, h, H,
                                     reinterpret_cast<float *>(base + OFF_KH), tid);
@@ -256,7 +258,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
     // the staging buffers are free: stream the next chunk's q, k, log_alpha, beta
     if (c0 + kC < sp.end) stage_chunk(p, maps, sp, c0 + kC, h, base, &stage_bar, tid);
     // V of this chunk must have landed; zero its invalid rows
-    ok = __syncthreads_and(mbar_wait(&v_bar, chunk_idx & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&v_bar, chunk_idx & 1, p.wait_cycles) || (note_timeout(p.site, 23), false));
     if (!ok) break;
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
       for (int e = tid; e < kC * 8; e += kThreads) {
@@ -278,7 +280,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_D1, desc_kmajor(sTBM, 192, 0, s), desc_mnmajor(sV, 64, 0, s), idu, s > 0);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles) || (note_timeout(p.site, 24), false));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -311,7 +313,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_D1, desc_kmajor(sQKW, 192, 0, s), desc_mnmajor(sSB, 128, 0, s), id, 1);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles) || (note_timeout(p.site, 25), false));
     phase++;
     if (!ok) break;
     fence_after_sync();
@@ -335,7 +337,7 @@ prefill_tc_kernel(PrefillParams p, const __grid_constant__ TmaMaps maps) {
         mma_bf16(tm + TM_S, desc_mnmajor(sKT, 64, 0, s), desc_mnmajor(sUB, 64, 0, s), ids, 1);
       mma_commit(&mma_bar);
     }
-    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles));
+    ok = __syncthreads_and(mbar_wait(&mma_bar, phase & 1, p.wait_cycles) || (note_timeout(p.site, 26), false));
     phase++;
     if (!ok) break;
     fence_after_sync();

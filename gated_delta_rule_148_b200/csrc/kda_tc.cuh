@@ -205,12 +205,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
          "r"(smem_u32(bar)) : "memory");
 }
 
-// TMA prefetch of a 3-D tensor map box into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
-               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2) : "memory");
-}
-
 // Bulk (TMA, non-tensor) copies; addresses 16-byte aligned, sizes multiples of 16.
 __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src_gmem, uint32_t bytes,
                                           uint64_t *bar) {

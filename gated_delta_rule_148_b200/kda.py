@@ -33,7 +33,8 @@ KDA_GATE_HEAD = 1
 
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_get_device_status",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_short_conv",
-            "kda_prefill_backward", "kda_prefill_backward_workspace_size", "kda_debug_set_fault")
+            "kda_prefill_backward", "kda_prefill_backward_workspace_size", "kda_debug_set_fault",
+            "kda_debug_timeout_site")
 KDA_FAULT_STARVE_STATE_LOADS = 1
 
 
@@ -124,6 +125,8 @@ def load(build_if_stale: bool = True) -> ctypes.CDLL:
             lib.kda_prefill_noalloc.restype = ctypes.c_int
             lib.kda_debug_set_fault.argtypes = [ctypes.c_int, ctypes.c_longlong]
             lib.kda_debug_set_fault.restype = ctypes.c_int
+            lib.kda_debug_timeout_site.argtypes = [ctypes.c_void_p]
+            lib.kda_debug_timeout_site.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -378,6 +381,11 @@ def debug_set_fault(fault: int, wait_cycles: int = 0) -> None:
     st = load().kda_debug_set_fault(int(fault), int(wait_cycles))
     if st != KDA_OK:
         raise KdaError(st, "kda_debug_set_fault")
+
+
+def debug_timeout_site(stream=None) -> int:
+    """kda_debug_timeout_site: code of the first bounded wait that ran out (0 = none)."""
+    return int(load().kda_debug_timeout_site(_stream_handle(stream)))
 
 
 def raw_prefill(args: PrefillArgs, stream=None) -> int:

@@ -109,7 +109,7 @@ typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1 } kda_gate;
  *   workspace    device scratch, 256-byte aligned.  kda_prefill_workspace_size()
  *                bytes select the fastest path (for bf16, d_k = d_v = 128,
  *                chunk 64: a two-kernel path that stores each chunk's
- *                intermediate tiles, 88 KB per 64 tokens and head).  A
+ *                intermediate tiles, about 73 KB per 64 tokens and head).  A
  *                smaller workspace selects a fused single-kernel path; a pad
  *                mask needs at least 16 bytes per sequence (rounded up to 256).
  *                May be NULL when pad_mask is NULL.
@@ -325,6 +325,18 @@ kda_status kda_get_device_status(void *stream);
  */
 #define KDA_FAULT_STARVE_STATE_LOADS 1
 kda_status kda_debug_set_fault(int fault, long long wait_cycles);
+
+/*
+ * Which bounded wait ran out first on the current device since the last call
+ * (0: none): a diagnostic beside KDA_ERR_DEVICE_TIMEOUT.  Synchronises
+ * `stream`, then returns and clears the code; -1 if a CUDA call failed.
+ * Codes: workspace-backed tensor-core prefill, intra-chunk kernel: 1 Gram
+ * products, 2 V tile, 3 W and U_v products; its state pass: 11 item load,
+ * 12 first product group of a chunk, 13 second product group, 14 buffer
+ * release (loading side); single-kernel tensor-core prefill: 21-26 (its six
+ * waits in program order).
+ */
+int kda_debug_timeout_site(void *stream);
 
 /* Static string for a status code; never NULL. */
 const char *kda_status_string(kda_status status);

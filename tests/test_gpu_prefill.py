@@ -454,6 +454,7 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     finally:
         kda.debug_set_fault(0)
     assert st == kda.KDA_ERR_DEVICE_TIMEOUT, kda.status_string(st)
+    assert kda.debug_timeout_site() == 11              # the state pass's item-load wait
     assert kda.get_device_status() == kda.KDA_OK       # the latch was cleared
     o, fs = _gpu(inp, "bf16")
     _check(inp, "bf16", o, fs)

@@ -565,47 +565,3 @@ def test_backward_zero_upstream_and_state_only():
     for t in range(N):
         np.testing.assert_allclose(g["dlog_alpha"][t, 0], (dSf[0, 0] * ST).sum(axis=1), rtol=1e-12)
 
-
-# ---------------------------------------------------------------- the regrouped chunk step
-def _regrouped(q, k, v, la, beta, chunk, S0):
-    """The chunk step as the tensor-core state pass groups it (its own numpy restatement,
-    fp64): with P'' = -(K e^{g_C-g})^T W - Diag(1 - e^{g_C}) and R = (Q e^g) - M W,
-    S <- S + P'' S + (K e^{g_C-g})^T U_v and O = R S + M U_v."""
-    q, k, v, la, beta = (np.asarray(x, np.float64) for x in (q, k, v, la, beta))
-    T, dk = k.shape
-    S = np.array(S0, np.float64)
-    o = np.zeros((T, v.shape[1]))
-    for c0 in range(0, T, chunk):
-        Q, K, V, b = q[c0:c0 + chunk], k[c0:c0 + chunk], v[c0:c0 + chunk], beta[c0:c0 + chunk]
-        g = np.cumsum(la[c0:c0 + chunk], axis=0)
-        C = K.shape[0]
-        A = np.zeros((C, C))
-        M = np.zeros((C, C))
-        for r in range(C):
-            for i in range(r + 1):
-                d = np.exp(g[r] - g[i])
-                M[r, i] = np.sum(Q[r] * K[i] * d)
-                if i < r:
-                    A[r, i] = b[r] * np.sum(K[r] * K[i] * d)
-        L = np.eye(C) + A
-        W = np.linalg.solve(L, b[:, None] * (K * np.exp(g)))
-        Uv = np.linalg.solve(L, b[:, None] * V)
-        Kt = K * np.exp(g[-1] - g)
-        P2 = -Kt.T @ W - np.diag(1.0 - np.exp(g[-1]))
-        R = Q * np.exp(g) - M @ W
-        o[c0:c0 + C] = R @ S + M @ Uv
-        S = S + P2 @ S + Kt.T @ Uv
-    return o, S
-
-
-@pytest.mark.parametrize("chunk,T", [(16, 50), (64, 200)])
-def test_regrouped_chunk_step_equals_recurrence(chunk, T):
-    """The single-product-group form the state pass runs (one group of products per
-    chunk on the chain, the outputs from a second group) is the recurrence, in fp64."""
-    dk, dv = 12, 10
-    q, k, v, la, beta = _one(21, T, dk, dv)
-    S0 = np.random.default_rng(22).normal(0, 0.1, (dk, dv)).astype(np.float32)
-    o, S = _run1(q, k, v, la, beta, S0)
-    o2, S2 = _regrouped(q, k, v, la, beta, chunk, S0)
-    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-10 * max(1.0, np.abs(o).max()))
-    np.testing.assert_allclose(S2, S, rtol=0, atol=1e-10 * max(1.0, np.abs(S).max()))
