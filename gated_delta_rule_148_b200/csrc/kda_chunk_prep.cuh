@@ -158,13 +158,14 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
 // into the 64-row tile `gkt` (global or shared memory, same swizzled layout), and
 // e^{g_C} into `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
 // beta_val (threads 0..63: beta of row tid, already in a register) is stored to
-// beta_out after the row loads are issued, so its latency overlaps theirs.
+// beta_out after the row loads are issued, so its latency overlaps theirs.  With
+// `sla`, log_alpha comes from that staged [64][128] f32 tile instead of global memory.
 template <bool GATE_HEAD>
 __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
     float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out,
-    const ExactRows &xr, int tid, bool wait_bulk = false) {
+    const ExactRows &xr, int tid, bool wait_bulk = false, const float *sla = nullptr) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -180,6 +181,8 @@ __device__ __forceinline__ void decay_and_tiles_global(
       if (GATE_HEAD) {
         const float gv = __ldg(log_alpha + (size_t)(c0 + qt * 16 + i) * H + h);
         la = make_float2(gv, gv);
+      } else if (sla) {
+        la = *reinterpret_cast<const float2 *>(sla + (qt * 16 + i) * kDK + c);
       } else {
         la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
       }

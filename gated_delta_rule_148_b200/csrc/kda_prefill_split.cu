@@ -147,14 +147,28 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, const P
   return __syncthreads_and(w);
 }
 
+// Tensor maps of the intra kernel's inputs: V [N, H, dv] (64-column boxes, 128-byte
+// swizzle, straight into its operand tile) and log_alpha [N, H, dk] (one item's
+// 64 x 128 f32 rows, no swizzle, staged for the decay prep).
+struct IntraMaps {
+  CUtensorMap v, la;
+};
+
+// log_alpha of the next item is loaded by TMA into the T_b and V tiles (32 KB) as soon
+// as the current item's products have read them; the plain per-thread loads it
+// replaces were limited by the number of misses an SM keeps in flight.  V follows once
+// the prep has read the staged rows.  (Not with the head-wise gate: 4 bytes per row.)
 template <bool GATE_HEAD>     // log_alpha [N, H] (one gate per token and head) instead of [N, H, dk]
 __global__ void __launch_bounds__(kThreadsA, 2)
-intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const SeqSpan *spans,
+intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqSpan *spans,
              const int *cbase, unsigned char *items, int h0, int Hg) {
+  constexpr bool kStageLa = !GATE_HEAD;
+  const CUtensorMap &vmap = maps.v;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t v_bar;
+  __shared__ __align__(8) uint64_t la_bar;
   __shared__ uint32_t valid_sh[2];
   __shared__ uint32_t unsafe_sh[4];     // channels with exact-path key rows
   __shared__ int tfirst_sh[128];        // their first exact-path key row
@@ -177,6 +191,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
     mbar_init(&v_bar, 1);
+    mbar_init(&la_bar, 1);
   }
   for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0, for good
     const int r = 64 + (e >> 3), ch = e & 7;
@@ -189,16 +204,23 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
   const uint32_t sQK = smem_u32(base + A_QK), sKH = smem_u32(base + A_KH);
   const uint32_t sTB = smem_u32(base + A_TB), sV = smem_u32(base + A_V);
-  uint32_t phase = 0, vphase = 0;
+  uint32_t phase = 0, vphase = 0, lphase = 0;
   bool ok = true;
+  constexpr uint32_t kLaBytes = 64 * kDK * 4;
+  static_assert(A_TB + kLaBytes <= A_TS, "staged log_alpha fits the T_b and V tiles");
 
   // V of an item is requested as soon as the previous item's products have read
   // the V tile, so its copy overlaps that item's read-out and stores.
   if (tid == 0 && (int)blockIdx.x < nitems) {
     const ItemPos ip = locate_item(p, spans, cbase, blockIdx.x, h0, Hg);
-    mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
-    tma_load_3d(sV, &vmap, 0, ip.h, ip.c0, &v_bar);
-    tma_load_3d(sV + 64 * 128, &vmap, 64, ip.h, ip.c0, &v_bar);
+    if (kStageLa) {
+      mbar_arrive_expect_tx(&la_bar, kLaBytes);
+      tma_load_3d(sTB, &maps.la, 0, ip.h, ip.c0, &la_bar);
+    } else {
+      mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+      tma_load_3d(sV, &vmap, 0, ip.h, ip.c0, &v_bar);
+      tma_load_3d(sV + 64 * 128, &vmap, 64, ip.h, ip.c0, &v_bar);
+    }
   }
   bool first = true;
   for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
@@ -215,8 +237,15 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
     if (tid < 4) unsafe_sh[tid] = 0u;
-    __syncthreads();
-    // ---- decay products and operand tiles (global loads; V is already on its way)
+    if (kStageLa) {
+      ok = wait_all(&la_bar, lphase & 1, p, 4);
+      lphase++;
+      if (!ok) break;
+    } else {
+      __syncthreads();
+    }
+    // ---- decay products and operand tiles (q, k from global memory; log_alpha staged or
+    //      from global memory; V is already on its way or follows)
     {
       prep::PrepTiles t;
       t.qg = base + A_QK; t.qg_R = 128; t.qg_row0 = 0;
@@ -226,7 +255,22 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
       prep::decay_and_tiles_global<GATE_HEAD>(
           reinterpret_cast<const uint16_t *>(p.q), reinterpret_cast<const uint16_t *>(p.k), p.log_alpha,
           c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
-          decay_sh, beta_val, beta_sh, xrows, tid, !first);
+          decay_sh, beta_val, beta_sh, xrows, tid, !first,
+          kStageLa ? reinterpret_cast<const float *>(base + A_TB) : nullptr);
+    }
+    if (kStageLa) {
+      // the staged rows are read: rows 64..127 of [T_b | 0] back to zero, V into its tile
+      fence_async_smem();
+      __syncthreads();
+      for (int e = tid; e < 64 * 8; e += kThreadsA) {
+        const int r = 64 + (e >> 3), ch = e & 7;
+        *reinterpret_cast<uint4 *>(base + A_TB + row_tile_chunk(r, 0, ch, 128)) = make_uint4(0, 0, 0, 0);
+      }
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+        tma_load_3d(sV, &vmap, 0, h, c0, &v_bar);
+        tma_load_3d(sV + 64 * 128, &vmap, 64, h, c0, &v_bar);
+      }
     }
     fence_async_smem();
     __syncthreads();
@@ -308,11 +352,16 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
     phase++;
     if (!ok) break;
     fence_after_sync();
-    if (tid == 0 && item + (int)gridDim.x < nitems) {   // the V tile is free: next item's V
+    if (tid == 0 && item + (int)gridDim.x < nitems) {   // the T_b and V tiles are free
       const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
-      mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
-      tma_load_3d(sV, &vmap, 0, nx.h, nx.c0, &v_bar);
-      tma_load_3d(sV + 64 * 128, &vmap, 64, nx.h, nx.c0, &v_bar);
+      if (kStageLa) {            // next item's log_alpha
+        mbar_arrive_expect_tx(&la_bar, kLaBytes);
+        tma_load_3d(sTB, &maps.la, 0, nx.h, nx.c0, &la_bar);
+      } else {                   // next item's V
+        mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
+        tma_load_3d(sV, &vmap, 0, nx.h, nx.c0, &v_bar);
+        tma_load_3d(sV + 64 * 128, &vmap, 64, nx.h, nx.c0, &v_bar);
+      }
     }
     if ((warp & 3) < 2) {
       // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> rows 0..63 of the Q G | K G
@@ -342,6 +391,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ CUtensorMap vmap, const Se
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
     mbar_wait(&v_bar, (vphase - 0) & 1, 20000);
+    if (kStageLa) mbar_wait(&la_bar, lphase & 1, 20000);
     if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
   }
   if (tid == 0) {
@@ -715,8 +765,13 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   chunk_index_kernel<<<1, 1024, 0, s>>>(p, spans, cbase);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap vmap;
-  if (!encode_3d(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV, CU_TENSOR_MAP_SWIZZLE_128B))
+  IntraMaps maps;
+  if (!encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
+  if (p.gate_head) maps.la = maps.v;      // not used: the head-wise gate is read per row
+  else if (!encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorNotSupported;
   auto intra = p.gate_head ? intra_kernel<true> : intra_kernel<false>;
   e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
@@ -731,7 +786,7 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
   if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
   const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
-  intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, vmap, spans, cbase, items, 0, p.H);
+  intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, maps, spans, cbase, items, 0, p.H);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / (narrow ? 32 : 64));
   state<<<gridB, kThreadsB, smem_b, s>>>(p, spans, cbase, items, 0, p.H);

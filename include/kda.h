@@ -331,7 +331,8 @@ kda_status kda_debug_set_fault(int fault, long long wait_cycles);
  * (0: none): a diagnostic beside KDA_ERR_DEVICE_TIMEOUT.  Synchronises
  * `stream`, then returns and clears the code; -1 if a CUDA call failed.
  * Codes: workspace-backed tensor-core prefill, intra-chunk kernel: 1 Gram
- * products, 2 V tile, 3 W and U_v products; its state pass: 11 item load,
+ * products, 2 V tile, 3 W and U_v products, 4 staged log_alpha rows; its state
+ * pass: 11 item load,
  * 12 first product group of a chunk, 13 second product group, 14 buffer
  * release (loading side); single-kernel tensor-core prefill: 21-26 (its six
  * waits in program order).
