@@ -571,11 +571,14 @@ def bench_conv(K, W, world, device, pk, xs, seed):
     if kda.get_device_status() != kda.KDA_OK:
         raise RuntimeError("device status after the short convolution")
     nb = len(xs) * (2 * T * D * 2 + 2 * 3 * D * 4 + D * 5 * 4)
+    tr = recorded_traffic("short_conv")     # recorded for 3 calls at T = 131072, D = 4096
+    if tr is not None:
+        tr = int(round(tr * (len(xs) / 3) * (T / 131072) * (D / 4096)))
     return {"workload": f"short_conv_{len(xs)}x_T{T}_D{D}_W4_bf16",
             "tokens_per_s": aggregate_rate(T, world, ms), "ms": ms,
             "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                         "algorithmic_bytes_per_step": nb}}
+                         "traffic": tr, "algorithmic_bytes_per_step": nb}}
 
 
 def main_conv_only(args, rank, world, device):
