@@ -159,13 +159,16 @@ __device__ __forceinline__ void decay_and_tiles(const uint16_t *sq16, const uint
 // e^{g_C} into `gdecay` (global) and `decay` (shared).  One __syncthreads(); 256 threads.
 // beta_val (threads 0..63: beta of row tid, already in a register) is stored to
 // beta_out after the row loads are issued, so its latency overlaps theirs.  With
-// `sla`, log_alpha comes from that staged [64][128] f32 tile instead of global memory.
+// `sla` (and `sq`, `sk`), log_alpha (and q, k) come from staged [64][128] row-major
+// tiles instead of global memory; they are read before the internal barrier, so the
+// operand tiles may be written over them.
 template <bool GATE_HEAD>
 __device__ __forceinline__ void decay_and_tiles_global(
     const uint16_t *q, const uint16_t *k, const float *log_alpha, int c0, int h, int H,
     const uint32_t *valid, const PrepTiles &t, unsigned char *gq, unsigned char *gkt,
     float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out,
-    const ExactRows &xr, int tid, bool wait_bulk = false, const float *sla = nullptr) {
+    const ExactRows &xr, int tid, bool wait_bulk = false, const float *sla = nullptr,
+    const uint16_t *sq = nullptr, const uint16_t *sk = nullptr) {
   const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
   const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
   float a0[16], a1[16];
@@ -186,8 +189,13 @@ __device__ __forceinline__ void decay_and_tiles_global(
       } else {
         la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
       }
-      qv[i] = __ldg(reinterpret_cast<const unsigned int *>(q + row));
-      kv[i] = __ldg(reinterpret_cast<const unsigned int *>(k + row));
+      if (sq) {
+        qv[i] = *reinterpret_cast<const uint32_t *>(sq + (qt * 16 + i) * kDK + c);
+        kv[i] = *reinterpret_cast<const uint32_t *>(sk + (qt * 16 + i) * kDK + c);
+      } else {
+        qv[i] = __ldg(reinterpret_cast<const unsigned int *>(q + row));
+        kv[i] = __ldg(reinterpret_cast<const unsigned int *>(k + row));
+      }
     }
     a0[i] = la.x;
     a1[i] = la.y;

@@ -148,27 +148,30 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, const P
 }
 
 // Tensor maps of the intra kernel's inputs: V [N, H, dv] (64-column boxes, 128-byte
-// swizzle, straight into its operand tile) and log_alpha [N, H, dk] (one item's
-// 64 x 128 f32 rows, no swizzle, staged for the decay prep).
+// swizzle, straight into its operand tile) and log_alpha, q, k [N, H, dk] (one item's
+// 64 x 128 rows, no swizzle, staged for the decay prep).
 struct IntraMaps {
-  CUtensorMap v, la;
+  CUtensorMap v, la, q, k;
 };
 
-// log_alpha of the next item is loaded by TMA into the T_b and V tiles (32 KB) as soon
-// as the current item's products have read them; the plain per-thread loads it
-// replaces were limited by the number of misses an SM keeps in flight.  V follows once
-// the prep has read the staged rows.  (Not with the head-wise gate: 4 bytes per row.)
+// The next item's inputs are loaded by TMA into tiles the current item no longer
+// needs, so the prep reads them from shared memory: q into the K e^{g_C-g} / T tile
+// once T_b is packed, log_alpha into the T_b and V tiles (32 KB) once the W and U_v
+// products have read them, k into the K e^{-g} tile once the item's bulk stores have
+// read it.  V follows once the prep has read the staged rows.  (The plain per-thread
+// loads this replaces were held up by the number of misses an SM keeps in flight.)
+// With the head-wise gate (4 bytes of gate per row) the inputs are plain loads.
 template <bool GATE_HEAD>     // log_alpha [N, H] (one gate per token and head) instead of [N, H, dk]
 __global__ void __launch_bounds__(kThreadsA, 2)
 intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqSpan *spans,
              const int *cbase, unsigned char *items, int h0, int Hg) {
-  constexpr bool kStageLa = !GATE_HEAD;
+  constexpr bool kStage = !GATE_HEAD;
   const CUtensorMap &vmap = maps.v;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t v_bar;
-  __shared__ __align__(8) uint64_t la_bar;
+  __shared__ __align__(8) uint64_t in_bar;     // the three staged inputs of an item
   __shared__ uint32_t valid_sh[2];
   __shared__ uint32_t unsafe_sh[4];     // channels with exact-path key rows
   __shared__ int tfirst_sh[128];        // their first exact-path key row
@@ -191,7 +194,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
     mbar_init(&v_bar, 1);
-    mbar_init(&la_bar, 1);
+    mbar_init(&in_bar, 3);
   }
   for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0, for good
     const int r = 64 + (e >> 3), ch = e & 7;
@@ -204,18 +207,32 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   const uint32_t my_cols = lane_base + (uint32_t)(wg * 32);
   const uint32_t sQK = smem_u32(base + A_QK), sKH = smem_u32(base + A_KH);
   const uint32_t sTB = smem_u32(base + A_TB), sV = smem_u32(base + A_V);
-  uint32_t phase = 0, vphase = 0, lphase = 0;
+  uint32_t phase = 0, vphase = 0, iphase = 0;
   bool ok = true;
-  constexpr uint32_t kLaBytes = 64 * kDK * 4;
+  constexpr uint32_t kLaBytes = 64 * kDK * 4, kQkBytes = 64 * kDK * 2;
   static_assert(A_TB + kLaBytes <= A_TS, "staged log_alpha fits the T_b and V tiles");
+  static_assert(kQkBytes <= A_TB - A_KH && kQkBytes <= A_XS - A_TS, "staged q, k fit their tiles");
+  auto stage_q = [&](int hh, int cc) {
+    mbar_arrive_expect_tx(&in_bar, kQkBytes);
+    tma_load_3d(smem_u32(base + A_TS), &maps.q, 0, hh, cc, &in_bar);
+  };
+  auto stage_k = [&](int hh, int cc) {
+    mbar_arrive_expect_tx(&in_bar, kQkBytes);
+    tma_load_3d(sKH, &maps.k, 0, hh, cc, &in_bar);
+  };
+  auto stage_la = [&](int hh, int cc) {
+    mbar_arrive_expect_tx(&in_bar, kLaBytes);
+    tma_load_3d(sTB, &maps.la, 0, hh, cc, &in_bar);
+  };
 
   // V of an item is requested as soon as the previous item's products have read
   // the V tile, so its copy overlaps that item's read-out and stores.
   if (tid == 0 && (int)blockIdx.x < nitems) {
     const ItemPos ip = locate_item(p, spans, cbase, blockIdx.x, h0, Hg);
-    if (kStageLa) {
-      mbar_arrive_expect_tx(&la_bar, kLaBytes);
-      tma_load_3d(sTB, &maps.la, 0, ip.h, ip.c0, &la_bar);
+    if (kStage) {
+      stage_q(ip.h, ip.c0);
+      stage_la(ip.h, ip.c0);
+      stage_k(ip.h, ip.c0);
     } else {
       mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
       tma_load_3d(sV, &vmap, 0, ip.h, ip.c0, &v_bar);
@@ -237,9 +254,9 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
       if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
     if (tid < 4) unsafe_sh[tid] = 0u;
-    if (kStageLa) {
-      ok = wait_all(&la_bar, lphase & 1, p, 4);
-      lphase++;
+    if (kStage) {
+      ok = wait_all(&in_bar, iphase & 1, p, 4);
+      iphase++;
       if (!ok) break;
     } else {
       __syncthreads();
@@ -255,10 +272,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
       prep::decay_and_tiles_global<GATE_HEAD>(
           reinterpret_cast<const uint16_t *>(p.q), reinterpret_cast<const uint16_t *>(p.k), p.log_alpha,
           c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
-          decay_sh, beta_val, beta_sh, xrows, tid, !first,
-          kStageLa ? reinterpret_cast<const float *>(base + A_TB) : nullptr);
+          decay_sh, beta_val, beta_sh, xrows, tid, !first && !kStage,
+          kStage ? reinterpret_cast<const float *>(base + A_TB) : nullptr,
+          kStage ? reinterpret_cast<const uint16_t *>(base + A_TS) : nullptr,
+          kStage ? reinterpret_cast<const uint16_t *>(base + A_KH) : nullptr);
     }
-    if (kStageLa) {
+    if (kStage) {
       // the staged rows are read: rows 64..127 of [T_b | 0] back to zero, V into its tile
       fence_async_smem();
       __syncthreads();
@@ -326,6 +345,10 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
+    if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {   // T is packed: next item's q
+      const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
+      stage_q(nx.h, nx.c0);
+    }
     // zero V rows of invalid positions (tail of the sequence, pads)
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
       for (int e = tid; e < kC * 16; e += kThreadsA) {
@@ -354,9 +377,8 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     fence_after_sync();
     if (tid == 0 && item + (int)gridDim.x < nitems) {   // the T_b and V tiles are free
       const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
-      if (kStageLa) {            // next item's log_alpha
-        mbar_arrive_expect_tx(&la_bar, kLaBytes);
-        tma_load_3d(sTB, &maps.la, 0, nx.h, nx.c0, &la_bar);
+      if (kStage) {            // next item's log_alpha
+        stage_la(nx.h, nx.c0);
       } else {                   // next item's V
         mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
         tma_load_3d(sV, &vmap, 0, nx.h, nx.c0, &v_bar);
@@ -384,14 +406,19 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
       bulk_store(it + IT_WQ, base + A_QK, 64 * 128);                              // -W, block 0
       bulk_store(it + IT_WQ + 128 * 128, base + A_QK + 128 * 128, 64 * 128);      // -W, block 1
       bulk_store(it + IT_UV, base + A_KH, 64 * 256);
-      bulk_commit();       // the next item's prep waits for these reads before it rewrites the tiles
+      bulk_commit();       // the next item's tile writes wait for these reads
+      if (kStage && item + (int)gridDim.x < nitems) {   // next item's k once U_v has left
+        const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
+        bulk_wait_read();
+        stage_k(nx.h, nx.c0);
+      }
     }
     first = false;
   }
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
     mbar_wait(&v_bar, (vphase - 0) & 1, 20000);
-    if (kStageLa) mbar_wait(&la_bar, lphase & 1, 20000);
+    if (kStage) mbar_wait(&in_bar, iphase & 1, 20000);
     if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
   }
   if (tid == 0) {
@@ -769,10 +796,16 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   if (!encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
-  if (p.gate_head) maps.la = maps.v;      // not used: the head-wise gate is read per row
-  else if (!encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (p.gate_head) {
+    maps.la = maps.q = maps.k = maps.v;      // not used: with the head-wise gate the inputs are plain loads
+  } else if (!encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return cudaErrorNotSupported;
+  }
   auto intra = p.gate_head ? intra_kernel<true> : intra_kernel<false>;
   e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
