@@ -117,3 +117,25 @@ def test_head_gate_equals_broadcast_channel_gate():
                          init_state=d["init_state"])
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(f1, f2)
+
+
+@pytest.mark.parametrize("pattern", ["per_token_-4", "spikes_-200"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_head_gate_strong_decay(pattern, dtype):
+    """Head-wise gates far outside the factorised range of the tensor-core Gram (-4 per
+    token on one head: -256 per chunk; single -200 steps mid-chunk on every head): the
+    two-kernel path (exact Gram terms for the key rows past the range, every channel at
+    once) and the CUDA-core path match the oracle."""
+    inp = _case(78, [700, 64, 130], 2, 128, 128, dtype)
+    la = inp["log_alpha"].copy()
+    if pattern == "per_token_-4":
+        la[:, 0] = -4.0
+    else:
+        la[[30, 100, 357, 500], :] = -200.0
+    inp["log_alpha"] = la
+    d = dev_inputs(inp, dtype)
+    o, fs = kda.prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                        init_state=d["init_state"])
+    torch.cuda.synchronize()
+    assert kda.get_device_status() == kda.KDA_OK
+    _check(inp, dtype, o, fs)
