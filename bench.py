@@ -43,9 +43,14 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 + log_alpha fp32 + bet
 STATE_BYTES = 128 * 128 * 4                  # one (sequence, head) fp32 state
 DECODE_ACTIVE_BYTES = 2 * STATE_BYTES + 768 + 512 + 4 + 256
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-# kernels one kda_prefill launches at H = 32 on the two-kernel path: pad/cu_seqlens
-# pre-pass, chunk index, the intra kernel and the state pass
+# kernels one kda_prefill launches on the tensor-core path: pad/cu_seqlens pre-pass, chunk
+# index, the intra kernel and the state pass; chunks of 128 / 256 add one chunk index and one
+# merge kernel per doubling
 LAUNCHES_PER_PREFILL = 2 + 2 * 1
+
+
+def launches_per_prefill(chunk: int) -> int:
+    return LAUNCHES_PER_PREFILL + {64: 0, 128: 2, 256: 4}[chunk]
 PREFILL_TRAFFIC_T = 131072   # token count the recorded prefill traffic is for
 
 
@@ -60,6 +65,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="headline prefill line only")
     ap.add_argument("--only", choices=["prefill", "decode", "conv", "backward"], default=None,
                     help="time one workload only (for profiling runs)")
+    ap.add_argument("--chunk", type=int, choices=[64, 128, 256], default=64,
+                    help="prefill chunk size (128 / 256: 64-row items merged into chunk items)")
     return ap.parse_args()
 
 
@@ -208,9 +215,9 @@ def prefill_setup(T, device):
     return w, inp, host, dev
 
 
-def run_prefill(kda, dev):
+def run_prefill(kda, dev, chunk=64):
     kda.prefill(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], dev["cu_seqlens"],
-                o=dev["o"], final_state=dev["fs"])
+                o=dev["o"], final_state=dev["fs"], chunk=chunk)
 
 
 def prefill_bytes(T, H):
@@ -334,11 +341,12 @@ def main_ours(args, rank, world, device):
     clocks = ClockSampler("GPU-" + str(props.uuid))
 
     T = args.T
+    C = args.chunk
     w, inp, host, dev = prefill_setup(T, device)
     H = 32
     K, W = args.steps, args.warmup
     for _ in range(W):
-        run_prefill(kda, dev)
+        run_prefill(kda, dev, C)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -347,7 +355,7 @@ def main_ours(args, rank, world, device):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for _ in range(K):
-        run_prefill(kda, dev)
+        run_prefill(kda, dev, C)
     e.record()
     torch.cuda.synchronize()
     if world > 1:
@@ -362,9 +370,10 @@ def main_ours(args, rank, world, device):
     algo_bytes = prefill_bytes(T, H)
     achieved = algo_bytes / (ms_step / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": prefill_traffic(T),
+                "frac": achieved / pk["hbm_gbs"], "traffic": prefill_traffic(T) if C == 64 else None,
                 "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
-                "kernel": "kda prefill (whole kda_prefill call: pre-pass, chunk index, intra and state kernels)",
+                "kernel": "kda prefill (whole kda_prefill call: pre-pass, chunk index, intra and state kernels"
+                          + (")" if C == 64 else ", chunk-item merges)"),
                 "algorithmic_bytes_per_launch": algo_bytes,
                 "flops_bound_frac": (141013.0 * T * H / (ms_step / 1e3) / 1e12) / pk["bf16_tflops"]}
 
@@ -372,10 +381,10 @@ def main_ours(args, rank, world, device):
             "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "global_batch": 1, "seq_len": T, "heads": H,
-                       "d_k": 128, "d_v": 128, "chunk": 64, "state": "fp32",
+                       "d_k": 128, "d_v": 128, "chunk": C, "state": "fp32",
                        "parallelism": f"replicas{world}" if world > 1 else "none",
                        "l2": f"inputs larger than L2 ({algo_bytes / 1e9:.2f} GB per step), no flush"},
-            "roofline": roofline, "clocks": clk, "gpu_launches": LAUNCHES_PER_PREFILL * K}
+            "roofline": roofline, "clocks": clk, "gpu_launches": launches_per_prefill(C) * K}
 
     # ---- e2e through the public API with host buffers
     Ke = max(1, min(K, 3))
@@ -385,7 +394,7 @@ def main_ours(args, rank, world, device):
     def e2e_step():
         for key in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens"):
             dev[key].copy_(host[key], non_blocking=True)
-        run_prefill(kda, dev)
+        run_prefill(kda, dev, C)
         o_host.copy_(dev["o"], non_blocking=True)
         fs_host.copy_(dev["fs"], non_blocking=True)
     e2e_step()
@@ -404,7 +413,7 @@ def main_ours(args, rank, world, device):
     d2h = o_host.numel() * o_host.element_size() + fs_host.numel() * 4
     line["e2e"] = {"value": aggregate_rate(T, world, ms2 / Ke), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
-    line["gpu_launches"] += LAUNCHES_PER_PREFILL * Ke
+    line["gpu_launches"] += launches_per_prefill(C) * Ke
     del o_host, fs_host
 
     if not args.no_extras:
@@ -417,7 +426,7 @@ def main_ours(args, rank, world, device):
             if Ts >= T:
                 continue
             _, _, _, dv_ = prefill_setup(Ts, device)
-            mss = time_loop(lambda: run_prefill(kda, dv_), max(3, K), W,
+            mss = time_loop(lambda: run_prefill(kda, dv_, C), max(3, K), W,
                             flush_buf=flush if Ts <= 16384 else None)
             ach = prefill_bytes(Ts, H) / (mss / 1e3) / 1e9
             sweep[str(Ts)] = {"tokens_per_s": Ts / (mss / 1e3), "ms": mss,
@@ -431,7 +440,7 @@ def main_ours(args, rank, world, device):
         del flush
         # ---- head-wise gate (one decay per token and head), same q, k, v, beta
         devh = dict(dev, log_alpha=torch.from_numpy(gen.head_gates(w.seed, T, H)).to(device))
-        msh = time_loop(lambda: run_prefill(kda, devh), K, W)
+        msh = time_loop(lambda: run_prefill(kda, devh, C), K, W)
         hb = prefill_bytes_head_gate(T, H)
         line["prefill_head_gate"] = {
             "tokens_per_s": aggregate_rate(T, world, msh), "ms": msh,
@@ -439,6 +448,9 @@ def main_ours(args, rank, world, device):
             "log_alpha": "[N, H] fp32", "l2": "inputs larger than L2"}
         line["gpu_launches"] += LAUNCHES_PER_PREFILL * K
         del devh
+        # ---- chunk 64 / 128 / 256 on the tensor-core path, the headline workload
+        line["prefill_chunk_sweep_tc"] = bench_chunk_sweep_tc(kda, dev, T, H, K, W, pk, ms_step, C)
+        line["gpu_launches"] += sum(launches_per_prefill(c) * K for c in (64, 128, 256) if c != C)
         # ---- chunk-size sweep on the path that takes every chunk size (CUDA cores, fp32 q/k/v)
         line["prefill_chunk_sweep"] = bench_chunk_sweep(K, W, device)
         line["gpu_launches"] += 2 * 3 * K
@@ -454,6 +466,23 @@ def main_ours(args, rank, world, device):
         line["cpu_baseline"] = cpu_baseline(inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def bench_chunk_sweep_tc(kda, dev, T, H, K, W, pk, ms_headline, C_headline):
+    """The headline prefill (bf16, B=1, H=32, d=128) at chunk 64, 128 and 256 on the
+    tensor-core path: 128 / 256 merge the 64-row items into chunk items (one or two extra
+    passes over the items) and halve / quarter the serial steps of the state pass."""
+    out = {"workload": f"prefill_T{T}_H{H}_d128_bf16", "path": "tensor cores (tcgen05)",
+           "l2": "inputs larger than L2"}
+    for c in (64, 128, 256):
+        ms = ms_headline if c == C_headline else time_loop(lambda: run_prefill(kda, dev, c), K, W)
+        ach = prefill_bytes(T, H) / (ms / 1e3) / 1e9
+        out[str(c)] = {"ms": ms, "tokens_per_s": T / (ms / 1e3), "hbm_frac": ach / pk["hbm_gbs"],
+                       "state_steps_per_sequence": -(-T // c)}
+    st = kda.get_device_status()
+    if st != kda.KDA_OK:
+        raise RuntimeError("device status after the tensor-core chunk sweep: " + kda.status_string(st))
+    return out
 
 
 def bench_chunk_sweep(K, W, device, T=16384):

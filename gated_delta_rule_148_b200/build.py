@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkda.so")
 SOURCES = ["kda_api.cu", "kda_decode.cu", "kda_prefill_simt.cu", "kda_prefill_tc.cu",
            "kda_noalloc.cu", "kda_prefill_split.cu", "kda_conv.cu",
-           "kda_backward.cu"]
+           "kda_backward.cu", "kda_prefill_bigchunk.cu"]
 HEADERS = ["kda_internal.cuh", "kda_tc.cuh", "kda_tril_inv.cuh", "kda_chunk_prep.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -106,8 +106,15 @@ bool split_eligible(const kda_prefill_args *a) {
          a->total_tokens >= 0 && a->H >= 1;
 }
 
+// Chunks of 128 or 256 rows: only on the tensor-core path (bf16, d_k = d_v = 128).
+bool bigchunk_eligible(const kda_prefill_args *a) {
+  return a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 && (a->chunk == 128 || a->chunk == 256) &&
+         a->num_seqs > 0 && a->total_tokens >= 0 && a->H >= 1;
+}
+
 size_t kda_prefill_workspace_size(const kda_prefill_args *a) {
   if (!a) return 0;
+  if (bigchunk_eligible(a)) return prefill_bigchunk_workspace(a->total_tokens, a->num_seqs, a->H, a->chunk);
   if (split_eligible(a)) return prefill_split_workspace(a->total_tokens, a->num_seqs, a->H);
   return spans_bytes(a->num_seqs);
 }
@@ -120,7 +127,9 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   if (!head_dim_ok(a->dk) || !head_dim_ok(a->dv)) return KDA_ERR_UNSUPPORTED;
   int chunk = a->chunk;
   if (chunk == 0) chunk = (a->dtype == KDA_BF16) ? 64 : 16;
-  if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+  const bool big = chunk == 128 || chunk == 256;
+  if (chunk != 16 && chunk != 32 && chunk != 64 && !big) return KDA_ERR_UNSUPPORTED;
+  if (big && (a->dtype != KDA_BF16 || a->dk != 128 || a->dv != 128)) return KDA_ERR_UNSUPPORTED;
   if (a->gate != KDA_GATE_CHANNEL && a->gate != KDA_GATE_HEAD) return KDA_ERR_INVALID_ARG;
   const bool gate_head = a->gate == KDA_GATE_HEAD;
   if (a->num_seqs == 0) return a->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
@@ -189,13 +198,18 @@ kda_status kda_prefill(const kda_prefill_args *a, void *stream) {
   p.spans = nullptr;
   // Two-kernel path when the workspace holds the per-chunk items; otherwise the
   // fused tensor-core kernel (or the CUDA-core kernel for other shapes).
+  // Chunks of 128 / 256 rows exist only on the workspace-backed tensor-core path.
+  if (big && (!a->workspace || a->workspace_bytes < prefill_bigchunk_workspace(a->total_tokens, a->num_seqs,
+                                                                                 a->H, chunk)))
+    return KDA_ERR_UNSUPPORTED;
   const bool split = prefill_split_supported(p, bf16) && a->workspace &&
                      a->workspace_bytes >= prefill_split_workspace(a->total_tokens, a->num_seqs, a->H);
-  SeqSpan *spans = (split || a->pad_mask) ? static_cast<SeqSpan *>(a->workspace) : nullptr;
+  SeqSpan *spans = (big || split || a->pad_mask) ? static_cast<SeqSpan *>(a->workspace) : nullptr;
   if (launch_prefill_prepass(p, bf16, spans, s) != cudaSuccess) return KDA_ERR_CUDA;
   p.spans = spans;
   cudaError_t e;
-  if (split) e = launch_prefill_split(p, spans, a->workspace, s);
+  if (big) e = launch_prefill_bigchunk(p, spans, a->workspace, s);
+  else if (split) e = launch_prefill_split(p, spans, a->workspace, s);
   else if (prefill_tc_supported(p, bf16)) e = launch_prefill_tc(p, s);
   else e = launch_prefill_simt(p, bf16, s);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;

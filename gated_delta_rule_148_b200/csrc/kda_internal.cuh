@@ -95,6 +95,13 @@ bool prefill_tc_supported(const PrefillParams &p, bool bf16);
 bool prefill_split_supported(const PrefillParams &p, bool bf16);
 size_t prefill_split_workspace(int N, int B, int H);
 cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
+// The two-kernel path's chunk index and intra kernel alone (64-row items of every chunk and head).
+cudaError_t launch_split_items(const PrefillParams &p, const SeqSpan *spans, int *cbase,
+                               unsigned char *items, cudaStream_t s);
+// Chunks of 128 or 256 rows: 64-row items merged into chunk items, then the state pass.
+bool prefill_bigchunk_supported(const PrefillParams &p, bool bf16);
+size_t prefill_bigchunk_workspace(int N, int B, int H, int chunk);
+cudaError_t launch_prefill_bigchunk(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s);
 size_t backward_workspace(int N, int H, int dk, int dv);

@@ -782,13 +782,11 @@ int num_sms() {
 
 }  // namespace
 
-// spans: B entries already written by the pre-pass; ws: workspace base.
-cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s) {
+// The chunk index and the intra kernel: cbase[b] (b <= num_seqs) = 64-row chunks of the
+// sequences before b; items = one 74 752-byte item per (64-row chunk, head).
+cudaError_t launch_split_items(const PrefillParams &p, const SeqSpan *spans, int *cbase,
+                               unsigned char *items, cudaStream_t s) {
   using namespace split;
-  if (p.num_seqs == 0) return cudaSuccess;
-  unsigned char *w = static_cast<unsigned char *>(ws);
-  int *cbase = reinterpret_cast<int *>(w + ws_cbase_off(p.num_seqs));
-  unsigned char *items = w + ws_items_off(p.num_seqs);
   chunk_index_kernel<<<1, 1024, 0, s>>>(p, spans, cbase);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -809,6 +807,22 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   auto intra = p.gate_head ? intra_kernel<true> : intra_kernel<false>;
   e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
   if (e != cudaSuccess) return e;
+  const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
+  if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+  const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
+  intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, maps, spans, cbase, items, 0, p.H);
+  return cudaGetLastError();
+}
+
+// spans: B entries already written by the pre-pass; ws: workspace base.
+cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s) {
+  using namespace split;
+  if (p.num_seqs == 0) return cudaSuccess;
+  unsigned char *w = static_cast<unsigned char *>(ws);
+  int *cbase = reinterpret_cast<int *>(w + ws_cbase_off(p.num_seqs));
+  unsigned char *items = w + ws_items_off(p.num_seqs);
+  cudaError_t e = launch_split_items(p, spans, cbase, items, s);
+  if (e != cudaSuccess) return e;
   // 32-column state slices while they fit one wave (more independent chains, shorter products);
   // 64-column slices once there are more chains than SMs (less work per column in total).
   const bool narrow = (size_t)p.num_seqs * p.H * (p.dv / 32) <= (size_t)num_sms();
@@ -816,11 +830,6 @@ cudaError_t launch_prefill_split(const PrefillParams &p, SeqSpan *spans, void *w
   const uint32_t smem_b = narrow ? StateTiles<32>::SMEM : StateTiles<64>::SMEM;
   e = cudaFuncSetAttribute(state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
   if (e != cudaSuccess) return e;
-  const size_t items_max = max_chunks(p.N, p.num_seqs) * (size_t)p.H;
-  if (items_max > 0x7FFFFFFFull) return cudaErrorInvalidValue;
-  const size_t gridA = items_max < (size_t)(2 * num_sms()) ? items_max : (size_t)(2 * num_sms());
-  intra<<<(unsigned)gridA, kThreadsA, A_SMEM, s>>>(p, maps, spans, cbase, items, 0, p.H);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const unsigned gridB = (unsigned)p.num_seqs * p.H * (p.dv / (narrow ? 32 : 64));
   state<<<gridB, kThreadsB, smem_b, s>>>(p, spans, cbase, items, 0, p.H);
   return cudaGetLastError();

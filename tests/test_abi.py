@@ -110,6 +110,9 @@ def _call(a):
     (lambda a: setattr(a, "dk", 96), kda.KDA_ERR_UNSUPPORTED),
     (lambda a: setattr(a, "dv", 256), kda.KDA_ERR_UNSUPPORTED),
     (lambda a: setattr(a, "chunk", 48), kda.KDA_ERR_UNSUPPORTED),
+    (lambda a: setattr(a, "chunk", 128), kda.KDA_ERR_UNSUPPORTED),            # d = 64
+    (lambda a: (setattr(a, "chunk", 256), setattr(a, "dtype", kda.KDA_F32)), kda.KDA_ERR_UNSUPPORTED),
+    (lambda a: setattr(a, "chunk", 512), kda.KDA_ERR_UNSUPPORTED),
     (lambda a: setattr(a, "q", None), kda.KDA_ERR_INVALID_ARG),
     (lambda a: setattr(a, "o", None), kda.KDA_ERR_INVALID_ARG),
     (lambda a: setattr(a, "cu_seqlens", None), kda.KDA_ERR_INVALID_ARG),
@@ -124,7 +127,8 @@ def _call(a):
                 setattr(a, "log_alpha", a.log_alpha + 2)), kda.KDA_ERR_INVALID_ARG),
     (lambda a: (setattr(a, "gate", kda.KDA_GATE_HEAD),                        # [N, H] gate
                 setattr(a, "o", a.log_alpha + N * H * 4 - 64)), kda.KDA_ERR_INVALID_ARG),
-], ids=["dtype", "H", "num_seqs", "dk", "dv", "chunk", "null_q", "null_o", "null_cu",
+], ids=["dtype", "H", "num_seqs", "dk", "dv", "chunk", "chunk128_d64", "chunk256_f32",
+        "chunk512", "null_q", "null_o", "null_cu",
         "misaligned_q", "misaligned_la", "o_overlaps_k", "mask_without_ws", "state_aliases_q",
         "tokens_without_seqs", "gate_value", "head_gate_misaligned", "o_overlaps_head_gate"])
 def test_prefill_rejects_bad_arguments(mutate, expect):
@@ -146,6 +150,25 @@ def test_workspace_size():
     n = kda.load().kda_prefill_workspace_size(ctypes.byref(a))
     assert n >= 8 * 16 and n % 256 == 0
     assert kda.load().kda_prefill_workspace_size(None) == 0
+
+
+def test_workspace_size_by_chunk():
+    """bf16, d = 128: chunk 64 needs the 64-row items (74 752 bytes per chunk and head);
+    chunks of 128 / 256 also need the merged items (164 352 and 360 960 bytes)."""
+    a = kda.PrefillArgs()
+    a.dtype, a.num_seqs, a.total_tokens, a.H, a.dk, a.dv = kda.KDA_BF16, 1, 131072, 32, 128, 128
+    size = {}
+    for c in (64, 128, 256):
+        a.chunk = c
+        size[c] = kda.load().kda_prefill_workspace_size(ctypes.byref(a))
+    items64 = (131072 // 64 + 1) * 32 * 74752
+    items128 = (131072 // 128 + 1) * 32 * 164352
+    items256 = (131072 // 256 + 1) * 32 * 360960
+    assert items64 < size[64] < items64 + 4096
+    assert items64 + items128 < size[128] < items64 + items128 + 8192
+    assert max(items64, items256) + items128 < size[256] < max(items64, items256) + items128 + 8192
+    a.dtype = kda.KDA_F32
+    assert kda.load().kda_prefill_workspace_size(ctypes.byref(a)) < 4096   # no tensor-core path
 
 
 def _good_decode():
