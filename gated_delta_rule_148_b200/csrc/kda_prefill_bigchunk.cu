@@ -162,13 +162,41 @@ struct MergeSmem<128> {  // -W_b, Q G_b, K~_a, -W_a, U_v,a, E
   static constexpr uint32_t SMEM = 196608 + 1024;
 };
 
-__device__ __forceinline__ void copy16(unsigned char *dst, const unsigned char *src, uint32_t bytes, int tid) {
-  for (uint32_t o = (uint32_t)tid * 16; o < bytes; o += kThreadsM * 16)
-    *reinterpret_cast<uint4 *>(dst + o) = *reinterpret_cast<const uint4 *>(src + o);
-}
-__device__ __forceinline__ void zero16(unsigned char *dst, uint32_t bytes, int tid) {
-  for (uint32_t o = (uint32_t)tid * 16; o < bytes; o += kThreadsM * 16)
-    *reinterpret_cast<uint4 *>(dst + o) = make_uint4(0u, 0u, 0u, 0u);
+// Byte ranges copied (or zeroed, src == nullptr) from the sub-chunk items into the merged
+// item.  Every thread keeps eight 16-byte loads in flight before it stores them.
+struct Seg {
+  unsigned char *dst;
+  const unsigned char *src;
+  uint32_t bytes;
+};
+constexpr int kMaxSegs = 24;
+
+__device__ __forceinline__ void copy_segments(const Seg *segs, int n, int tid) {
+  uint32_t total = 0;
+  for (int i = 0; i < n; ++i) total += segs[i].bytes >> 4;
+  int sgi = 0;               // this thread's indices only grow: a cursor over the segments
+  uint32_t seg0 = 0, seg1 = segs[0].bytes >> 4;
+  for (uint32_t first = (uint32_t)tid; first < total; first += 8 * kThreadsM) {
+    uint4 v[8];
+    unsigned char *dst[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      dst[u] = nullptr;
+      const uint32_t idx = first + (uint32_t)u * kThreadsM;
+      if (idx >= total) continue;
+      while (idx >= seg1) {
+        seg0 = seg1;
+        seg1 += segs[++sgi].bytes >> 4;
+      }
+      const uint32_t off = (idx - seg0) * 16;
+      dst[u] = segs[sgi].dst + off;
+      v[u] = segs[sgi].src ? __ldg(reinterpret_cast<const uint4 *>(segs[sgi].src + off))
+                           : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (dst[u]) *reinterpret_cast<uint4 *>(dst[u]) = v[u];
+  }
 }
 
 __device__ __forceinline__ void unpack8(uint4 w, float *f) {
@@ -253,77 +281,84 @@ merge_kernel(PrefillParams p, const SeqSpan *spans, const int *cb_in, const int 
     gam_b[tid] = has_b ? reinterpret_cast<const float *>(xb + IN::GC)[tid] : 1.f;
   }
 
-  // ---- parts that are copies of a sub-chunk's parts (or zero rows)
-  if constexpr (c == 64) {
-    for (int kb = 0; kb < 2; ++kb) {
-      copy16(o + O::W(0) + kb * 16384, xa + I64_WQ + kb * 16384, 8192, tid);            // -W_a
-      copy16(o + O::Q(0) + kb * 16384, xa + I64_WQ + kb * 16384 + 8192, 8192, tid);     // Q G_a
-      copy16(o + O::UV + kb * 16384, xa + I64_UV + kb * 8192, 8192, tid);               // U_v,a
-    }
-    copy16(o + O::M(0, 0), xa + I64_M, 8192, tid);                                       // M_a
-    zero16(o + O::M(0, 0) + 16384, 8192, tid);                                           // upper right
-    if (has_b) {
-      for (int kb = 0; kb < 2; ++kb)
-        copy16(o + O::K(0) + kb * 16384 + 8192, xb + I64_KT + kb * 8192, 8192, tid);    // K~_b
-      copy16(o + O::M(0, 0) + 16384 + 8192, xb + I64_M, 8192, tid);                     // M_b
-    } else {
-      for (int kb = 0; kb < 2; ++kb) {
-        zero16(o + O::W(0) + kb * 16384 + 8192, 8192, tid);
-        zero16(o + O::Q(0) + kb * 16384 + 8192, 8192, tid);
-        copy16(o + O::K(0) + kb * 16384, xa + I64_KT + kb * 8192, 8192, tid);
-        zero16(o + O::K(0) + kb * 16384 + 8192, 8192, tid);
-        zero16(o + O::UV + kb * 16384 + 8192, 8192, tid);
-      }
-      zero16(o + O::M(0, 0) + 8192, 8192, tid);
-      zero16(o + O::M(0, 0) + 16384 + 8192, 8192, tid);
-    }
-  } else {
-    copy16(o + O::W(0), xa + Item<128>::W(0), kPart, tid);
-    copy16(o + O::Q(0), xa + Item<128>::Q(0), kPart, tid);
-    copy16(o + O::M(0, 0), xa + Item<128>::M(0, 0), kPart, tid);
-    for (int kb = 0; kb < 2; ++kb)
-      copy16(o + O::UV + kb * 32768, xa + Item<128>::UV + kb * 16384, 16384, tid);
-    if (has_b) {
-      copy16(o + O::K(1), xb + Item<128>::K(0), kPart, tid);
-      copy16(o + O::M(1, 1), xb + Item<128>::M(0, 0), kPart, tid);
-    } else {
-      zero16(o + O::W(1), kPart, tid);
-      zero16(o + O::Q(1), kPart, tid);
-      copy16(o + O::K(0), xa + Item<128>::K(0), kPart, tid);
-      zero16(o + O::K(1), kPart, tid);
-      zero16(o + O::M(1, 0), kPart, tid);
-      zero16(o + O::M(1, 1), kPart, tid);
-      for (int kb = 0; kb < 2; ++kb) zero16(o + O::UV + kb * 32768 + 16384, 16384, tid);
-    }
-  }
-  __syncthreads();
-  if (tid < kDK) reinterpret_cast<float *>(o + O::GC)[tid] = gam_a[tid] * gam_b[tid];
-  if (!has_b) return;
-
-  // ---- the merged rows: two product groups
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char *base = smem_raw + pad;
   const int warp = tid >> 5, r = (warp & 3) * 32 + (tid & 31), wg = warp >> 2;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  if (warp == 0) tmem_alloc(&tmem_base_sh, 256);
-  if (tid == 0) {
-    mbar_init(&load_bar, 1);
-    mbar_init(&mma_bar, 1);
-    mbar_arrive_expect_tx(&load_bar, SM::LOAD_TX);
-    if constexpr (c == 64) {
-      bulk_load(base + SM::WQB, xb + I64_WQ, 32768, &load_bar);
-      bulk_load(base + SM::KTA, xa + I64_KT, 16384, &load_bar);
-      bulk_load(base + SM::WA, xa + I64_WQ, 8192, &load_bar);
-      bulk_load(base + SM::WA + 16384, xa + I64_WQ + 16384, 8192, &load_bar);
-      bulk_load(base + SM::UVA, xa + I64_UV, 16384, &load_bar);
-    } else {
-      bulk_load(base + SM::WB, xb + Item<128>::W(0), kPart, &load_bar);
-      bulk_load(base + SM::QB, xb + Item<128>::Q(0), kPart, &load_bar);
-      bulk_load(base + SM::KA, xa + Item<128>::K(0), kPart, &load_bar);
-      bulk_load(base + SM::WA, xa + Item<128>::W(0), kPart, &load_bar);
-      bulk_load(base + SM::UVA, xa + Item<128>::UV, kPart, &load_bar);
+  if (has_b) {
+    // the operand tiles of the two product groups load while the copies below run
+    if (warp == 0) tmem_alloc(&tmem_base_sh, 256);
+    if (tid == 0) {
+      mbar_init(&load_bar, 1);
+      mbar_init(&mma_bar, 1);
+      mbar_arrive_expect_tx(&load_bar, SM::LOAD_TX);
+      if constexpr (c == 64) {
+        bulk_load(base + SM::WQB, xb + I64_WQ, 32768, &load_bar);
+        bulk_load(base + SM::KTA, xa + I64_KT, 16384, &load_bar);
+        bulk_load(base + SM::WA, xa + I64_WQ, 8192, &load_bar);
+        bulk_load(base + SM::WA + 16384, xa + I64_WQ + 16384, 8192, &load_bar);
+        bulk_load(base + SM::UVA, xa + I64_UV, 16384, &load_bar);
+      } else {
+        bulk_load(base + SM::WB, xb + Item<128>::W(0), kPart, &load_bar);
+        bulk_load(base + SM::QB, xb + Item<128>::Q(0), kPart, &load_bar);
+        bulk_load(base + SM::KA, xa + Item<128>::K(0), kPart, &load_bar);
+        bulk_load(base + SM::WA, xa + Item<128>::W(0), kPart, &load_bar);
+        bulk_load(base + SM::UVA, xa + Item<128>::UV, kPart, &load_bar);
+      }
     }
   }
+
+  // ---- parts that are copies of a sub-chunk's parts (or zero rows)
+  Seg sg[kMaxSegs];
+  int n = 0;
+  auto add = [&](unsigned char *dst, const unsigned char *src, uint32_t bytes) { sg[n++] = Seg{dst, src, bytes}; };
+  if constexpr (c == 64) {
+    for (int kb = 0; kb < 2; ++kb) {
+      add(o + O::W(0) + kb * 16384, xa + I64_WQ + kb * 16384, 8192);            // -W_a
+      add(o + O::Q(0) + kb * 16384, xa + I64_WQ + kb * 16384 + 8192, 8192);     // Q G_a
+      add(o + O::UV + kb * 16384, xa + I64_UV + kb * 8192, 8192);               // U_v,a
+    }
+    add(o + O::M(0, 0), xa + I64_M, 8192);                                       // M_a
+    add(o + O::M(0, 0) + 16384, nullptr, 8192);                                  // upper right
+    if (has_b) {
+      for (int kb = 0; kb < 2; ++kb)
+        add(o + O::K(0) + kb * 16384 + 8192, xb + I64_KT + kb * 8192, 8192);    // K~_b
+      add(o + O::M(0, 0) + 16384 + 8192, xb + I64_M, 8192);                     // M_b
+    } else {
+      for (int kb = 0; kb < 2; ++kb) {
+        add(o + O::W(0) + kb * 16384 + 8192, nullptr, 8192);
+        add(o + O::Q(0) + kb * 16384 + 8192, nullptr, 8192);
+        add(o + O::K(0) + kb * 16384, xa + I64_KT + kb * 8192, 8192);
+        add(o + O::K(0) + kb * 16384 + 8192, nullptr, 8192);
+        add(o + O::UV + kb * 16384 + 8192, nullptr, 8192);
+      }
+      add(o + O::M(0, 0) + 8192, nullptr, 8192);
+      add(o + O::M(0, 0) + 16384 + 8192, nullptr, 8192);
+    }
+  } else {
+    add(o + O::W(0), xa + Item<128>::W(0), kPart);
+    add(o + O::Q(0), xa + Item<128>::Q(0), kPart);
+    add(o + O::M(0, 0), xa + Item<128>::M(0, 0), kPart);
+    for (int kb = 0; kb < 2; ++kb)
+      add(o + O::UV + kb * 32768, xa + Item<128>::UV + kb * 16384, 16384);
+    if (has_b) {
+      add(o + O::K(1), xb + Item<128>::K(0), kPart);
+      add(o + O::M(1, 1), xb + Item<128>::M(0, 0), kPart);
+    } else {
+      add(o + O::W(1), nullptr, kPart);
+      add(o + O::Q(1), nullptr, kPart);
+      add(o + O::K(0), xa + Item<128>::K(0), kPart);
+      add(o + O::K(1), nullptr, kPart);
+      add(o + O::M(1, 0), nullptr, kPart);
+      add(o + O::M(1, 1), nullptr, kPart);
+      for (int kb = 0; kb < 2; ++kb) add(o + O::UV + kb * 32768 + 16384, nullptr, 16384);
+    }
+  }
+  copy_segments(sg, n, tid);
+  if (tid < kDK) reinterpret_cast<float *>(o + O::GC)[tid] = gam_a[tid] * gam_b[tid];
+  if (!has_b) return;
+
+  // ---- the merged rows: two product groups
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -469,15 +504,22 @@ constexpr int kComputeThreads = 256;
 constexpr int kThreadsS = kComputeThreads + 32;
 constexpr int NS = 32, kW = 16;
 
+// Ring parts per chunk, in the order they are read: the 2P row blocks of [-W ; Q G] (first
+// product group), the slice's 64-column U_v block with e^{g_C} behind it (the decay of S and
+// the U conversion), the P row blocks of K~ and the NM blocks of M (second group).  A chunk's
+// first-group tiles take the slots its predecessor's last tiles and first-group tiles
+// release, so they load a whole chunk step ahead.
 template <int C>
 struct Ring {
   static constexpr int P = C / 128;
-  static constexpr int NSLOT = C == 128 ? 6 : 5;
-  static constexpr uint32_t UVB = NSLOT * kPart;             // this slice's 64-column U_v block
-  static constexpr uint32_t GCB = UVB + (uint32_t)C * 128;    // e^{g_C}
-  static constexpr uint32_t SB = (GCB + 512 + 1023) / 1024 * 1024;   // S: 128 rows x 64 B
+  static constexpr int NSLOT = 6;
+  static constexpr int STEP_PARTS = 1 + Item<C>::PARTS;
+  static constexpr uint32_t SLOT = kPart + 1024;             // 32 KB tile (or U_v block + e^{g_C})
+  static constexpr uint32_t GC_IN_SLOT = (uint32_t)C * 128;
+  static constexpr uint32_t SB = NSLOT * SLOT;               // S: 128 rows x 64 B
   static constexpr uint32_t UB = SB + 128 * 64;              // U: C rows x 64 B
   static constexpr uint32_t SMEM = UB + (uint32_t)C * 64 + 1024;
+  static_assert(GC_IN_SLOT + 512 <= SLOT, "U_v block and e^{g_C} share a slot");
   static constexpr uint32_t TM_S = 0, TM_D1 = NS;            // D1 buffers of 2P blocks of NS columns
   static constexpr uint32_t TM_COLS = C == 128 ? 256 : 512;
   static_assert(TM_D1 + 2 * 2 * P * NS <= TM_COLS, "tensor memory");
@@ -507,10 +549,10 @@ __global__ void __launch_bounds__(kThreadsS, 1)
 state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsigned char *items) {
   using R = Ring<C>;
   using IT = Item<C>;
-  constexpr int P = R::P, NSLOT = R::NSLOT, PARTS = IT::PARTS;
+  constexpr int P = R::P, NSLOT = R::NSLOT, PARTS = IT::PARTS, SP = R::STEP_PARTS;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ __align__(8) uint64_t mma_bar, uv_full, uv_free;
+  __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t full_bar[NSLOT], free_bar[NSLOT];
   __shared__ int err_sh;
 
@@ -536,8 +578,6 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   if (warp == 0) tmem_alloc(&tmem_base_sh, R::TM_COLS);
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
-    mbar_init(&uv_full, 1);
-    mbar_init(&uv_free, 1);
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&free_bar[i], 1);
@@ -550,23 +590,14 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
   const uint32_t tm = tmem_base_sh;
 
   if (warp == kComputeThreads / 32) {
-    // ---------------- producer: U_v block and e^{g_C} per chunk, item parts through the ring
+    // ---------------- producer: every part of every chunk through the ring, in reading order
     if ((tid & 31) == 0 && !(p.fault & FAULT_STARVE_STATE_LOADS)) {
-      int t = 0, jl = -1;
+      int t = 0;
       bool stop = false;
       for (int j = 0; j < nch && !stop; ++j) {
         const unsigned char *it = items + ((size_t)(cb + j) * H + h) * IT::BYTES;
-        if (j >= 1 && !mbar_wait(&uv_free, (j - 1) & 1, p.wait_cycles)) {
-          note_timeout(p.site, 15);
-          atomicOr(p.err, ERR_BIT_TIMEOUT);
-          break;
-        }
-        if (*reinterpret_cast<volatile int *>(&err_sh)) break;
-        mbar_arrive_expect_tx(&uv_full, (uint32_t)C * 128 + 512);
-        bulk_load(base + R::UVB, it + IT::UV + (uint32_t)uv_blk * C * 128, (uint32_t)C * 128, &uv_full);
-        bulk_load(base + R::GCB, it + IT::GC, 512, &uv_full);
-        jl = j;
-        for (int q = 0; q < PARTS; ++q, ++t) {
+        for (int qq = 0; qq < SP; ++qq, ++t) {
+          const int q = qq < 2 * P ? qq : (qq == 2 * P ? -1 : qq - 1);   // item tile, or -1: U_v
           const int slot = t % NSLOT, use = t / NSLOT;
           if (use >= 1 && !mbar_wait(&free_bar[slot], (use - 1) & 1, p.wait_cycles)) {
             note_timeout(p.site, 14);
@@ -574,8 +605,16 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&full_bar[slot], kPart);
-          bulk_load(base + (uint32_t)slot * kPart, it + (uint32_t)q * kPart, kPart, &full_bar[slot]);
+          if (*reinterpret_cast<volatile int *>(&err_sh)) { stop = true; break; }
+          unsigned char *dst = base + (uint32_t)slot * R::SLOT;
+          if (q < 0) {
+            mbar_arrive_expect_tx(&full_bar[slot], R::GC_IN_SLOT + 512);
+            bulk_load(dst, it + IT::UV + (uint32_t)uv_blk * C * 128, R::GC_IN_SLOT, &full_bar[slot]);
+            bulk_load(dst + R::GC_IN_SLOT, it + IT::GC, 512, &full_bar[slot]);
+          } else {
+            mbar_arrive_expect_tx(&full_bar[slot], kPart);
+            bulk_load(dst, it + (uint32_t)q * kPart, kPart, &full_bar[slot]);
+          }
         }
       }
       // every load issued here has landed before the CTA exits
@@ -583,7 +622,6 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
         const int tt = t - q;
         mbar_wait(&full_bar[tt % NSLOT], (tt / NSLOT) & 1, p.wait_cycles);
       }
-      if (jl >= 0) mbar_wait(&uv_full, jl & 1, p.wait_cycles);
     }
   } else {
     // ---------------- compute warps
@@ -603,48 +641,58 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
     auto slot_ready = [&](int t) -> bool {
       return mbar_wait(&full_bar[t % NSLOT], (t / NSLOT) & 1, p.wait_cycles);
     };
+    auto slot_ptr = [&](int t) -> unsigned char * { return base + (uint32_t)(t % NSLOT) * R::SLOT; };
+
+    // ring part of item tile q of chunk j, and of chunk j's U_v block
+    auto tile_part = [&](int j, int q) { return j * SP + (q < 2 * P ? q : q + 1); };
+    auto uv_part = [&](int j) { return j * SP + 2 * P; };
+    float sv[kW];            // this thread's slice of S at the start of the current chunk
 
     auto begin_chunk = [&](int j) {
-      if (!mbar_wait(&uv_full, j & 1, p.wait_cycles)) { err_sh = 1; note_timeout(p.site, 16); }
-      float v[kW];
-      tmem_ld16(tm + my_cols + R::TM_S, v);
-      store_row32(base + R::SB, lr, wg * (kW / 8), v);
+      tmem_ld16(tm + my_cols + R::TM_S, sv);
+      store_row32(base + R::SB, lr, wg * (kW / 8), sv);
       fence_async_smem();
       fence_before_sync();
       compute_sync();
       if (tid == 0) {
         fence_after_sync();
         const uint32_t id = idesc_bf16(128, NS, 0, 1);
-        const int t0 = j * PARTS;
         bool good = !err_sh;
         for (int i = 0; i < 2 * P && good; ++i) {
-          if (!slot_ready(t0 + i)) { good = false; err_sh = 1; note_timeout(p.site, 11); break; }
-          const uint64_t a0 = desc_kmajor(smem_u32(base + (uint32_t)((t0 + i) % NSLOT) * kPart), 128, 0, 0);
+          const int t = tile_part(j, i);
+          if (!slot_ready(t)) { good = false; err_sh = 1; note_timeout(p.site, 11); break; }
+          const uint64_t a0 = desc_kmajor(smem_u32(slot_ptr(t)), 128, 0, 0);
           const uint32_t d = tm + R::TM_D1 + (uint32_t)(((j & 1) * 2 * P + i) * NS);
 #pragma unroll
           for (int s = 0; s < 8; ++s)
             mma_bf16(d, a0 + (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4), desc32(sSB, s), id, s > 0);
         }
-        for (int i = 0; i < 2 * P; ++i) mma_commit(&free_bar[(t0 + i) % NSLOT]);
+        for (int i = 0; i < 2 * P; ++i) mma_commit(&free_bar[tile_part(j, i) % NSLOT]);
         mma_commit(&mma_bar);
         ++commits;
       }
-      const float decay = reinterpret_cast<const float *>(base + R::GCB)[lr];
-#pragma unroll
-      for (int jj = 0; jj < kW; ++jj) v[jj] *= decay;
-      tmem_st16(tm + my_cols + R::TM_S, v);
     };
 
     if (nch > 0) begin_chunk(0);
     for (int j = 0; j < nch; ++j) {
       const int c0 = sp.begin + j * C;
       const uint32_t d1 = R::TM_D1 + (uint32_t)((j & 1) * 2 * P * NS);
+      // U_v rows of this thread and e^{g_C}: S is scaled in TMEM while the first group runs
+      // (the group reads the bf16 copy)
+      if (!slot_ready(uv_part(j))) { err_sh = 1; note_timeout(p.site, 16); }
+      unsigned char *uvs = slot_ptr(uv_part(j));
       uint4 uv[P][kW / 8];
 #pragma unroll
       for (int i = 0; i < P; ++i)
 #pragma unroll
         for (int q = 0; q < kW / 8; ++q)
-          uv[i][q] = *reinterpret_cast<const uint4 *>(base + R::UVB + row_tile_chunk(128 * i + lr, 0, uv_c0 + q, C));
+          uv[i][q] = *reinterpret_cast<const uint4 *>(uvs + row_tile_chunk(128 * i + lr, 0, uv_c0 + q, C));
+      {
+        const float decay = reinterpret_cast<const float *>(uvs + R::GC_IN_SLOT)[lr];
+#pragma unroll
+        for (int jj = 0; jj < kW; ++jj) sv[jj] *= decay;
+        tmem_st16(tm + my_cols + R::TM_S, sv);
+      }
       // ---- U = U_v - W S -> bf16 operand
       if (!mbar_wait(&mma_bar, phase & 1, p.wait_cycles)) { err_sh = 1; note_timeout(p.site, 12); }
       phase++;
@@ -666,28 +714,27 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
       fence_async_smem();
       fence_before_sync();
       compute_sync();
-      if (tid == 0) mbar_arrive(&uv_free);     // the U_v block and e^{g_C} of chunk j are read
+      if (tid == 0) mbar_arrive(&free_bar[uv_part(j) % NSLOT]);   // U_v block and e^{g_C} of chunk j read
       if (*reinterpret_cast<volatile int *>(&err_sh)) { ok = false; break; }
       // ---- S += K~^T U;  O += M U
       if (tid == 0) {
         fence_after_sync();
         const uint32_t ids = idesc_bf16(128, NS, 1, 1);
         const uint32_t ido = idesc_bf16(128, NS, 0, 1);
-        const int t0 = j * PARTS;
         bool good = true;
         for (int i = 0; i < P && good; ++i) {
-          const int t = t0 + 2 * P + i;
+          const int t = tile_part(j, 2 * P + i);
           if (!slot_ready(t)) { good = false; break; }
-          const uint64_t as = desc_mnmajor(smem_u32(base + (uint32_t)(t % NSLOT) * kPart), 128, 0, 0);
+          const uint64_t as = desc_mnmajor(smem_u32(slot_ptr(t)), 128, 0, 0);
 #pragma unroll
           for (int s = 0; s < 8; ++s)
             mma_bf16(tm + R::TM_S, as + (uint64_t)((16 * s * 128) >> 4), desc32(sUB, 8 * i + s), ids, 1);
         }
         for (int i = 0; i < P && good; ++i)
           for (int k = 0; k <= i && good; ++k) {
-            const int t = t0 + 3 * P + i * (i + 1) / 2 + k;
+            const int t = tile_part(j, 3 * P + i * (i + 1) / 2 + k);
             if (!slot_ready(t)) { good = false; break; }
-            const uint64_t a0 = desc_kmajor(smem_u32(base + (uint32_t)(t % NSLOT) * kPart), 128, 0, 0);
+            const uint64_t a0 = desc_kmajor(smem_u32(slot_ptr(t)), 128, 0, 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
               mma_bf16(tm + d1 + (uint32_t)((P + i) * NS),
@@ -695,7 +742,7 @@ state_kernel(PrefillParams p, const SeqSpan *spans, const int *cbase, const unsi
                        desc32(sUB, 8 * k + s), ido, 1);
           }
         if (!good) { err_sh = 1; note_timeout(p.site, 11); }
-        for (int q = 2 * P; q < PARTS; ++q) mma_commit(&free_bar[(t0 + q) % NSLOT]);
+        for (int q = 2 * P; q < PARTS; ++q) mma_commit(&free_bar[tile_part(j, q) % NSLOT]);
         mma_commit(&mma_bar);
         ++commits;
       }
