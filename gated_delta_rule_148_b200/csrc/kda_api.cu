@@ -304,8 +304,8 @@ kda_status kda_short_conv(const kda_conv_args *a, void *stream) {
 }
 
 size_t kda_prefill_backward_workspace_size(const kda_backward_args *a) {
-  if (!a || a->total_tokens < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0) return 0;
-  return backward_workspace(a->total_tokens, a->H, a->dk, a->dv);
+  if (!a || a->total_tokens < 0 || a->num_seqs < 0 || a->H < 1 || a->dk <= 0 || a->dv <= 0) return 0;
+  return backward_workspace(a->total_tokens, a->num_seqs, a->H, a->dk, a->dv);
 }
 
 kda_status kda_prefill_backward(const kda_backward_args *a, void *stream) {
@@ -324,7 +324,8 @@ kda_status kda_prefill_backward(const kda_backward_args *a, void *stream) {
   if (N > 0 && (!a->q || !a->k || !a->v || !a->log_alpha || !a->beta || !a->grad_o || !a->grad_q ||
                 !a->grad_k || !a->grad_v || !a->grad_log_alpha || !a->grad_beta))
     return KDA_ERR_INVALID_ARG;
-  if (N > 0 && (!a->workspace || a->workspace_bytes < backward_workspace(a->total_tokens, a->H, a->dk, a->dv)))
+  if (N > 0 && (!a->workspace ||
+                a->workspace_bytes < backward_workspace(a->total_tokens, a->num_seqs, a->H, a->dk, a->dv)))
     return KDA_ERR_INVALID_ARG;
   const Range q{a->q, N * H * dk * es}, k{a->k, N * H * dk * es}, v{a->v, N * H * dv * es};
   const Range la{a->log_alpha, N * H * lad * 4}, be{a->beta, N * H * 4};

@@ -80,7 +80,7 @@ struct BackwardParams {
   const float *init_state;
   const float *d_o, *d_final_state;
   float *gq, *gk, *gv, *gla, *gbeta, *g_init_state;
-  float *ws;              // [N, H, dk, dv]: the state before every position
+  void *ws;               // chunk index, per-chunk quantities, states at chunk starts and ends
   unsigned *err;
   int gate_head;
 };
@@ -104,7 +104,7 @@ size_t prefill_bigchunk_workspace(int N, int B, int H, int chunk);
 cudaError_t launch_prefill_bigchunk(const PrefillParams &p, SeqSpan *spans, void *ws, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s);
-size_t backward_workspace(int N, int H, int dk, int dv);
+size_t backward_workspace(int N, int B, int H, int dk, int dv);
 cudaError_t launch_backward(const BackwardParams &p, bool bf16, cudaStream_t s);
 
 // ---------------------------------------------------------------- helpers

@@ -370,6 +370,13 @@ def prefill_backward(q, k, v, log_alpha, beta, cu_seqlens, grad_o, grad_final_st
     return g
 
 
+def prefill_backward_workspace_bytes(N: int, B: int, H: int, dk: int, dv: int) -> int:
+    """kda_prefill_backward_workspace_size() for these sizes (at least 1 byte)."""
+    a = BackwardArgs()
+    a.num_seqs, a.total_tokens, a.H, a.dk, a.dv = B, N, H, dk, dv
+    return max(int(load().kda_prefill_backward_workspace_size(ctypes.byref(a))), 1)
+
+
 def get_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the latched device status."""
     return int(load().kda_get_device_status(_stream_handle(stream)))

@@ -253,11 +253,14 @@ kda_status kda_short_conv(const kda_conv_args *args, void *stream);
 /*
  * Backward pass of kda_prefill (training): the gradients of <o, grad_o> +
  * <final_state, grad_final_state> with respect to q, k, v, log_alpha, beta and
- * init_state, by reverse-mode differentiation of the recurrence (the blockwise
- * algorithm serves training as well as inference: "Kimi Linear wlasnie
- * pokonal ...", remio.ai, section "Jak Kimi Linear wykorzystuje inteligentniejsza
- * pamiec rekurencyjna").  Token-serial fp32 on CUDA cores, one CTA per
- * (sequence, head): a reference-grade backward, not a tuned one.
+ * init_state, by the blockwise algorithm ("Kimi Linear wlasnie pokonal ...",
+ * remio.ai, section "Jak Kimi Linear wykorzystuje inteligentniejsza pamiec
+ * rekurencyjna": the chunked form serves training as well as inference).  Chunks
+ * of 64 rows: the chunk quantities (pairwise decay products, so exact for any
+ * log_alpha <= 0) and every gradient of a chunk's rows are computed for all
+ * chunks in parallel; only the state at each chunk start (forward) and its
+ * gradient at each chunk end (backward) are chained over a sequence's chunks.
+ * fp32 on CUDA cores.
  * Fields (device pointers, caller-owned):
  *   dtype, num_seqs, total_tokens, H, dk, dv, q, k, v, log_alpha, beta,
  *   cu_seqlens, pad_mask, init_state, gate   as for kda_prefill (chunk is not
@@ -268,9 +271,12 @@ kda_status kda_short_conv(const kda_conv_args *args, void *stream);
  *   grad_log_alpha   fp32, the layout of log_alpha; grad_beta [N, H] fp32;
  *   grad_init_state  [B, H, dk, dv] fp32 or NULL (not written).
  *                All outputs 16-byte aligned and not overlapping any input or
- *                each other; pad positions get zero gradients.
- *   workspace    kda_prefill_backward_workspace_size() bytes, 256-byte aligned
- *                (the state before every position: N * H * dk * dv * 4 bytes).
+ *                each other; pad positions get zero gradients; rows outside
+ *                every sequence are not written.
+ *   workspace    kda_prefill_backward_workspace_size() bytes, 256-byte aligned:
+ *                per 64-row chunk and head the chunk quantities, the state at
+ *                the chunk start and its gradient at the chunk end, about
+ *                5 KB per token and head for d_k = d_v = 128.
  */
 typedef struct {
   kda_dtype dtype;

@@ -1,4 +1,4 @@
-"""GPU parity of kda_prefill_backward (token-serial fp32) against the oracle's fp64
+"""GPU parity of kda_prefill_backward (blockwise, fp32) against the oracle's fp64
 reverse-mode pass (itself pinned by central differences).  Tolerance: 1e-4 normalised
 max-abs error for every gradient, bf16 inputs included (the backward computes in fp32
 from the bf16 values); pad positions get exactly zero gradients.
