@@ -127,23 +127,60 @@ __device__ __forceinline__ bool row_valid(const BackwardParams &p, const ChunkPo
   return r < cp.n && (p.mask == nullptr || p.mask[cp.r0 + r] != 0);
 }
 
-// Loads the chunk's k, q (channel-major, [DK][LP]) and log_alpha, summed into g; pads
-// and rows past the sequence are identity steps (zeros).
-template <int DK, bool BF16>
-__device__ void load_keys(const BackwardParams &p, const ChunkPos &cp, int h, float *kT, float *qT,
-                          float *gT, int tid) {
-  for (int e = tid; e < C * DK; e += kThreads) {
-    const int r = e / DK, c = e % DK;
-    float kv = 0.f, qv = 0.f, lv = 0.f;
-    if (row_valid(p, cp, r)) {
-      const size_t row = (size_t)(cp.r0 + r);
-      kv = load_elem<BF16>(p.k, (row * p.H + h) * DK + c);
-      qv = load_elem<BF16>(p.q, (row * p.H + h) * DK + c);
-      lv = p.log_alpha[la_index(row, h, p.H, DK, c, p.gate_head)];
+// Loads ROWS rows x W columns of a row-major array (bf16 or fp32) in 16-byte pieces, every
+// piece of the thread in flight before the first is used, and hands each element to
+// store(row, column, value); with MASKED, rows whose bit in vmask is clear read as 0.
+// Element (r, c) is at first + r * stride + c.
+template <bool BF16, int ROWS, int W, bool MASKED = true, typename F>
+__device__ __forceinline__ void load_rows(const void *src, size_t first, size_t stride, uint64_t vmask,
+                                          int tid, F store) {
+  constexpr int V = BF16 ? 8 : 4, PER = W / V, TOTAL = ROWS * PER, K = (TOTAL + kThreads - 1) / kThreads;
+  uint4 raw[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int e = tid + k * kThreads, r = e / PER, q = e % PER;
+    raw[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (e < TOTAL && (!MASKED || ((vmask >> r) & 1ull)))
+      raw[k] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const char *>(src) +
+                                                     (first + (size_t)r * stride + (size_t)q * V) * (BF16 ? 2 : 4)));
+  }
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int e = tid + k * kThreads, r = e / PER, c0 = (e % PER) * V;
+    if (e >= TOTAL) continue;
+    const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+    if constexpr (BF16) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        store(r, c0 + 2 * v, __uint_as_float(w[v] << 16));
+        store(r, c0 + 2 * v + 1, __uint_as_float(w[v] & 0xFFFF0000u));
+      }
+    } else {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) store(r, c0 + v, __uint_as_float(w[v]));
     }
-    kT[c * LP + r] = kv;
-    qT[c * LP + r] = qv;
-    gT[c * LP + r] = lv;
+  }
+}
+
+__device__ __forceinline__ uint64_t valid_rows(const BackwardParams &p, const ChunkPos &cp) {
+  uint64_t m = 0;
+  for (int r = 0; r < cp.n; ++r)
+    if (p.mask == nullptr || p.mask[cp.r0 + r] != 0) m |= 1ull << r;
+  return m;
+}
+
+// log_alpha of the chunk into gT ([DK][LP], channel-major), then summed over rows into g.
+template <int DK>
+__device__ void load_gates(const BackwardParams &p, const ChunkPos &cp, int h, uint64_t vmask, float *gT,
+                           int tid) {
+  if (p.gate_head) {
+    for (int e = tid; e < C * DK; e += kThreads) {
+      const int r = e % C, c = e / C;
+      gT[c * LP + r] = ((vmask >> r) & 1ull) ? p.log_alpha[(size_t)(cp.r0 + r) * p.H + h] : 0.f;
+    }
+  } else {
+    load_rows<false, C, DK>(p.log_alpha, ((size_t)cp.r0 * p.H + h) * DK, (size_t)p.H * DK, vmask, tid,
+                            [&](int r, int c, float x) { gT[c * LP + r] = x; });
   }
   __syncthreads();
   if (tid < DK) {
@@ -171,12 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1) intra_kernel(BackwardParams p, co
   if (!locate(p, cbase, blockIdx.x / H, cp)) return;
   float *it = items + (size_t)blockIdx.x * IT::FLOATS;
 
-  for (int e = tid; e < C * DV; e += kThreads) {
-    const int r = e / DV, c = e % DV;
-    vv[e] = row_valid(p, cp, r) ? load_elem<BF16>(p.v, ((size_t)(cp.r0 + r) * H + h) * DV + c) : 0.f;
-  }
-  if (tid < C) bs[tid] = row_valid(p, cp, tid) ? p.beta[(size_t)(cp.r0 + tid) * H + h] : 0.f;
-  load_keys<DK, BF16>(p, cp, h, kT, qT, gT, tid);
+  const uint64_t vmask = valid_rows(p, cp);
+  const size_t first = (size_t)cp.r0 * H + h;
+  load_rows<BF16, C, DV>(p.v, first * DV, (size_t)H * DV, vmask, tid, [&](int r, int c, float x) { vv[r * DV + c] = x; });
+  load_rows<BF16, C, DK>(p.k, first * DK, (size_t)H * DK, vmask, tid, [&](int r, int c, float x) { kT[c * LP + r] = x; });
+  load_rows<BF16, C, DK>(p.q, first * DK, (size_t)H * DK, vmask, tid, [&](int r, int c, float x) { qT[c * LP + r] = x; });
+  if (tid < C) bs[tid] = ((vmask >> tid) & 1ull) ? p.beta[(size_t)(cp.r0 + tid) * H + h] : 0.f;
+  load_gates<DK>(p, cp, h, vmask, gT, tid);
 
   // ---- P_ij, Mf_ij (j <= i): rows rp and 63 - rp, columns j = jg + 8 m
   {
@@ -216,18 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1) intra_kernel(BackwardParams p, co
       }
   }
   __syncthreads();
-  // ---- T = (I + A)^{-1}, A_ij = beta_i P_ij (j < i): column j by forward substitution
-  if (tid < C) {
-    const int j = tid;
-    for (int i = 0; i < C; ++i) Ts[i * LP + j] = i == j ? 1.f : 0.f;
-    for (int i = j + 1; i < C; ++i) {
-      float s = 0.f;
-      for (int m = j; m < i; ++m) s = fmaf(Ps[i * LP + m], Ts[m * LP + j], s);
-      Ts[i * LP + j] = -bs[i] * s;
-    }
+  // ---- M and P out; Q e^g, K~, gamma out; K e^g row-major (in place of q) for the W product
+  for (int e = tid; e < C * C; e += kThreads) {
+    const int i = e / C, j = e % C;
+    it[IT::M + e] = j <= i ? Ms[i * LP + j] : 0.f;
+    it[IT::P + e] = j < i ? Ps[i * LP + j] : 0.f;
+    Ts[i * LP + j] = 0.f;
   }
-  __syncthreads();
-  // ---- outputs that need no product: Q e^g, K~, gamma, M, T, P; then K e^g in place of k
   for (int e = tid; e < C * DK; e += kThreads) {
     const int r = e / DK, c = e % DK;
     const float g = gT[c * LP + r], gC = gT[c * LP + C - 1];
@@ -235,47 +268,104 @@ __global__ void __launch_bounds__(kThreads, 1) intra_kernel(BackwardParams p, co
     it[IT::KT + e] = kT[c * LP + r] * __expf(gC - g);
   }
   if (tid < DK) it[IT::GAM + tid] = __expf(gT[tid * LP + C - 1]);
-  for (int e = tid; e < C * C; e += kThreads) {
-    const int i = e / C, j = e % C;
-    it[IT::M + e] = j <= i ? Ms[i * LP + j] : 0.f;
-    it[IT::T + e] = Ts[i * LP + j];
-    it[IT::P + e] = j < i ? Ps[i * LP + j] : 0.f;
-  }
   __syncthreads();
+  float *kg = qT;                              // [C][DK + 4], K e^g row-major
+  constexpr int KGL = DK + 4;
   for (int e = tid; e < C * DK; e += kThreads) {
-    const int c = e / C, r = e % C;
-    kT[c * LP + r] *= __expf(gT[c * LP + r]);
+    const int r = e / DK, c = e % DK;
+    kg[r * KGL + c] = kT[c * LP + r] * __expf(gT[c * LP + r]);
+  }
+  // ---- T = (I + A)^{-1}, A_ij = beta_i P_ij (j < i), by doubling: 16 x 16 diagonal
+  // blocks by forward substitution (a thread per column), then T21 = -T22 A21 T11 for the
+  // 32 x 32 blocks and the 64 x 64 matrix (Ms is the scratch X = A21 T11)
+  if (tid < C) {
+    const int b0 = tid & ~15, j = tid;
+    Ts[j * LP + j] = 1.f;
+    for (int i = j + 1; i < b0 + 16; ++i) {
+      float s = 0.f;
+      for (int m = j; m < i; ++m) s = fmaf(Ps[i * LP + m], Ts[m * LP + j], s);
+      Ts[i * LP + j] = -bs[i] * s;
+    }
   }
   __syncthreads();
-  // ---- W = T_b (K e^g), U_v = T_b V: thread (row half, column)
+  for (int half = 16; half < C; half *= 2) {
+    // blocks of 2*half: rows/cols [o, o + 2 half); X = A21 T11 (half x half), T21 = -T22 X
+    const int nblk = C / (2 * half), outs = nblk * half * half;
+    for (int e = tid; e < outs; e += kThreads) {
+      const int bl = e / (half * half), r = (e / half) % half, cc = e % half;
+      const int o = bl * 2 * half, i = o + half + r, j = o + cc;
+      float s = 0.f;
+      for (int m = cc; m < half; ++m) s = fmaf(Ps[i * LP + o + m], Ts[(o + m) * LP + j], s);
+      Ms[i * LP + j] = bs[i] * s;
+    }
+    __syncthreads();
+    for (int e = tid; e < outs; e += kThreads) {
+      const int bl = e / (half * half), r = (e / half) % half, cc = e % half;
+      const int o = bl * 2 * half, i = o + half + r, j = o + cc;
+      float s = 0.f;
+      for (int m = 0; m <= r; ++m) s = fmaf(Ts[i * LP + o + half + m], Ms[(o + half + m) * LP + j], s);
+      Ts[i * LP + j] = -s;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < C * C; e += kThreads) it[IT::T + e] = Ts[(e / C) * LP + e % C];
+  // ---- W = T_b (K e^g), U_v = T_b V: thread (4 rows, 8 columns)
   {
-    const int c = tid % 128, i0 = (tid / 128) * 32;
-    if (c < DK) {
-      for (int i = i0; i < i0 + 32; ++i) {
-        float s = 0.f;
-        for (int j = 0; j <= i; ++j) s = fmaf(Ts[i * LP + j] * bs[j], kT[c * LP + j], s);
-        it[IT::W + (size_t)i * DK + c] = s;
+    const int cb = tid & 15, i0 = (tid >> 4) * 4, c0 = cb * 8;
+    auto product = [&](const float *src, int ld, int ncol, size_t off, int ldo) {
+      if (c0 >= ncol) return;
+      float acc[4][8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[a][u] = 0.f;
+      for (int j = 0; j <= i0 + 3; ++j) {
+        const float4 x0 = *reinterpret_cast<const float4 *>(src + j * ld + c0);
+        const float4 x1 = *reinterpret_cast<const float4 *>(src + j * ld + c0 + 4);
+        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const float bj = bs[j];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float t = Ts[(i0 + a) * LP + j] * bj;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[a][u] = fmaf(t, xs[u], acc[a][u]);
+        }
       }
-    }
-    if (c < DV) {
-      for (int i = i0; i < i0 + 32; ++i) {
-        float s = 0.f;
-        for (int j = 0; j <= i; ++j) s = fmaf(Ts[i * LP + j] * bs[j], vv[j * DV + c], s);
-        it[IT::UV + (size_t)i * DV + c] = s;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        float *dst = it + off + (size_t)(i0 + a) * ldo + c0;
+        *reinterpret_cast<float4 *>(dst) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
       }
-    }
+    };
+    __syncthreads();
+    product(kg, KGL, DK, IT::W, DK);
+    product(vv, DV, DV, IT::UV, DV);
   }
 }
 
 // ============================================================ (2) forward chain
 // One CTA per (sequence, head, 32 columns of d_v): S at every chunk start into the
-// workspace; the next chunk's W and K~ arrive by cp.async while the current one runs.
+// workspace; the next chunk's W, K~, U_v slice and gamma arrive by cp.async while the
+// current one runs.  Each thread holds a 2 x 4 block of U and a 4 x 4 block of S's update.
+// Forward chain buffers (two): W and K~ ([C][DK + 4]), the U_v slice ([C][NS + 4]), gamma.
+// Backward chain: two buffers of Q e^g and W ([C][DK], read as float4 along d_k), the dO
+// slice and gamma; one of K~ ([C][DK + 4]) and M ([C][C]).
 template <int DK, int DV>
 struct ChainSmem {
-  static constexpr int LD = DK + 4;                   // padded row of a [C][DK] tile
-  static constexpr int TILE = C * LD;                 // floats
-  static constexpr int BUF = 2 * TILE + C * NS + DK;  // W, K~ (or Q e^g, W), U_v / dO slice, gamma
-  static constexpr int FLOATS = 2 * BUF + DK * NS + C * NS + C * LP;
+  static constexpr int LD = DK + 4;
+  static constexpr int TILE = C * LD;
+  static constexpr int SLP = NS + 4;
+  static constexpr int BUF = 2 * TILE + C * SLP + DK;
+  static constexpr int FLOATS = 2 * BUF + DK * SLP + C * SLP;
+};
+template <int DK, int DV>
+struct DChainSmem {
+  static constexpr int LD = DK + 4, LQ = DK;
+  static constexpr int SLP = NS + 4;
+  static constexpr int BUF = 2 * C * LQ + C * SLP + DK;
+  static constexpr int ABUF = C * LD + C * C;
+  static constexpr int FLOATS = 2 * BUF + ABUF + DK * SLP + C * SLP;
 };
 
 __device__ __forceinline__ void cp_rows(float *dst, int ld_dst, const float *src, int ld_src, int rows,
@@ -292,11 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 states_kernel(BackwardParams p, const int *cbase, const float *items, float *states) {
   using IT = Item<DK, DV>;
   using SMc = ChainSmem<DK, DV>;
-  constexpr int LD = SMc::LD;
+  constexpr int LD = SMc::LD, SLP = SMc::SLP;
   extern __shared__ __align__(16) float sm[];
   float *buf[2] = {sm, sm + SMc::BUF};
-  float *S = sm + 2 * SMc::BUF;           // [DK][NS]
-  float *U = S + DK * NS;                 // [C][NS]
+  float *S = sm + 2 * SMc::BUF;               // [DK][SLP]
+  float *U = S + DK * SLP;                    // [C][SLP]
   if (device_error_latched(p.err)) return;
   const int tiles = DV / NS, sl = blockIdx.x % tiles, bh = blockIdx.x / tiles;
   const int b = bh / p.H, h = bh % p.H, n0 = sl * NS, tid = threadIdx.x;
@@ -304,40 +394,69 @@ states_kernel(BackwardParams p, const int *cbase, const float *items, float *sta
   const float *I0 = p.init_state ? p.init_state + (size_t)bh * DK * DV : nullptr;
   for (int e = tid; e < DK * NS; e += kThreads) {
     const int c = e / NS, n = e % NS;
-    S[e] = I0 ? I0[(size_t)c * DV + n0 + n] : 0.f;
+    S[c * SLP + n] = I0 ? I0[(size_t)c * DV + n0 + n] : 0.f;
   }
   auto load = [&](int j, float *bf) {
     const float *it = items + ((size_t)(cb + j) * p.H + h) * IT::FLOATS;
     cp_rows(bf, LD, it + IT::W, DK, C, DK, tid);
     cp_rows(bf + SMc::TILE, LD, it + IT::KT, DK, C, DK, tid);
-    cp_rows(bf + 2 * SMc::TILE, NS, it + IT::UV + n0, DV, C, NS, tid);
-    cp_rows(bf + 2 * SMc::TILE + C * NS, DK, it + IT::GAM, DK, 1, DK, tid);
+    cp_rows(bf + 2 * SMc::TILE, SLP, it + IT::UV + n0, DV, C, NS, tid);
+    cp_rows(bf + 2 * SMc::TILE + C * SLP, DK, it + IT::GAM, DK, 1, DK, tid);
     tc::cp_async_commit();
   };
   if (nch > 0) load(0, buf[0]);
-  const int n = tid % NS, r0 = tid / NS;          // 8 row groups
+  const int n4 = (tid & 7) * 4, i2 = (tid >> 3) * 2, c4 = (tid >> 3) * 4;
   for (int j = 0; j < nch; ++j) {
     float *bf = buf[j & 1];
     tc::cp_async_wait_all();
     __syncthreads();
     if (j + 1 < nch) load(j + 1, buf[(j + 1) & 1]);
-    const float *Wt = bf, *Kt = bf + SMc::TILE, *Uv = bf + 2 * SMc::TILE, *gam = Uv + C * NS;
+    const float *Wt = bf, *Kt = bf + SMc::TILE, *Uv = bf + 2 * SMc::TILE, *gam = Uv + C * SLP;
     float *Sg = states + ((size_t)(cb + j) * p.H + h) * DK * DV + n0;
-    for (int e = tid; e < DK * NS; e += kThreads) Sg[(size_t)(e / NS) * DV + e % NS] = S[e];
-    // U = U_v - W S  (rows r0 + 8 m)
-    for (int m = 0; m < C / 8; ++m) {
-      const int i = r0 + 8 * m;
-      float s = Uv[i * NS + n];
-      for (int c = 0; c < DK; ++c) s = fmaf(-Wt[i * LD + c], S[c * NS + n], s);
-      U[i * NS + n] = s;
+    for (int e = tid; e < DK * NS / 4; e += kThreads) {
+      const int c = e / (NS / 4), q = (e % (NS / 4)) * 4;
+      *reinterpret_cast<float4 *>(Sg + (size_t)c * DV + q) = *reinterpret_cast<const float4 *>(S + c * SLP + q);
+    }
+    {   // U = U_v - W S: rows i2, i2 + 1, columns n4 .. n4 + 3
+      float a0[4], a1[4];
+      const float4 u0 = *reinterpret_cast<const float4 *>(Uv + i2 * SLP + n4);
+      const float4 u1 = *reinterpret_cast<const float4 *>(Uv + (i2 + 1) * SLP + n4);
+      a0[0] = u0.x; a0[1] = u0.y; a0[2] = u0.z; a0[3] = u0.w;
+      a1[0] = u1.x; a1[1] = u1.y; a1[2] = u1.z; a1[3] = u1.w;
+#pragma unroll 4
+      for (int c = 0; c < DK; ++c) {
+        const float w0 = Wt[i2 * LD + c], w1 = Wt[(i2 + 1) * LD + c];
+        const float4 sv = *reinterpret_cast<const float4 *>(S + c * SLP + n4);
+        a0[0] = fmaf(-w0, sv.x, a0[0]); a0[1] = fmaf(-w0, sv.y, a0[1]);
+        a0[2] = fmaf(-w0, sv.z, a0[2]); a0[3] = fmaf(-w0, sv.w, a0[3]);
+        a1[0] = fmaf(-w1, sv.x, a1[0]); a1[1] = fmaf(-w1, sv.y, a1[1]);
+        a1[2] = fmaf(-w1, sv.z, a1[2]); a1[3] = fmaf(-w1, sv.w, a1[3]);
+      }
+      *reinterpret_cast<float4 *>(U + i2 * SLP + n4) = make_float4(a0[0], a0[1], a0[2], a0[3]);
+      *reinterpret_cast<float4 *>(U + (i2 + 1) * SLP + n4) = make_float4(a1[0], a1[1], a1[2], a1[3]);
     }
     __syncthreads();
-    // S <- Diag(gamma) S + K~^T U  (rows r0 + 8 m of S)
-    for (int m = 0; m < DK / 8; ++m) {
-      const int c = r0 + 8 * m;
-      float s = gam[c] * S[c * NS + n];
-      for (int i = 0; i < C; ++i) s = fmaf(Kt[i * LD + c], U[i * NS + n], s);
-      S[c * NS + n] = s;
+    if (c4 < DK) {   // S <- Diag(gamma) S + K~^T U: rows c4 .. c4 + 3, columns n4 .. n4 + 3
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float4 sv = *reinterpret_cast<const float4 *>(S + (c4 + a) * SLP + n4);
+        const float g = gam[c4 + a];
+        acc[a][0] = g * sv.x; acc[a][1] = g * sv.y; acc[a][2] = g * sv.z; acc[a][3] = g * sv.w;
+      }
+#pragma unroll 4
+      for (int i = 0; i < C; ++i) {
+        const float4 kt = *reinterpret_cast<const float4 *>(Kt + i * LD + c4);
+        const float4 uv = *reinterpret_cast<const float4 *>(U + i * SLP + n4);
+        const float ks[4] = {kt.x, kt.y, kt.z, kt.w}, us[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(ks[a], us[bb], acc[a][bb]);
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4 *>(S + (c4 + a) * SLP + n4) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
     }
   }
   tc::cp_async_wait_all();
@@ -346,17 +465,19 @@ states_kernel(BackwardParams p, const int *cbase, const float *items, float *sta
 // ============================================================ (3) backward chain
 // Chunks in reverse: dS' (gradient of the state after chunk j) into the workspace, then
 //   dU = M^T dO + K~ dS',  dS <- (Q e^g)^T dO + Diag(gamma) dS' - W^T dU.
+// Buffers: K~ and M (one slot, reloaded for chunk j-1 once dU of chunk j is done), and Q e^g,
+// W, the dO slice (zero on pads) and gamma (two slots, one chunk ahead).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 dstates_kernel(BackwardParams p, const int *cbase, const float *items, float *dstates) {
   using IT = Item<DK, DV>;
-  using SMc = ChainSmem<DK, DV>;
-  constexpr int LD = SMc::LD;
+  using SMc = DChainSmem<DK, DV>;
+  constexpr int LD = SMc::LD, LQ = SMc::LQ, SLP = SMc::SLP;
   extern __shared__ __align__(16) float sm[];
   float *buf[2] = {sm, sm + SMc::BUF};
-  float *dS = sm + 2 * SMc::BUF;          // [DK][NS]
-  float *dU = dS + DK * NS;               // [C][NS]
-  float *Mt = dU + C * NS;                // [C][LP]
+  float *Kt = sm + 2 * SMc::BUF, *Mt = Kt + C * LD;     // [C][LD], [C][C]
+  float *dS = Kt + SMc::ABUF;             // [DK][SLP]
+  float *dU = dS + DK * SLP;              // [C][SLP]
   if (device_error_latched(p.err)) return;
   const int tiles = DV / NS, sl = blockIdx.x % tiles, bh = blockIdx.x / tiles;
   const int b = bh / p.H, h = bh % p.H, n0 = sl * NS, tid = threadIdx.x, H = p.H;
@@ -365,81 +486,119 @@ dstates_kernel(BackwardParams p, const int *cbase, const float *items, float *ds
   const float *F = p.d_final_state ? p.d_final_state + (size_t)bh * DK * DV : nullptr;
   for (int e = tid; e < DK * NS; e += kThreads) {
     const int c = e / NS, n = e % NS;
-    dS[e] = F ? F[(size_t)c * DV + n0 + n] : 0.f;
+    dS[c * SLP + n] = F ? F[(size_t)c * DV + n0 + n] : 0.f;
   }
-  // buffer: Q e^g, W, dO slice, gamma; M separately (read after the buffer's tiles)
-  auto load = [&](int j, float *bf) {
+  auto load_b = [&](int j, float *bf) {
     const float *it = items + ((size_t)(cb + j) * H + h) * IT::FLOATS;
-    cp_rows(bf, LD, it + IT::QG, DK, C, DK, tid);
-    cp_rows(bf + SMc::TILE, LD, it + IT::W, DK, C, DK, tid);
-    cp_rows(bf + 2 * SMc::TILE + C * NS, DK, it + IT::GAM, DK, 1, DK, tid);
+    cp_rows(bf, LQ, it + IT::QG, DK, C, DK, tid);
+    cp_rows(bf + C * LQ, LQ, it + IT::W, DK, C, DK, tid);
+    cp_rows(bf + 2 * C * LQ + C * SLP, DK, it + IT::GAM, DK, 1, DK, tid);
+    float *dO = bf + 2 * C * LQ;
+    for (int e = tid; e < C * NS / 4; e += kThreads) {
+      const int r = e / (NS / 4), q = (e % (NS / 4)) * 4, row = j * C + r;
+      const bool ok = row < nrow && (p.mask == nullptr || p.mask[cs + row] != 0);
+      const float *src = p.d_o + ((size_t)(cs + (ok ? row : 0)) * H + h) * DV + n0 + q;
+      tc::cp_async16(tc::smem_u32(dO + r * SLP + q), src, ok ? 16u : 0u);
+    }
     tc::cp_async_commit();
   };
-  const int n = tid % NS, r0 = tid / NS;
-  if (nch > 0) load(nch - 1, buf[(nch - 1) & 1]);
+  auto load_a = [&](int j) {
+    const float *it = items + ((size_t)(cb + j) * H + h) * IT::FLOATS;
+    cp_rows(Kt, LD, it + IT::KT, DK, C, DK, tid);
+    cp_rows(Mt, C, it + IT::M, C, C, C, tid);
+    tc::cp_async_commit();
+  };
+  const int n4 = (tid & 7) * 4, i2 = (tid >> 3) * 2, c4 = (tid >> 3) * 4;
+  if (nch > 0) {
+    load_b(nch - 1, buf[(nch - 1) & 1]);
+    load_a(nch - 1);
+  }
   for (int j = nch - 1; j >= 0; --j) {
     float *bf = buf[j & 1];
-    const float *it = items + ((size_t)(cb + j) * H + h) * IT::FLOATS;
-    // dO slice (pads and rows past the sequence are 0), M, K~ rows read from global below
-    float *dO = bf + 2 * SMc::TILE;
-    for (int e = tid; e < C * NS; e += kThreads) {
-      const int r = e / NS, nn = e % NS, row = j * C + r;
-      const bool ok = row < nrow && (p.mask == nullptr || p.mask[cs + row] != 0);
-      dO[e] = ok ? p.d_o[((size_t)(cs + row) * H + h) * DV + n0 + nn] : 0.f;
-    }
-    for (int e = tid; e < C * C; e += kThreads) Mt[(e / C) * LP + e % C] = it[IT::M + e];
     tc::cp_async_wait_all();
     __syncthreads();
-    if (j > 0) load(j - 1, buf[(j - 1) & 1]);
+    if (j > 0) load_b(j - 1, buf[(j - 1) & 1]);
     float *dSg = dstates + ((size_t)(cb + j) * H + h) * DK * DV + n0;
-    for (int e = tid; e < DK * NS; e += kThreads) dSg[(size_t)(e / NS) * DV + e % NS] = dS[e];
-    const float *Qg = bf, *Wt = bf + SMc::TILE, *gam = dO + C * NS;
-    const float *Kt = it + IT::KT;
-    // dU = M^T dO + K~ dS'
-    for (int m = 0; m < C / 8; ++m) {
-      const int i = r0 + 8 * m;
-      float s = 0.f;
-      for (int r = i; r < C; ++r) s = fmaf(Mt[r * LP + i], dO[r * NS + n], s);
-      const float *kr = Kt + (size_t)i * DK;
-      for (int c = 0; c < DK; ++c) s = fmaf(__ldg(kr + c), dS[c * NS + n], s);
-      dU[i * NS + n] = s;
+    for (int e = tid; e < DK * NS / 4; e += kThreads) {
+      const int c = e / (NS / 4), q = (e % (NS / 4)) * 4;
+      *reinterpret_cast<float4 *>(dSg + (size_t)c * DV + q) = *reinterpret_cast<const float4 *>(dS + c * SLP + q);
+    }
+    const float *Qg = bf, *Wt = bf + C * LQ, *dO = bf + 2 * C * LQ, *gam = dO + C * SLP;
+    {   // dU = M^T dO + K~ dS': rows i2, i2 + 1, columns n4 .. n4 + 3
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int r = i2; r < C; ++r) {
+        const float m0 = Mt[r * C + i2], m1 = Mt[r * C + i2 + 1];
+        const float4 d = *reinterpret_cast<const float4 *>(dO + r * SLP + n4);
+        a0[0] = fmaf(m0, d.x, a0[0]); a0[1] = fmaf(m0, d.y, a0[1]); a0[2] = fmaf(m0, d.z, a0[2]); a0[3] = fmaf(m0, d.w, a0[3]);
+        a1[0] = fmaf(m1, d.x, a1[0]); a1[1] = fmaf(m1, d.y, a1[1]); a1[2] = fmaf(m1, d.z, a1[2]); a1[3] = fmaf(m1, d.w, a1[3]);
+      }
+#pragma unroll 4
+      for (int c = 0; c < DK; ++c) {
+        const float k0 = Kt[i2 * LD + c], k1 = Kt[(i2 + 1) * LD + c];
+        const float4 d = *reinterpret_cast<const float4 *>(dS + c * SLP + n4);
+        a0[0] = fmaf(k0, d.x, a0[0]); a0[1] = fmaf(k0, d.y, a0[1]); a0[2] = fmaf(k0, d.z, a0[2]); a0[3] = fmaf(k0, d.w, a0[3]);
+        a1[0] = fmaf(k1, d.x, a1[0]); a1[1] = fmaf(k1, d.y, a1[1]); a1[2] = fmaf(k1, d.z, a1[2]); a1[3] = fmaf(k1, d.w, a1[3]);
+      }
+      *reinterpret_cast<float4 *>(dU + i2 * SLP + n4) = make_float4(a0[0], a0[1], a0[2], a0[3]);
+      *reinterpret_cast<float4 *>(dU + (i2 + 1) * SLP + n4) = make_float4(a1[0], a1[1], a1[2], a1[3]);
     }
     __syncthreads();
-    // dS <- (Q e^g)^T dO + Diag(gamma) dS' - W^T dU
-    float nd[DK / 8];
+    if (j > 0) load_a(j - 1);
+    if (c4 < DK) {   // dS <- (Q e^g)^T dO + Diag(gamma) dS' - W^T dU: rows c4 .. c4 + 3
+      float acc[4][4];
 #pragma unroll
-    for (int m = 0; m < DK / 8; ++m) {
-      const int c = r0 + 8 * m;
-      float s = gam[c] * dS[c * NS + n];
-      for (int i = 0; i < C; ++i) s = fmaf(Qg[i * LD + c], dO[i * NS + n], fmaf(-Wt[i * LD + c], dU[i * NS + n], s));
-      nd[m] = s;
+      for (int a = 0; a < 4; ++a) {
+        const float4 sv = *reinterpret_cast<const float4 *>(dS + (c4 + a) * SLP + n4);
+        const float g = gam[c4 + a];
+        acc[a][0] = g * sv.x; acc[a][1] = g * sv.y; acc[a][2] = g * sv.z; acc[a][3] = g * sv.w;
+      }
+#pragma unroll 2
+      for (int i = 0; i < C; ++i) {
+        const float4 q = *reinterpret_cast<const float4 *>(Qg + i * LQ + c4);
+        const float4 w = *reinterpret_cast<const float4 *>(Wt + i * LQ + c4);
+        const float4 d = *reinterpret_cast<const float4 *>(dO + i * SLP + n4);
+        const float4 u = *reinterpret_cast<const float4 *>(dU + i * SLP + n4);
+        const float qs[4] = {q.x, q.y, q.z, q.w}, ws[4] = {w.x, w.y, w.z, w.w};
+        const float ds[4] = {d.x, d.y, d.z, d.w}, us[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(qs[a], ds[bb], fmaf(-ws[a], us[bb], acc[a][bb]));
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4 *>(dS + (c4 + a) * SLP + n4) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
     }
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < DK / 8; ++m) dS[(r0 + 8 * m) * NS + n] = nd[m];
   }
   tc::cp_async_wait_all();
   __syncthreads();
   if (p.g_init_state) {
     float *O = p.g_init_state + (size_t)bh * DK * DV + n0;
-    for (int e = tid; e < DK * NS; e += kThreads) O[(size_t)(e / NS) * DV + e % NS] = dS[e];
+    for (int e = tid; e < DK * NS; e += kThreads) O[(size_t)(e / NS) * DV + e % NS] = dS[(e / NS) * SLP + e % NS];
   }
 }
 
 // ============================================================ (4) gradients of a chunk
-// Shared memory (fp32): the d_k-side accumulators dQg, dK~, dW ([C][DK]), dM, dT_b
-// ([C][LP]), dgamma, dbeta; then d_v in 32-column slices: S, dS' ([DK][NS + 1]), dO, U,
-// dU, V ([C][NS + 1]).  After the slices the slice region holds g (channel-major), T,
-// K e^g (later k) ([C][DK + 1]) and dg_C.
-constexpr int NSP = NS + 1;
-
+// Phase 1, d_v in 32-column slices: U, dU and dV of the slice, and its share of the
+// d_v-contractions d(Q e^g) = dO S^T, dK~ = U dS'^T, dW = -dU S^T (4 x DK/16 blocks per
+// thread, in registers), dM = dO U^T and dO-part of dT_b = dU V^T (4 x 4 blocks), dgamma.
+// W, K~, M, T of the chunk stay in shared memory.  Phase 2 (shared memory reused): the
+// chain through T, the pairwise terms with one thread per channel, log_alpha's sums.
 template <int DK, int DV>
 struct GradSmem {
-  static constexpr int CT = C * DK;
-  static constexpr int ACC = 3 * CT + 2 * C * LP + DK + C;
-  static constexpr int SL = 2 * DK * NSP + 4 * C * NSP;
-  static constexpr int PH2 = DK * LP + C * LP + C * (DK + 1) + DK;
-  static constexpr int FLOATS = ACC + (SL > PH2 ? SL : PH2);
+  static constexpr int LD = DK + 4, SPI = NS + 1, SPC = DK + 4;
+  // phase 1 (T at 0 throughout)
+  static constexpr int T0 = 0;
+  static constexpr int W1 = T0 + C * LP, K1 = W1 + C * LD, M1 = K1 + C * LD;
+  static constexpr int SS = M1 + C * LP, SDS = SS + NS * SPC;      // [NS][DK + 4]
+  static constexpr int SDO = SDS + NS * SPC, SU = SDO + C * SPI, SDU = SU + C * SPI, SV = SDU + C * SPI;
+  static constexpr int END1 = SV + C * SPI;
+  // phase 2
+  static constexpr int DQG = T0 + C * LP, DKT = DQG + C * DK, DW = DKT + C * DK;
+  static constexpr int DM = DW + C * DK, DTB = DM + C * LP, GT = DTB + C * LP;
+  static constexpr int KB = GT + DK * LP, DGC = KB + C * (DK + 1), END2 = DGC + DK;
+  static constexpr int DGAM = (END1 > END2 ? END1 : END2), DBETA = DGAM + DK;
+  static constexpr int FLOATS = DBETA + C;
 };
 
 template <int DK, int DV, bool BF16>
@@ -448,15 +607,10 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
             const float *dstates) {
   using IT = Item<DK, DV>;
   using G = GradSmem<DK, DV>;
-  constexpr int KP = DK + 1;
+  constexpr int LD = G::LD, SPI = G::SPI, SPC = G::SPC, KP = DK + 1, CW = DK / 16;
   extern __shared__ __align__(16) float sm[];
-  float *dQg = sm, *dKt = dQg + G::CT, *dW = dKt + G::CT;        // [C][DK]
-  float *dM = dW + G::CT, *dTb = dM + C * LP;                     // [C][LP]
-  float *dgam = dTb + C * LP, *dbeta = dgam + DK;                 // [DK], [C]
-  float *reg = sm + G::ACC;
-  float *sS = reg, *sdS = sS + DK * NSP;                          // [DK][NSP]
-  float *sdO = sdS + DK * NSP, *sU = sdO + C * NSP, *sdU = sU + C * NSP, *sV = sdU + C * NSP;   // [C][NSP]
-  float *gT = reg, *Ts = gT + DK * LP, *kb = Ts + C * LP, *dgC = kb + C * KP;
+  float *Ts = sm + G::T0;
+  float *dgam = sm + G::DGAM, *dbeta = sm + G::DBETA;
   if (device_error_latched(p.err)) return;
   const int H = p.H, h = blockIdx.x % H, tid = threadIdx.x;
   const size_t gidx = blockIdx.x;
@@ -464,136 +618,223 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
   if (!locate(p, cbase, (int)(gidx / H), cp)) return;
   const float *it = items + gidx * IT::FLOATS;
   const float *Sg = states + gidx * DK * DV, *dSg = dstates + gidx * DK * DV;
-  uint64_t vmask = 0;       // valid rows of the chunk
-  for (int r = 0; r < C; ++r)
-    if (row_valid(p, cp, r)) vmask |= 1ull << r;
+  const uint64_t vmask = valid_rows(p, cp);
   auto valid = [&](int r) { return (vmask >> r) & 1ull; };
+  const size_t first = (size_t)cp.r0 * H + h;
   auto betaf = [&](int r) -> float { return valid(r) ? p.beta[(size_t)(cp.r0 + r) * H + h] : 0.f; };
 
-  for (int e = tid; e < G::ACC; e += kThreads) sm[e] = 0.f;
-  __syncthreads();
-
-  // ---- d_v slices: U, dU, dV and the slice's share of every d_v-contraction
+  // ---- phase 1
+  float *Wt = sm + G::W1, *Kt = sm + G::K1, *Mt = sm + G::M1;
+  float *sS = sm + G::SS, *sdS = sm + G::SDS, *sdO = sm + G::SDO, *sU = sm + G::SU;
+  float *sdU = sm + G::SDU, *sV = sm + G::SV;
+  cp_rows(Wt, LD, it + IT::W, DK, C, DK, tid);
+  cp_rows(Kt, LD, it + IT::KT, DK, C, DK, tid);
+  tc::cp_async_commit();
+  for (int e = tid; e < C * C; e += kThreads) {
+    Mt[(e / C) * LP + e % C] = it[IT::M + e];
+    Ts[(e / C) * LP + e % C] = it[IT::T + e];
+  }
+  if (tid < DK) dgam[tid] = 0.f;
+  // register accumulators: rows rb*4 .. +3 and channels cbk*CW .. +CW-1 of dQg, dK~, dW;
+  // rows (tid & 15)*4 .. +3 and columns (tid >> 4)*4 .. +3 of dM and dT_b
+  const int rb = tid >> 4, cbk = tid & 15, i0 = rb * 4, c0 = cbk * CW;
+  const int mi0 = (tid & 15) * 4, mj0 = (tid >> 4) * 4;
+  float aq[4][CW], ak[4][CW], aw[4][CW], am[4][4], at[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+#pragma unroll
+    for (int u = 0; u < CW; ++u) aq[a][u] = ak[a][u] = aw[a][u] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) am[a][u] = at[a][u] = 0.f;
+  }
+  const int n4 = (tid & 7) * 4, i2 = (tid >> 3) * 2;
   for (int n0 = 0; n0 < DV; n0 += NS) {
-    for (int e = tid; e < DK * NS; e += kThreads) {
-      const int c = e / NS, n = e % NS;
-      sS[c * NSP + n] = Sg[(size_t)c * DV + n0 + n];
-      sdS[c * NSP + n] = dSg[(size_t)c * DV + n0 + n];
-    }
-    for (int e = tid; e < C * NS; e += kThreads) {
-      const int r = e / NS, n = e % NS;
-      const bool ok = valid(r);
-      const size_t row = (size_t)(cp.r0 + r) * H + h;
-      sdO[r * NSP + n] = ok ? p.d_o[row * DV + n0 + n] : 0.f;
-      sV[r * NSP + n] = ok ? load_elem<BF16>(p.v, row * DV + n0 + n) : 0.f;
+    __syncthreads();     // previous slice's readers are done
+    load_rows<false, DK, NS, false>(Sg, n0, DV, 0, tid, [&](int c, int n, float x) { sS[n * SPC + c] = x; });
+    load_rows<false, DK, NS, false>(dSg, n0, DV, 0, tid, [&](int c, int n, float x) { sdS[n * SPC + c] = x; });
+    load_rows<false, C, NS>(p.d_o, first * DV + n0, (size_t)H * DV, vmask, tid,
+                            [&](int r, int n, float x) { sdO[r * SPI + n] = x; });
+    load_rows<BF16, C, NS>(p.v, first * DV + n0, (size_t)H * DV, vmask, tid,
+                           [&](int r, int n, float x) { sV[r * SPI + n] = x; });
+    tc::cp_async_wait_all();
+    __syncthreads();
+    {   // U = U_v - W S and dU = M^T dO + K~ dS' (rows i2, i2 + 1; columns n4 .. n4 + 3)
+      float u[2][4], du[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          u[a][bb] = __ldg(it + IT::UV + (size_t)(i2 + a) * DV + n0 + n4 + bb);
+          du[a][bb] = 0.f;
+        }
+      for (int c = 0; c < DK; c += 4) {
+        const float4 w0 = *reinterpret_cast<const float4 *>(Wt + i2 * LD + c);
+        const float4 w1 = *reinterpret_cast<const float4 *>(Wt + (i2 + 1) * LD + c);
+        const float4 k0 = *reinterpret_cast<const float4 *>(Kt + i2 * LD + c);
+        const float4 k1 = *reinterpret_cast<const float4 *>(Kt + (i2 + 1) * LD + c);
+        const float wa[2][4] = {{w0.x, w0.y, w0.z, w0.w}, {w1.x, w1.y, w1.z, w1.w}};
+        const float ka[2][4] = {{k0.x, k0.y, k0.z, k0.w}, {k1.x, k1.y, k1.z, k1.w}};
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          const float4 sv = *reinterpret_cast<const float4 *>(sS + (n4 + bb) * SPC + c);
+          const float4 dv = *reinterpret_cast<const float4 *>(sdS + (n4 + bb) * SPC + c);
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            u[a][bb] -= wa[a][0] * sv.x + wa[a][1] * sv.y + wa[a][2] * sv.z + wa[a][3] * sv.w;
+            du[a][bb] += ka[a][0] * dv.x + ka[a][1] * dv.y + ka[a][2] * dv.z + ka[a][3] * dv.w;
+          }
+        }
+      }
+      for (int r = i2; r < C; ++r) {
+        const float m0 = Mt[r * LP + i2], m1 = Mt[r * LP + i2 + 1];
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          const float d = sdO[r * SPI + n4 + bb];
+          du[0][bb] = fmaf(m0, d, du[0][bb]);
+          du[1][bb] = fmaf(m1, d, du[1][bb]);
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          sU[(i2 + a) * SPI + n4 + bb] = u[a][bb];
+          sdU[(i2 + a) * SPI + n4 + bb] = du[a][bb];
+        }
     }
     __syncthreads();
-    const int n = tid % NS, rg = tid / NS;
-    for (int m = 0; m < C / 8; ++m) {            // U = U_v - W S
-      const int i = rg + 8 * m;
-      float s = it[IT::UV + (size_t)i * DV + n0 + n];
-      const float *wr = it + IT::W + (size_t)i * DK;
-      for (int c = 0; c < DK; ++c) s = fmaf(-__ldg(wr + c), sS[c * NSP + n], s);
-      sU[i * NSP + n] = s;
-    }
-    for (int m = 0; m < C / 8; ++m) {            // dU = M^T dO + K~ dS'
-      const int i = rg + 8 * m;
-      float s = 0.f;
-      for (int r = i; r < C; ++r) s = fmaf(__ldg(it + IT::M + (size_t)r * C + i), sdO[r * NSP + n], s);
-      const float *kr = it + IT::KT + (size_t)i * DK;
-      for (int c = 0; c < DK; ++c) s = fmaf(__ldg(kr + c), sdS[c * NSP + n], s);
-      sdU[i * NSP + n] = s;
-    }
-    __syncthreads();
-    for (int m = 0; m < C / 8; ++m) {            // dV = T_b^T dU
-      const int jr = rg + 8 * m;
-      if (jr >= cp.n) continue;
-      float s = 0.f;
-      for (int i = jr; i < C; ++i) s = fmaf(__ldg(it + IT::T + (size_t)i * C + jr), sdU[i * NSP + n], s);
-      p.gv[((size_t)(cp.r0 + jr) * H + h) * DV + n0 + n] = s * betaf(jr);
-    }
-    {   // d_k-side shares: thread (row i, channel group cg)
-      const int i = tid >> 2, cg = tid & 3;
-      for (int c = cg; c < DK; c += 4) {
-        float q = 0.f, kt = 0.f, w = 0.f;
-#pragma unroll 8
-        for (int nn = 0; nn < NS; ++nn) {
-          const float sc = sS[c * NSP + nn];
-          q = fmaf(sdO[i * NSP + nn], sc, q);
-          kt = fmaf(sU[i * NSP + nn], sdS[c * NSP + nn], kt);
-          w = fmaf(-sdU[i * NSP + nn], sc, w);
+    {   // dV = T_b^T dU (rows i2, i2 + 1 as jr)
+      float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int i = i2; i < C; ++i) {
+        const float t0 = Ts[i * LP + i2], t1 = Ts[i * LP + i2 + 1];
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          const float d = sdU[i * SPI + n4 + bb];
+          dv[0][bb] = fmaf(t0, d, dv[0][bb]);
+          dv[1][bb] = fmaf(t1, d, dv[1][bb]);
         }
-        dQg[i * DK + c] += q;
-        dKt[i * DK + c] += kt;
-        dW[i * DK + c] += w;
       }
-      for (int jr = cg; jr < C; jr += 4) {
-        float mm = 0.f, tb = 0.f;
-#pragma unroll 8
-        for (int nn = 0; nn < NS; ++nn) {
-          mm = fmaf(sdO[i * NSP + nn], sU[jr * NSP + nn], mm);
-          tb = fmaf(sdU[i * NSP + nn], sV[jr * NSP + nn], tb);
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int jr = i2 + a;
+        if (jr < cp.n) {
+          const float bj = betaf(jr);
+          float *dst = p.gv + ((size_t)(cp.r0 + jr) * H + h) * DV + n0 + n4;
+          *reinterpret_cast<float4 *>(dst) = make_float4(dv[a][0] * bj, dv[a][1] * bj, dv[a][2] * bj, dv[a][3] * bj);
         }
-        if (jr <= i) dM[i * LP + jr] += mm;
-        dTb[i * LP + jr] += tb;
       }
+    }
+    // d_k-side shares of this slice
+#pragma unroll 2
+    for (int nn = 0; nn < NS; ++nn) {
+      float ro[4], ru[4], rd[4], cs[CW], cd[CW];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        ro[a] = sdO[(i0 + a) * SPI + nn];
+        ru[a] = sU[(i0 + a) * SPI + nn];
+        rd[a] = sdU[(i0 + a) * SPI + nn];
+      }
+#pragma unroll
+      for (int u = 0; u < CW; u += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(sS + nn * SPC + c0 + u);
+        const float4 y = *reinterpret_cast<const float4 *>(sdS + nn * SPC + c0 + u);
+        cs[u] = x.x; cs[u + 1] = x.y; cs[u + 2] = x.z; cs[u + 3] = x.w;
+        cd[u] = y.x; cd[u + 1] = y.y; cd[u + 2] = y.z; cd[u + 3] = y.w;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int u = 0; u < CW; ++u) {
+          aq[a][u] = fmaf(ro[a], cs[u], aq[a][u]);
+          ak[a][u] = fmaf(ru[a], cd[u], ak[a][u]);
+          aw[a][u] = fmaf(-rd[a], cs[u], aw[a][u]);
+        }
+      float mo[4], md[4], mu[4], mv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        mo[a] = sdO[(mi0 + a) * SPI + nn];
+        md[a] = sdU[(mi0 + a) * SPI + nn];
+        mu[a] = sU[(mj0 + a) * SPI + nn];
+        mv[a] = sV[(mj0 + a) * SPI + nn];
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          am[a][bb] = fmaf(mo[a], mu[bb], am[a][bb]);
+          at[a][bb] = fmaf(md[a], mv[bb], at[a][bb]);
+        }
     }
     if (tid < DK) {
       float s = 0.f;
-      for (int nn = 0; nn < NS; ++nn) s = fmaf(sS[tid * NSP + nn], sdS[tid * NSP + nn], s);
+      for (int nn = 0; nn < NS; ++nn) s = fmaf(sS[nn * SPC + tid], sdS[nn * SPC + tid], s);
       dgam[tid] += s;
     }
-    __syncthreads();
   }
-
-  // ---- phase 2: g (channel-major), T, K e^g into the slice region
-  for (int e = tid; e < C * DK; e += kThreads) {
-    const int r = e / DK, c = e % DK;
-    gT[c * LP + r] = valid(r) ? p.log_alpha[la_index((size_t)(cp.r0 + r), h, H, DK, c, p.gate_head)] : 0.f;
-  }
-  for (int e = tid; e < C * C; e += kThreads) Ts[(e / C) * LP + e % C] = it[IT::T + e];
   __syncthreads();
-  if (tid < DK) {
-    float acc = 0.f;
-    for (int r = 0; r < C; ++r) {
-      acc += gT[tid * LP + r];
-      gT[tid * LP + r] = acc;
+
+  // ---- phase 2: accumulators to shared memory; g (channel-major), K e^g
+  float *dQg = sm + G::DQG, *dKt = sm + G::DKT, *dW = sm + G::DW;
+  float *dM = sm + G::DM, *dTb = sm + G::DTB, *gT = sm + G::GT, *kb = sm + G::KB, *dgC = sm + G::DGC;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+#pragma unroll
+    for (int u = 0; u < CW; ++u) {
+      dQg[(i0 + a) * DK + c0 + u] = aq[a][u];
+      dKt[(i0 + a) * DK + c0 + u] = ak[a][u];
+      dW[(i0 + a) * DK + c0 + u] = aw[a][u];
+    }
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) {
+      dM[(mi0 + a) * LP + mj0 + bb] = (mj0 + bb <= mi0 + a) ? am[a][bb] : 0.f;
+      dTb[(mi0 + a) * LP + mj0 + bb] = at[a][bb];
     }
   }
-  __syncthreads();
-  for (int e = tid; e < C * DK; e += kThreads) {
-    const int r = e / DK, c = e % DK;
-    kb[r * KP + c] = valid(r) ? load_elem<BF16>(p.k, ((size_t)(cp.r0 + r) * H + h) * DK + c) * __expf(gT[c * LP + r])
-                              : 0.f;
-  }
-  __syncthreads();
-  {   // dT_b += dW (K e^g)^T: thread (column jr, row group ig)
+  load_rows<BF16, C, DK>(p.k, first * DK, (size_t)H * DK, vmask, tid, [&](int r, int c, float x) { kb[r * KP + c] = x; });
+  load_gates<DK>(p, cp, h, vmask, gT, tid);
+  {   // dT_b += dW (K e^g)^T: thread (column jr, rows ig + 4 a)
     const int jr = tid & 63, ig = tid >> 6;
     float acc[C / 4];
 #pragma unroll
     for (int a = 0; a < C / 4; ++a) acc[a] = 0.f;
     for (int c = 0; c < DK; ++c) {
-      const float kg = kb[jr * KP + c];
+      const float kg = kb[jr * KP + c] * __expf(gT[c * LP + jr]);
 #pragma unroll
       for (int a = 0; a < C / 4; ++a) acc[a] = fmaf(dW[(ig + 4 * a) * DK + c], kg, acc[a]);
     }
 #pragma unroll
     for (int a = 0; a < C / 4; ++a) dTb[(ig + 4 * a) * LP + jr] += acc[a];
   }
-  __syncthreads();
-  if (tid < DK) {   // d(K e^g) = T_b^T dW, in place of dW (thread per channel)
-    const int c = tid;
-    float col[C];
+  {   // d(K e^g) = T_b^T dW: thread (rows i0 .. as jr, channels c0 ..); written after a barrier
+    float acc[4][CW];
 #pragma unroll
-    for (int i = 0; i < C; ++i) col[i] = dW[i * DK + c];
-#pragma unroll 4
-    for (int jr = 0; jr < C; ++jr) {
-      float s = 0.f;
-      for (int i = jr; i < C; ++i) s = fmaf(Ts[i * LP + jr], col[i], s);
-      dW[jr * DK + c] = s * betaf(jr);
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int u = 0; u < CW; ++u) acc[a][u] = 0.f;
+    for (int i = i0; i < C; ++i) {
+      float tv[4], wv[CW];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) tv[a] = Ts[i * LP + i0 + a];
+#pragma unroll
+      for (int u = 0; u < CW; u += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(dW + i * DK + c0 + u);
+        wv[u] = x.x; wv[u + 1] = x.y; wv[u + 2] = x.z; wv[u + 3] = x.w;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int u = 0; u < CW; ++u) acc[a][u] = fmaf(tv[a], wv[u], acc[a][u]);
     }
-  } else if (tid - DK < C) {   // dbeta (T_b part): sum_i dT_b,ij T_ij
-    const int jr = tid - DK;
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float bj = betaf(i0 + a);
+#pragma unroll
+      for (int u = 0; u < CW; ++u) dW[(i0 + a) * DK + c0 + u] = acc[a][u] * bj;
+    }
+  }
+  if (tid < C) {   // dbeta (T_b part): sum_i dT_b,ij T_ij
+    const int jr = tid;
     float s = 0.f;
     for (int i = jr; i < C; ++i) s = fmaf(dTb[i * LP + jr], Ts[i * LP + jr], s);
     dbeta[jr] = s;
@@ -601,46 +842,63 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
   __syncthreads();
   for (int e = tid; e < C * C; e += kThreads) dTb[(e / C) * LP + e % C] *= betaf(e % C);   // dT
   __syncthreads();
-  if (tid < C) {   // X = dT T^T, in place (thread per row)
-    const int i = tid;
-    float row[C];
+  {   // X = dT T^T (4 x 4 blocks), then dA = -T^T X, strictly lower
+    float acc[4][4];
 #pragma unroll
-    for (int m = 0; m < C; ++m) row[m] = dTb[i * LP + m];
-#pragma unroll 4
-    for (int jr = 0; jr < C; ++jr) {
-      float s = 0.f;
-      for (int m = 0; m <= jr; ++m) s = fmaf(row[m], Ts[jr * LP + m], s);
-      dTb[i * LP + jr] = s;
-    }
-  }
-  __syncthreads();
-  if (tid < C) {   // dA_ij = -sum_{m >= i} T_mi X_mj (j < i), in place (thread per column)
-    const int jr = tid;
-    float col[C];
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int m = 0; m < C; ++m) col[m] = dTb[m * LP + jr];
-#pragma unroll 4
-    for (int i = 0; i < C; ++i) {
-      float s = 0.f;
-      if (jr < i)
-        for (int m = i; m < C; ++m) s = fmaf(Ts[m * LP + i], col[m], s);
-      dTb[i * LP + jr] = -s;
+      for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+    for (int m = 0; m < C; ++m) {
+      float dv[4], tv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        dv[a] = dTb[(mi0 + a) * LP + m];
+        tv[a] = Ts[(mj0 + a) * LP + m];
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(dv[a], tv[bb], acc[a][bb]);
     }
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) dTb[(mi0 + a) * LP + mj0 + bb] = acc[a][bb];
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+    for (int m = 0; m < C; ++m) {
+      float tv[4], xv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        tv[a] = Ts[m * LP + mi0 + a];
+        xv[a] = dTb[m * LP + mj0 + a];
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(tv[a], xv[bb], acc[a][bb]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb)
+        dTb[(mi0 + a) * LP + mj0 + bb] = (mj0 + bb < mi0 + a) ? -acc[a][bb] : 0.f;
+    __syncthreads();
   }
-  __syncthreads();
   if (tid < C) {   // dbeta += sum_j dA_ij P_ij
     const int i = tid;
     float s = 0.f;
     for (int jr = 0; jr < i; ++jr) s = fmaf(dTb[i * LP + jr], __ldg(it + IT::P + (size_t)i * C + jr), s);
     dbeta[i] += s;
   }
-  // raw k replaces K e^g; dg_C = colsum(dK~ * K~) + dgamma * gamma
-  for (int e = tid; e < C * DK; e += kThreads) {
-    const int r = e / DK, c = e % DK;
-    kb[r * KP + c] = valid(r) ? load_elem<BF16>(p.k, ((size_t)(cp.r0 + r) * H + h) * DK + c) : 0.f;
-  }
+  // dP = beta_i dA; dg_C = colsum(dK~ * K~) + dgamma * gamma
   __syncthreads();
-  for (int e = tid; e < C * C; e += kThreads) dTb[(e / C) * LP + e % C] *= betaf(e / C);        // dP
+  for (int e = tid; e < C * C; e += kThreads) dTb[(e / C) * LP + e % C] *= betaf(e / C);
   if (tid < DK) {
     const int c = tid;
     const float gC = gT[c * LP + C - 1];
@@ -649,60 +907,51 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
     dgC[c] = s;
   }
   __syncthreads();
-  auto qval = [&](int r, int c) -> float {
-    return valid(r) ? load_elem<BF16>(p.q, ((size_t)(cp.r0 + r) * H + h) * DK + c) : 0.f;
-  };
-  // ---- pairwise terms with the chain through e^{+-g}; two threads per channel split the rows
-  // (pairs j <= i: rows 0-44 and 45-63 as i, then rows 0-18 and 19-63 as j)
-  const int c = tid % 128, half = tid / 128;
-  if (c < DK) {
+  // ---- pairwise terms (j <= i) and the chain through e^{+-g}, one thread per channel:
+  // row i's own terms accumulate in registers, its partners' (rows j) in shared memory
+  if (tid < DK) {
+    const int c = tid;
     const float gC = gT[c * LP + C - 1];
-    const int ia = half ? 45 : 0, ib = half ? C : 45;
-    for (int i = ia; i < ib; ++i) {
-      const float gi = gT[c * LP + i], ki = kb[i * KP + c], qi = qval(i, c);
+    auto qload = [&](int i) -> float {
+      return valid(i) ? load_elem<BF16>(p.q, ((size_t)(cp.r0 + i) * H + h) * DK + c) : 0.f;
+    };
+    float qn = qload(0), qn2 = qload(1);
+    for (int i = 0; i < C; ++i) {
+      const float gi = gT[c * LP + i], ki = kb[i * KP + c];
+      const float qi = qn;
+      qn = qn2;
+      qn2 = i + 2 < C ? qload(i + 2) : 0.f;     // two rows ahead
+      const float eg = __expf(gi), et = __expf(gC - gi);
+      const float tq = dQg[i * DK + c], tk = dW[i * DK + c], tt = dKt[i * DK + c];
+      dW[i * DK + c] = 0.f;
+      dKt[i * DK + c] = 0.f;
       float dk = 0.f, dq = 0.f, dg = 0.f;
       for (int jr = 0; jr <= i; ++jr) {
-        const float e = __expf(gi - gT[c * LP + jr]) * kb[jr * KP + c];
-        const float dp = dTb[i * LP + jr], dm = dM[i * LP + jr];    // dP is 0 on the diagonal
-        dk = fmaf(dp, e, dk);
-        dq = fmaf(dm, e, dq);
-        dg = fmaf(fmaf(dp, ki, dm * qi), e, dg);
+        const float kj = kb[jr * KP + c];
+        const float e = __expf(gi - gT[c * LP + jr]);
+        const float dp = dTb[i * LP + jr], dm = dM[i * LP + jr];
+        const float a = fmaf(dp, ki, dm * qi) * e;     // both sides' common factor
+        dk = fmaf(dp * kj, e, dk);
+        dq = fmaf(dm * kj, e, dq);
+        dg = fmaf(a, kj, dg);
+        dW[jr * DK + c] += a;                          // d k_j
+        dKt[jr * DK + c] -= a * kj;                    // d g_j
       }
-      const float eg = __expf(gi), et = __expf(gC - gi);
-      dq = fmaf(dQg[i * DK + c], eg, dq);
-      dg = fmaf(dQg[i * DK + c], qi * eg, dg);
-      dk = fmaf(dW[i * DK + c], eg, dk);
-      dg = fmaf(dW[i * DK + c], ki * eg, dg);
-      dk = fmaf(dKt[i * DK + c], et, dk);
-      dg = fmaf(-dKt[i * DK + c], ki * et, dg);
+      dq = fmaf(tq, eg, dq);
+      dg = fmaf(tq, qi * eg, dg);
+      dk = fmaf(tk, eg, dk);
+      dg = fmaf(tk, ki * eg, dg);
+      dk = fmaf(tt, et, dk);
+      dg = fmaf(-tt, ki * et, dg);
       dQg[i * DK + c] = dq;
-      dW[i * DK + c] = dk;
-      dKt[i * DK + c] = dg;
+      dW[i * DK + c] += dk;
+      dKt[i * DK + c] += dg;
     }
-  }
-  __syncthreads();
-  if (c < DK) {
-    const int ja = half ? 19 : 0, jb = half ? C : 19;
-    for (int jr = ja; jr < jb; ++jr) {
-      const float gj = gT[c * LP + jr], kj = kb[jr * KP + c];
-      float dk = 0.f, dg = 0.f;
-      for (int i = jr; i < C; ++i) {
-        const float e = __expf(gT[c * LP + i] - gj);
-        const float a = fmaf(dTb[i * LP + jr], kb[i * KP + c], dM[i * LP + jr] * qval(i, c));
-        dk = fmaf(a, e, dk);
-        dg = fmaf(a * kj, e, dg);
-      }
-      dW[jr * DK + c] += dk;
-      dKt[jr * DK + c] -= dg;
-    }
-  }
-  __syncthreads();
-  // ---- g -> log_alpha (reverse cumulative sum, dg_C on every row), outputs
-  if (tid < DK) {
-    float acc = dgC[tid];
+    // g -> log_alpha: reverse cumulative sum, dg_C on every row
+    float acc = dgC[c];
     for (int r = C - 1; r >= 0; --r) {
-      acc += dKt[r * DK + tid];
-      dKt[r * DK + tid] = acc;
+      acc += dKt[r * DK + c];
+      dKt[r * DK + c] = acc;
     }
   }
   __syncthreads();
@@ -748,16 +997,16 @@ cudaError_t launch(const BackwardParams &p, cudaStream_t s) {
   intra_kernel<DK, DV, BF16><<<(unsigned)gch, kThreads, smem1, s>>>(p, cbase, items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const unsigned gridc = (unsigned)B * p.H * (DV / NS);
-  const int smem2 = ChainSmem<DK, DV>::FLOATS * 4;
+  const int smem2 = ChainSmem<DK, DV>::FLOATS * 4, smem3 = DChainSmem<DK, DV>::FLOATS * 4;
   if ((e = cudaFuncSetAttribute(states_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2)) !=
       cudaSuccess)
     return e;
   states_kernel<DK, DV><<<gridc, kThreads, smem2, s>>>(p, cbase, items, states);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(dstates_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2)) !=
+  if ((e = cudaFuncSetAttribute(dstates_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem3)) !=
       cudaSuccess)
     return e;
-  dstates_kernel<DK, DV><<<gridc, kThreads, smem2, s>>>(p, cbase, items, dstates);
+  dstates_kernel<DK, DV><<<gridc, kThreads, smem3, s>>>(p, cbase, items, dstates);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int smem4 = GradSmem<DK, DV>::FLOATS * 4;
   if ((e = cudaFuncSetAttribute(grad_kernel<DK, DV, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
