@@ -103,13 +103,19 @@ typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1 } kda_gate;
  *   final_state  [B, H, dk, dv] fp32 or NULL (not written).  It may be the same
  *                pointer as init_state (in-place update) but may not otherwise
  *                overlap an input.
- *   chunk        0 (default: 64 for bf16, 16 for fp32), 16, 32 or 64.  The
- *                result is defined by the recurrence and does not depend on the
- *                chunk size beyond rounding.
+ *   chunk        0 (default: 64 for bf16, 16 for fp32), 16, 32 or 64; 128 or
+ *                256 for bf16 with d_k = d_v = 128 and the full workspace (the
+ *                tensor-core path merges 64-row chunks into longer ones: the
+ *                pages' chunk of 256, "Kimi Linear's 75% KV cache cut ...",
+ *                theclarity.today, fourth paragraph), else KDA_ERR_UNSUPPORTED.
+ *                The result is defined by the recurrence and does not depend on
+ *                the chunk size beyond rounding.
  *   workspace    device scratch, 256-byte aligned.  kda_prefill_workspace_size()
  *                bytes select the fastest path (for bf16, d_k = d_v = 128,
  *                chunk 64: a two-kernel path that stores each chunk's
- *                intermediate tiles, about 73 KB per 64 tokens and head).  A
+ *                intermediate tiles, about 73 KB per 64 tokens and head; chunk
+ *                128 / 256 also store the merged chunk items, about 2.5 / 3 KB
+ *                per token and head in all).  A
  *                smaller workspace selects a fused single-kernel path; a pad
  *                mask needs at least 16 bytes per sequence (rounded up to 256).
  *                May be NULL when pad_mask is NULL.
@@ -341,7 +347,9 @@ kda_status kda_debug_set_fault(int fault, long long wait_cycles);
  * pass: 11 item load,
  * 12 first product group of a chunk, 13 second product group, 14 buffer
  * release (loading side); single-kernel tensor-core prefill: 21-26 (its six
- * waits in program order).
+ * waits in program order); chunks of 128 / 256: the state pass uses 11-14 as
+ * above (11 any item tile) and 16 for the U_v block, the merge kernels 31
+ * (operand loads), 32 and 33 (their two product groups).
  */
 int kda_debug_timeout_site(void *stream);
 
