@@ -647,7 +647,7 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
 #pragma unroll
     for (int u = 0; u < 4; ++u) am[a][u] = at[a][u] = 0.f;
   }
-  const int n4 = (tid & 7) * 4, i2 = (tid >> 3) * 2;
+  const int nl = tid & 7, i2 = (tid >> 3) * 2;
   for (int n0 = 0; n0 < DV; n0 += NS) {
     __syncthreads();     // previous slice's readers are done
     load_rows<false, DK, NS, false>(Sg, n0, DV, 0, tid, [&](int c, int n, float x) { sS[n * SPC + c] = x; });
@@ -658,13 +658,14 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
                            [&](int r, int n, float x) { sV[r * SPI + n] = x; });
     tc::cp_async_wait_all();
     __syncthreads();
-    {   // U = U_v - W S and dU = M^T dO + K~ dS' (rows i2, i2 + 1; columns n4 .. n4 + 3)
+    {   // U = U_v - W S and dU = M^T dO + K~ dS' (rows i2, i2 + 1; columns nl + 8 bb: lanes
+        // read neighbouring rows of S, so the float4 reads fall in distinct banks)
       float u[2][4], du[2][4];
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          u[a][bb] = __ldg(it + IT::UV + (size_t)(i2 + a) * DV + n0 + n4 + bb);
+          u[a][bb] = __ldg(it + IT::UV + (size_t)(i2 + a) * DV + n0 + nl + 8 * bb);
           du[a][bb] = 0.f;
         }
       for (int c = 0; c < DK; c += 4) {
@@ -676,8 +677,8 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
         const float ka[2][4] = {{k0.x, k0.y, k0.z, k0.w}, {k1.x, k1.y, k1.z, k1.w}};
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          const float4 sv = *reinterpret_cast<const float4 *>(sS + (n4 + bb) * SPC + c);
-          const float4 dv = *reinterpret_cast<const float4 *>(sdS + (n4 + bb) * SPC + c);
+          const float4 sv = *reinterpret_cast<const float4 *>(sS + (nl + 8 * bb) * SPC + c);
+          const float4 dv = *reinterpret_cast<const float4 *>(sdS + (nl + 8 * bb) * SPC + c);
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             u[a][bb] -= wa[a][0] * sv.x + wa[a][1] * sv.y + wa[a][2] * sv.z + wa[a][3] * sv.w;
@@ -689,7 +690,7 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
         const float m0 = Mt[r * LP + i2], m1 = Mt[r * LP + i2 + 1];
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          const float d = sdO[r * SPI + n4 + bb];
+          const float d = sdO[r * SPI + nl + 8 * bb];
           du[0][bb] = fmaf(m0, d, du[0][bb]);
           du[1][bb] = fmaf(m1, d, du[1][bb]);
         }
@@ -698,8 +699,8 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
       for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          sU[(i2 + a) * SPI + n4 + bb] = u[a][bb];
-          sdU[(i2 + a) * SPI + n4 + bb] = du[a][bb];
+          sU[(i2 + a) * SPI + nl + 8 * bb] = u[a][bb];
+          sdU[(i2 + a) * SPI + nl + 8 * bb] = du[a][bb];
         }
     }
     __syncthreads();
@@ -709,7 +710,7 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
         const float t0 = Ts[i * LP + i2], t1 = Ts[i * LP + i2 + 1];
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          const float d = sdU[i * SPI + n4 + bb];
+          const float d = sdU[i * SPI + nl + 8 * bb];
           dv[0][bb] = fmaf(t0, d, dv[0][bb]);
           dv[1][bb] = fmaf(t1, d, dv[1][bb]);
         }
@@ -719,8 +720,9 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
         const int jr = i2 + a;
         if (jr < cp.n) {
           const float bj = betaf(jr);
-          float *dst = p.gv + ((size_t)(cp.r0 + jr) * H + h) * DV + n0 + n4;
-          *reinterpret_cast<float4 *>(dst) = make_float4(dv[a][0] * bj, dv[a][1] * bj, dv[a][2] * bj, dv[a][3] * bj);
+          float *dst = p.gv + ((size_t)(cp.r0 + jr) * H + h) * DV + n0 + nl;
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) dst[8 * bb] = dv[a][bb] * bj;
         }
       }
     }
@@ -907,24 +909,29 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
     dgC[c] = s;
   }
   __syncthreads();
-  // ---- pairwise terms (j <= i) and the chain through e^{+-g}, one thread per channel:
-  // row i's own terms accumulate in registers, its partners' (rows j) in shared memory
-  if (tid < DK) {
-    const int c = tid;
+  // ---- the chain through e^{+-g} (elementwise, in place), then the pairwise terms (j <= i).
+  // Two threads per channel: rows as i in [0, 45) and [45, 64) (equal pair counts); a pair
+  // adds to row i's and row j's sums in shared memory (atomically: the other thread of the
+  // channel may add to the same row), d(Q e^g) only to row i (owned by this thread).
+  const int c = tid % 128, half = tid / 128;
+  const int ia = half ? 45 : 0, ib = half ? C : 45;
+  if (c < DK) {
     const float gC = gT[c * LP + C - 1];
-    auto qload = [&](int i) -> float {
-      return valid(i) ? load_elem<BF16>(p.q, ((size_t)(cp.r0 + i) * H + h) * DK + c) : 0.f;
-    };
-    float qn = qload(0), qn2 = qload(1);
-    for (int i = 0; i < C; ++i) {
+    for (int i = ia; i < ib; ++i) {
       const float gi = gT[c * LP + i], ki = kb[i * KP + c];
-      const float qi = qn;
-      qn = qn2;
-      qn2 = i + 2 < C ? qload(i + 2) : 0.f;     // two rows ahead
+      const float qi = valid(i) ? load_elem<BF16>(p.q, (first + (size_t)i * H) * DK + c) : 0.f;
       const float eg = __expf(gi), et = __expf(gC - gi);
       const float tq = dQg[i * DK + c], tk = dW[i * DK + c], tt = dKt[i * DK + c];
-      dW[i * DK + c] = 0.f;
-      dKt[i * DK + c] = 0.f;
+      dQg[i * DK + c] = tq * eg;
+      dW[i * DK + c] = fmaf(tk, eg, tt * et);
+      dKt[i * DK + c] = fmaf(tq, qi * eg, ki * fmaf(tk, eg, -tt * et));
+    }
+  }
+  __syncthreads();
+  if (c < DK) {
+    for (int i = ia; i < ib; ++i) {
+      const float gi = gT[c * LP + i], ki = kb[i * KP + c];
+      const float qi = valid(i) ? load_elem<BF16>(p.q, (first + (size_t)i * H) * DK + c) : 0.f;
       float dk = 0.f, dq = 0.f, dg = 0.f;
       for (int jr = 0; jr <= i; ++jr) {
         const float kj = kb[jr * KP + c];
@@ -934,24 +941,20 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
         dk = fmaf(dp * kj, e, dk);
         dq = fmaf(dm * kj, e, dq);
         dg = fmaf(a, kj, dg);
-        dW[jr * DK + c] += a;                          // d k_j
-        dKt[jr * DK + c] -= a * kj;                    // d g_j
+        atomicAdd(dW + jr * DK + c, a);                // d k_j
+        atomicAdd(dKt + jr * DK + c, -a * kj);         // d g_j
       }
-      dq = fmaf(tq, eg, dq);
-      dg = fmaf(tq, qi * eg, dg);
-      dk = fmaf(tk, eg, dk);
-      dg = fmaf(tk, ki * eg, dg);
-      dk = fmaf(tt, et, dk);
-      dg = fmaf(-tt, ki * et, dg);
-      dQg[i * DK + c] = dq;
-      dW[i * DK + c] += dk;
-      dKt[i * DK + c] += dg;
+      dQg[i * DK + c] += dq;
+      atomicAdd(dW + i * DK + c, dk);
+      atomicAdd(dKt + i * DK + c, dg);
     }
-    // g -> log_alpha: reverse cumulative sum, dg_C on every row
-    float acc = dgC[c];
+  }
+  __syncthreads();
+  if (tid < DK) {   // g -> log_alpha: reverse cumulative sum, dg_C on every row
+    float acc = dgC[tid];
     for (int r = C - 1; r >= 0; --r) {
-      acc += dKt[r * DK + c];
-      dKt[r * DK + c] = acc;
+      acc += dKt[r * DK + tid];
+      dKt[r * DK + tid] = acc;
     }
   }
   __syncthreads();
