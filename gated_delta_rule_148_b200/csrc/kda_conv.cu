@@ -13,11 +13,13 @@
 //
 // Layout: x, y [N, D] (bf16 or fp32), weight [D, W] fp32, bias [D] fp32,
 // conv_state [B, W-1, D] fp32.  The operation is HBM-bound (read x, write y):
-// kernel A gives each CTA 128 packed positions and up to 2048 channels; the pad
-// mask of those positions is compacted once per CTA (warp ballots) into the list
-// of valid rows, and each thread walks those rows for its 8 consecutive channels
-// with the window in registers and the next 8 rows' loads already in flight (a
-// ring of raw 16- or 32-byte loads), so each thread keeps 8 loads outstanding.  Kernel B writes the new
+// kernel A gives each CTA a contiguous span of packed positions (about N / (2 x SMs
+// per channel block): one wave) and up to 2048 channels; the pad mask of the span
+// is compacted once (warp ballots, 256 positions a pass) into the list of valid
+// rows, and each thread walks those rows for its 8 consecutive channels with the
+// window in registers and the next 8 rows' loads already in flight (a ring of raw
+// 16- or 32-byte loads), so each thread keeps 8 loads outstanding and fills its
+// ring once per span.  Kernel B writes the new
 // state after kernel A, one thread per (sequence, channel), so conv_state may be
 // updated in place.
 #include "kda_internal.cuh"
@@ -25,13 +27,14 @@
 namespace kda {
 namespace conv {
 
-constexpr int kSeg = 128;            // packed positions per CTA
+constexpr int kSeg = 256;            // packed positions per compaction pass (one per thread)
+constexpr int kMaxSpan = 4096;       // packed positions per CTA at most (the list of valid rows)
 constexpr int kThreads = 256;
 constexpr int kPer = 8;              // channels per thread
 constexpr int kChan = kPer * kThreads;  // channels per CTA
 constexpr int kRing = 8;             // rows whose loads are in flight ahead of the walk (bf16)
 constexpr int kMaxW = 4;
-static_assert(kSeg <= kThreads, "one compaction ballot per position");
+static_assert(kSeg == kThreads, "one compaction ballot per position");
 
 // Source of a window entry: a packed position (>= 0) or state row j (encoded -1 - j).
 struct Hist {
@@ -128,21 +131,23 @@ __device__ __forceinline__ void store_row(void *y, size_t row, int D, int c, con
   }
 }
 
-// Kernel A: outputs of packed positions [kSeg*blockIdx.x, +kSeg), channels
-// [kChan*blockIdx.y, +kChan).  Thread t owns channels 8t .. 8t+7 and walks the
-// CTA's valid rows in order with the window in registers, so each x row is read
-// once; the loads of one row are coalesced across the CTA's threads, and the
-// ring keeps the loads of the next kRing rows in flight.
+// Kernel A: outputs of packed positions [span*blockIdx.x, +span), channels
+// [kChan*blockIdx.y, +kChan), span chosen on the host so that the grid is about
+// one wave (every CTA then fills its load ring once, not once per short block).
+// Thread t owns channels 8t .. 8t+7 and walks the CTA's valid rows in order with
+// the window in registers, so each x row is read once; the loads of one row are
+// coalesced across the CTA's threads, and the ring keeps the loads of the next
+// kRing rows in flight.
 template <bool BF16, int KW>      // KW: the window width W (1..4), fixed at compile time
-__global__ void __launch_bounds__(kThreads, 2) conv_kernel(ConvParams p) {
-  __shared__ int vpos[kSeg];
+__global__ void __launch_bounds__(kThreads, 2) conv_kernel(ConvParams p, int span) {
+  __shared__ int vpos[kMaxSpan];
   __shared__ int wcnt[kThreads / 32];
   __shared__ Hist hist_sh;
   if (device_error_latched(p.err)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int W = KW;
   const int D = p.D, B = p.num_seqs;
-  const int s0 = blockIdx.x * kSeg, s1 = min(s0 + kSeg, p.N);
+  const int s0 = blockIdx.x * span, s1 = min(s0 + span, p.N);
   const int c_lo = blockIdx.y * kChan, nch = min(kChan, D - c_lo);
   if (blockIdx.x == 0 && blockIdx.y == 0) {       // cu_seqlens: 0, non-decreasing, ends at N
     bool bad = false;
@@ -172,21 +177,25 @@ __global__ void __launch_bounds__(kThreads, 2) conv_kernel(ConvParams p) {
     const int sb = max(p.cu[b], 0);
     const int a = max(s0, sb), e = min(s1, p.cu[b + 1]);
     if (a >= e) continue;
-    // ---- compact the valid positions of [a, e) (in order) into vpos
-    const int pos = a + tid;
-    const bool ok = pos < e && (p.mask == nullptr || p.mask[pos] != 0);
-    const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
-    if (lane == 0) wcnt[warp] = __popc(bits);
+    // ---- compact the valid positions of [a, e) (in order) into vpos, kSeg at a time
     if (tid == 0) hist_sh = history_before(p.mask, sb, a, W);
-    __syncthreads();
-    int before = 0, nvalid = 0;
+    int nvalid = 0;
+    for (int a0 = a; a0 < e; a0 += kSeg) {
+      const int pos = a0 + tid;
+      const bool ok = pos < e && (p.mask == nullptr || p.mask[pos] != 0);
+      const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
+      if (lane == 0) wcnt[warp] = __popc(bits);
+      __syncthreads();
+      int before = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) {
-      before += (w < warp) ? wcnt[w] : 0;
-      nvalid += wcnt[w];
+      for (int w = 0; w < kThreads / 32; ++w) {
+        before += (w < warp) ? wcnt[w] : 0;
+        tot += wcnt[w];
+      }
+      if (ok) vpos[nvalid + before + __popc(bits & ((1u << lane) - 1u))] = pos;
+      nvalid += tot;
+      __syncthreads();     // wcnt is rewritten by the next pass
     }
-    if (ok) vpos[before + __popc(bits & ((1u << lane) - 1u))] = pos;
-    __syncthreads();
     if (mine) {
       // ---- the window before the first valid row (oldest first)
       float win[kMaxW - 1][kPer];
@@ -287,12 +296,26 @@ __global__ void __launch_bounds__(kThreads) conv_state_kernel(ConvParams p) {
 cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s) {
   using namespace conv;
   if (p.N > 0) {
-    const dim3 grid((unsigned)((p.N + kSeg - 1) / kSeg), (unsigned)((p.D + kChan - 1) / kChan));
-    using Kern = void (*)(ConvParams);
+    // positions per CTA: about one wave of two CTAs per SM over the channel blocks,
+    // at least kSeg and at most kMaxSpan
+    static int sms = 0;
+    if (sms == 0) {
+      int dev = 0, v = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        v = 148;
+      sms = v;
+    }
+    const int cblocks = (p.D + kChan - 1) / kChan;
+    const long long slots = (long long)2 * sms / cblocks > 0 ? (long long)2 * sms / cblocks : 1;
+    long long span = ((long long)p.N + slots - 1) / slots;
+    span = span < kSeg ? kSeg : (span > kMaxSpan ? kMaxSpan : span);
+    const dim3 grid((unsigned)((p.N + span - 1) / span), (unsigned)cblocks);
+    using Kern = void (*)(ConvParams, int);
     static const Kern kerns[2][4] = {
         {conv_kernel<false, 1>, conv_kernel<false, 2>, conv_kernel<false, 3>, conv_kernel<false, 4>},
         {conv_kernel<true, 1>, conv_kernel<true, 2>, conv_kernel<true, 3>, conv_kernel<true, 4>}};
-    kerns[bf16 ? 1 : 0][p.W - 1]<<<grid, kThreads, 0, s>>>(p);
+    kerns[bf16 ? 1 : 0][p.W - 1]<<<grid, kThreads, 0, s>>>(p, (int)span);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

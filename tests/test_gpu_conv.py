@@ -115,3 +115,20 @@ def test_conv_empty_sequences_keep_state():
     assert norm_err(to_np(y), y_ref) <= CTOL["f32"]
     np.testing.assert_array_equal(to_np(so), s_ref.astype(np.float32))
     np.testing.assert_array_equal(to_np(so)[0], c["state"][0])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv_long_spans_many_pads(dtype):
+    """A packed batch long enough that each CTA's span of positions (about one wave of CTAs)
+    exceeds one 256-position compaction pass, with 30 % pads, sequence boundaries inside
+    spans and a carried state: every output and the new state against the oracle."""
+    lengths = [40000, 1, 3, 65000, 257, 30000]
+    D, W = 72, 4
+    c = gen.conv_inputs(97, lengths, D, W, dtype, pad_frac=0.3)
+    d = _dev(c, dtype)
+    so = torch.empty((len(lengths), W - 1, D), device="cuda")
+    y = _run(d, so)
+    y_ref, s_ref = orc.short_conv(c["x"], c["weight"], c["bias"], c["cu_seqlens"], c["pad_mask"], c["state"])
+    assert norm_err(to_np(y), y_ref) <= CTOL[dtype]
+    assert np.all(to_np(y)[c["pad_mask"] == 0] == 0.0)
+    np.testing.assert_array_equal(to_np(so), s_ref.astype(np.float32))
