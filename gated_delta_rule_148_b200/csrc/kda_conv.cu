@@ -297,7 +297,7 @@ cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s) {
   using namespace conv;
   if (p.N > 0) {
     // positions per CTA: about one wave of two CTAs per SM over the channel blocks,
-    // at least kSeg and at most kMaxSpan
+    // at least 32 and at most kMaxSpan
     static int sms = 0;
     if (sms == 0) {
       int dev = 0, v = 0;
@@ -309,7 +309,7 @@ cudaError_t launch_short_conv(const ConvParams &p, bool bf16, cudaStream_t s) {
     const int cblocks = (p.D + kChan - 1) / kChan;
     const long long slots = (long long)2 * sms / cblocks > 0 ? (long long)2 * sms / cblocks : 1;
     long long span = ((long long)p.N + slots - 1) / slots;
-    span = span < kSeg ? kSeg : (span > kMaxSpan ? kMaxSpan : span);
+    span = span < 32 ? 32 : (span > kMaxSpan ? kMaxSpan : span);
     const dim3 grid((unsigned)((p.N + span - 1) / span), (unsigned)cblocks);
     using Kern = void (*)(ConvParams, int);
     static const Kern kerns[2][4] = {
