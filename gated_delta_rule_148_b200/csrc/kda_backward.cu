@@ -601,6 +601,109 @@ struct GradSmem {
   static constexpr int FLOATS = DBETA + C;
 };
 
+// Pairwise terms of one channel, split by 16-row blocks.  With dP (strictly lower) and
+// dM (lower) of the chunk, per channel c the sums
+//   S1_i = sum_{j<=i} dP_ij k_j e^{g_i - g_j},  S2_i = sum_{j<=i} dM_ij k_j e^{g_i - g_j},
+//   S3_j = sum_{i>=j} (dP_ij k_i + dM_ij q_i) e^{g_i - g_j}
+// give d k_i += S1_i + S3_i, d q_i += S2_i, d g_i += k_i S1_i + q_i S2_i - k_i S3_i.  For j in
+// an earlier block than i, with R = g at the last row before i's block,
+// e^{g_i - g_j} = e^{g_i - R} e^{R - g_j}, both factors <= 1: those sums become dense
+// products with per-row factors (no overflow, one exponential per row and block).  Pairs
+// inside a block take e^{g_i - g_j} directly.  Results are added to shared memory
+// atomically (both threads of a channel add to some rows).
+struct PairCtx {
+  const float *gc;        // g of the channel, rows 0..63 (stride 1)
+  const float *kb;        // k, [C][KP]
+  int KP, c, DK;
+  const float *dP, *dM;   // [C][LP]
+  float *dk, *dq, *dg;    // [C][DK]
+};
+
+// i-side sums for rows of block B (> 0) from rows j < 16 B
+template <int B>
+__device__ __forceinline__ void pair_cross_i(const PairCtx &x, const float *qrow) {
+  constexpr int NJ = 16 * B;
+  const float R = x.gc[NJ - 1];
+  float y[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) y[j] = x.kb[j * x.KP + x.c] * __expf(R - x.gc[j]);
+#pragma unroll 2
+  for (int ii = 0; ii < 16; ++ii) {
+    const int i = NJ + ii;
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      s1 = fmaf(x.dP[i * LP + j], y[j], s1);
+      s2 = fmaf(x.dM[i * LP + j], y[j], s2);
+    }
+    const float a = __expf(x.gc[i] - R);
+    s1 *= a;
+    s2 *= a;
+    atomicAdd(x.dk + i * x.DK + x.c, s1);
+    atomicAdd(x.dq + i * x.DK + x.c, s2);
+    atomicAdd(x.dg + i * x.DK + x.c, fmaf(x.kb[i * x.KP + x.c], s1, qrow[ii] * s2));
+  }
+}
+
+// j-side sums for rows j < 16 B from the rows of block B
+template <int B>
+__device__ __forceinline__ void pair_cross_j(const PairCtx &x, const float *qrow) {
+  constexpr int NJ = 16 * B;
+  const float R = x.gc[NJ - 1];
+  float z[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) z[j] = 0.f;
+#pragma unroll 2
+  for (int ii = 0; ii < 16; ++ii) {
+    const int i = NJ + ii;
+    const float a = __expf(x.gc[i] - R);
+    const float ka = x.kb[i * x.KP + x.c] * a, qa = qrow[ii] * a;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) z[j] = fmaf(x.dP[i * LP + j], ka, fmaf(x.dM[i * LP + j], qa, z[j]));
+  }
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const float s3 = z[j] * __expf(R - x.gc[j]);
+    atomicAdd(x.dk + j * x.DK + x.c, s3);
+    atomicAdd(x.dg + j * x.DK + x.c, -x.kb[j * x.KP + x.c] * s3);
+  }
+}
+
+// pairs inside block B (j <= i, both in the block)
+template <int B>
+__device__ __forceinline__ void pair_block(const PairCtx &x, const float *qrow) {
+  constexpr int O = 16 * B;
+  float kk[16], gg[16], s3[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    kk[r] = x.kb[(O + r) * x.KP + x.c];
+    gg[r] = x.gc[O + r];
+    s3[r] = 0.f;
+  }
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) {
+    const int i = O + ii;
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int jj = 0; jj <= ii; ++jj) {
+      const int j = O + jj;
+      const float e = __expf(gg[ii] - gg[jj]);
+      const float dp = x.dP[i * LP + j], dm = x.dM[i * LP + j];
+      s1 = fmaf(dp * kk[jj], e, s1);
+      s2 = fmaf(dm * kk[jj], e, s2);
+      s3[jj] = fmaf(fmaf(dp, kk[ii], dm * qrow[ii]), e, s3[jj]);
+    }
+    atomicAdd(x.dk + i * x.DK + x.c, s1);
+    atomicAdd(x.dq + i * x.DK + x.c, s2);
+    atomicAdd(x.dg + i * x.DK + x.c, fmaf(kk[ii], s1, qrow[ii] * s2));
+  }
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) {
+    atomicAdd(x.dk + (O + jj) * x.DK + x.c, s3[jj]);
+    atomicAdd(x.dg + (O + jj) * x.DK + x.c, -kk[jj] * s3[jj]);
+  }
+}
+
 template <int DK, int DV, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 grad_kernel(BackwardParams p, const int *cbase, const float *items, const float *states,
@@ -909,10 +1012,8 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
     dgC[c] = s;
   }
   __syncthreads();
-  // ---- the chain through e^{+-g} (elementwise, in place), then the pairwise terms (j <= i).
-  // Two threads per channel: rows as i in [0, 45) and [45, 64) (equal pair counts); a pair
-  // adds to row i's and row j's sums in shared memory (atomically: the other thread of the
-  // channel may add to the same row), d(Q e^g) only to row i (owned by this thread).
+  // ---- the chain through e^{+-g} (elementwise, in place), then the pairwise terms (two
+  // threads per channel, rows as i in [0, 45) and [45, 64) for the elementwise pass).
   const int c = tid % 128, half = tid / 128;
   const int ia = half ? 45 : 0, ib = half ? C : 45;
   if (c < DK) {
@@ -929,24 +1030,33 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
   }
   __syncthreads();
   if (c < DK) {
-    for (int i = ia; i < ib; ++i) {
-      const float gi = gT[c * LP + i], ki = kb[i * KP + c];
-      const float qi = valid(i) ? load_elem<BF16>(p.q, (first + (size_t)i * H) * DK + c) : 0.f;
-      float dk = 0.f, dq = 0.f, dg = 0.f;
-      for (int jr = 0; jr <= i; ++jr) {
-        const float kj = kb[jr * KP + c];
-        const float e = __expf(gi - gT[c * LP + jr]);
-        const float dp = dTb[i * LP + jr], dm = dM[i * LP + jr];
-        const float a = fmaf(dp, ki, dm * qi) * e;     // both sides' common factor
-        dk = fmaf(dp * kj, e, dk);
-        dq = fmaf(dm * kj, e, dq);
-        dg = fmaf(a, kj, dg);
-        atomicAdd(dW + jr * DK + c, a);                // d k_j
-        atomicAdd(dKt + jr * DK + c, -a * kj);         // d g_j
+    // the channel's g as a contiguous row, q of the rows this thread's blocks read
+    const PairCtx x{gT + c * LP, kb, KP, c, DK, dTb, dM, dW, dQg, dKt};
+    float qrow[2][16];
+    auto load_q = [&](int blk, float *dst) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int i = 16 * blk + r;
+        dst[r] = valid(i) ? load_elem<BF16>(p.q, (first + (size_t)i * H) * DK + c) : 0.f;
       }
-      dQg[i * DK + c] += dq;
-      atomicAdd(dW + i * DK + c, dk);
-      atomicAdd(dKt + i * DK + c, dg);
+    };
+    if (half == 0) {         // blocks 0, 1 inside; rows of blocks 1, 2 from earlier blocks
+      load_q(0, qrow[0]);
+      load_q(1, qrow[1]);
+      pair_block<0>(x, qrow[0]);
+      pair_block<1>(x, qrow[1]);
+      pair_cross_i<1>(x, qrow[1]);
+      pair_cross_j<1>(x, qrow[1]);
+      load_q(2, qrow[0]);
+      pair_cross_i<2>(x, qrow[0]);
+      pair_cross_j<2>(x, qrow[0]);
+    } else {                 // blocks 2, 3 inside; rows of block 3 from earlier blocks
+      load_q(2, qrow[0]);
+      load_q(3, qrow[1]);
+      pair_block<2>(x, qrow[0]);
+      pair_block<3>(x, qrow[1]);
+      pair_cross_i<3>(x, qrow[1]);
+      pair_cross_j<3>(x, qrow[1]);
     }
   }
   __syncthreads();
