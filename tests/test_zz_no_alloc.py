@@ -93,3 +93,19 @@ def test_noalloc_rejects_more_sequences_than_its_scratch_holds():
         kda.KDA_BF16, kda.NOALLOC_MAX_SEQS + 1, kda.NOALLOC_MAX_SEQS + 1, 1, 64, 64)
     st = kda.load().kda_prefill_noalloc(ctypes.byref(a), None)
     assert st == kda.KDA_ERR_INVALID_ARG
+
+
+def test_noalloc_refuses_chunks_of_128_and_256():
+    """Chunks of 128 / 256 need the merged chunk items of the full workspace, which the
+    fixed scratch cannot hold: the call is refused and writes nothing."""
+    inp = _padded_case(123, [300, 77], pads=False)
+    d = dev_inputs(inp, "bf16")
+    N, H = d["q"].shape[0], d["q"].shape[1]
+    o = torch.full((N, H, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    for chunk in (128, 256):
+        with pytest.raises(kda.KdaError) as e:
+            kda.prefill_noalloc(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"], o,
+                                chunk=chunk)
+        assert e.value.status == kda.KDA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.all(o == 7.0)
