@@ -184,3 +184,45 @@ def test_long_prefill_128k_sampled_heads(chunk):
     o, fs = _run(inp, chunk)
     _check(inp, o, fs, heads=[0, 21])
     assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("chunk", CHUNKS)
+def test_many_short_sequences_with_pads(chunk):
+    """2000 sequences of 1-300 tokens (most shorter than one chunk, many with an odd number of
+    64-row sub-chunks), H = 2, 10 % interior pads, nonzero states."""
+    rng = np.random.default_rng(141)
+    lengths = [int(x) for x in rng.integers(1, 301, size=2000)]
+    inp = gen.random_case(142, lengths, 2, 128, 128, "bf16", init_state=True)
+    N = int(inp["cu_seqlens"][-1])
+    m = (rng.uniform(size=N) > 0.1).astype(np.uint8)
+    for key in ("q", "k", "v"):
+        inp[key][m == 0] = 0.0
+    inp["pad_mask"] = m
+    o, fs = _run(inp, chunk)
+    _check(inp, o, fs)
+    assert np.all(to_np(o)[m == 0] == 0.0)
+
+
+def test_graph_replay_chunk_128():
+    """The chunk-128 path (index, intra, merge, state kernels) captured in a CUDA graph and
+    replayed: the same outputs as the eager call, bit for bit."""
+    inp = gen.random_case(143, [700, 333], 4, 128, 128, "bf16", init_state=True)
+    d = dev_inputs(inp, "bf16")
+    ws = kda.prefill_workspace(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"], chunk=128)
+    o = torch.empty((d["q"].shape[0], 4, 128), dtype=torch.bfloat16, device="cuda")
+    fs = torch.empty((2, 4, 128, 128), dtype=torch.float32, device="cuda")
+    run = lambda: kda.prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                              init_state=d["init_state"], o=o, final_state=fs, chunk=128, workspace=ws)
+    run()
+    torch.cuda.synchronize()
+    o_ref, fs_ref = o.clone(), fs.clone()
+    o.zero_()
+    fs.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    g.replay()
+    torch.cuda.synchronize()
+    assert kda.get_device_status() == kda.KDA_OK
+    assert torch.equal(o, o_ref) and torch.equal(fs, fs_ref)
+    _check(inp, o, fs)
