@@ -216,42 +216,68 @@ __global__ void __launch_bounds__(kThreads, 1) intra_kernel(BackwardParams p, co
   if (tid < C) bs[tid] = ((vmask >> tid) & 1ull) ? p.beta[(size_t)(cp.r0 + tid) * H + h] : 0.f;
   load_gates<DK>(p, cp, h, vmask, gT, tid);
 
-  // ---- P_ij, Mf_ij (j <= i): rows rp and 63 - rp, columns j = jg + 8 m
-  {
-    const int rp = tid >> 3, jg = tid & 7;
-    const int rows[2] = {rp, C - 1 - rp};
-    float aP[2][8], aM[2][8];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int m = 0; m < 8; ++m) aP[a][m] = aM[a][m] = 0.f;
+  // ---- P_ij, Mf_ij (j <= i) by 16-row blocks.  Pairs inside a block: e^{g_i - g_j} per
+  // channel.  Rows i after the block of j: with L the log decay at the block's last row,
+  // e^{g_i - g_j} = e^{g_i - L} e^{L - g_j} (both <= 1), so P and Mf over those rows are
+  // products of staged factor tiles (32 channels at a time, staged in the T tile).
+  for (int pr = tid; pr < 4 * 136; pr += kThreads) {
+    const int b = pr / 136, q = pr % 136;
+    int ii = 0;
+    while ((ii + 1) * (ii + 2) / 2 <= q) ++ii;
+    const int i = 16 * b + ii, j = 16 * b + (q - ii * (ii + 1) / 2);
+    float sp = 0.f, smf = 0.f;
     for (int c = 0; c < DK; ++c) {
-      const float *kc = kT + c * LP, *gc = gT + c * LP;
+      const float e = __expf(gT[c * LP + i] - gT[c * LP + j]) * kT[c * LP + j];
+      sp = fmaf(kT[c * LP + i], e, sp);
+      smf = fmaf(qT[c * LP + i], e, smf);
+    }
+    Ps[i * LP + j] = sp;
+    Ms[i * LP + j] = smf;
+  }
+  {
+    constexpr int CH = 32, SL = CH + 1;
+    float *Fs = Ts, *Gs = Ts + 16 * SL, *Hs = Gs + 48 * SL;     // [16][SL], [48][SL], [48][SL]
+    const int jl = tid & 15, ig = tid >> 4;
+    for (int bs0 = 0; bs0 < 3; ++bs0) {
+      const int j0 = 16 * bs0, i0 = j0 + 16, nr = C - i0, L = j0 + 15;
+      float ap[3] = {0.f, 0.f, 0.f}, am[3] = {0.f, 0.f, 0.f};
+      for (int c0 = 0; c0 < DK; c0 += CH) {
+        __syncthreads();       // the previous chunk's tiles are read
+        for (int e = tid; e < (16 + nr) * CH; e += kThreads) {
+          const int r = e / CH, cc = e % CH, c = c0 + cc;
+          const float gl = gT[c * LP + L];
+          if (r < 16) {
+            Fs[r * SL + cc] = kT[c * LP + j0 + r] * __expf(gl - gT[c * LP + j0 + r]);
+          } else {
+            const int i = i0 + r - 16;
+            const float a = __expf(gT[c * LP + i] - gl);
+            Gs[(r - 16) * SL + cc] = kT[c * LP + i] * a;
+            Hs[(r - 16) * SL + cc] = qT[c * LP + i] * a;
+          }
+        }
+        __syncthreads();
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        const int i = rows[a];
-        const float gi = gc[i], ki = kc[i], qi = qT[c * LP + i];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int j = jg + 8 * m;
-          if (j <= i) {
-            const float e = __expf(gi - gc[j]) * kc[j];
-            aP[a][m] = fmaf(ki, e, aP[a][m]);
-            aM[a][m] = fmaf(qi, e, aM[a][m]);
+        for (int m = 0; m < 3; ++m) {
+          const int r = ig + 16 * m;
+          if (r < nr) {
+#pragma unroll 8
+            for (int cc = 0; cc < CH; ++cc) {
+              const float f = Fs[jl * SL + cc];
+              ap[m] = fmaf(Gs[r * SL + cc], f, ap[m]);
+              am[m] = fmaf(Hs[r * SL + cc], f, am[m]);
+            }
           }
         }
       }
-    }
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int i = rows[a], j = jg + 8 * m;
-        if (j <= i) {
-          Ps[i * LP + j] = aP[a][m];
-          Ms[i * LP + j] = aM[a][m];
+      for (int m = 0; m < 3; ++m) {
+        const int r = ig + 16 * m;
+        if (r < nr) {
+          Ps[(i0 + r) * LP + j0 + jl] = ap[m];
+          Ms[(i0 + r) * LP + j0 + jl] = am[m];
         }
       }
+    }
   }
   __syncthreads();
   // ---- M and P out; Q e^g, K~, gamma out; K e^g row-major (in place of q) for the W product
