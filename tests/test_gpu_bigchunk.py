@@ -226,3 +226,24 @@ def test_graph_replay_chunk_128():
     assert kda.get_device_status() == kda.KDA_OK
     assert torch.equal(o, o_ref) and torch.equal(fs, fs_ref)
     _check(inp, o, fs)
+
+
+def test_bounded_wait_runs_out_in_the_ring_state_pass():
+    """Failure detection without a GPU fault on the chunk-128 path: with the planted fault the
+    state pass's producer issues no part loads, so the first waits on the ring's slots run out
+    (after ~1 ms here); the call returns, the status reads KDA_ERR_DEVICE_TIMEOUT with an
+    item-load site, and the next normal call on the same context matches the oracle."""
+    inp = gen.random_case(144, [700, 130], 2, 128, 128, "bf16", init_state=True)
+    d = dev_inputs(inp, "bf16")
+    kda.debug_set_fault(kda.KDA_FAULT_STARVE_STATE_LOADS, 2_000_000)
+    try:
+        kda.prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                    init_state=d["init_state"], chunk=128)
+        st = kda.get_device_status()
+    finally:
+        kda.debug_set_fault(0)
+    assert st == kda.KDA_ERR_DEVICE_TIMEOUT, kda.status_string(st)
+    assert kda.debug_timeout_site() in (11, 16)       # a tile slot or the U_v slot
+    assert kda.get_device_status() == kda.KDA_OK
+    o, fs = _run(inp, 128)
+    _check(inp, o, fs)
