@@ -156,9 +156,10 @@ struct IntraMaps {
 
 // The next item's inputs are loaded by TMA into tiles the current item no longer
 // needs, so the prep reads them from shared memory: q into the K e^{g_C-g} / T tile
-// once T_b is packed, log_alpha into the T_b and V tiles (32 KB) once the W and U_v
-// products have read them, k into the K e^{-g} tile once the item's bulk stores have
-// read it.  V follows once the prep has read the staged rows.  (The plain per-thread
+// and k into the K e^{-g} / A region once the inverse has read A and T_b is packed
+// (U_v then leaves by direct stores, not through that region), log_alpha into the
+// T_b and V tiles (32 KB) once the W and U_v products have read them.  V follows
+// once the prep has read the staged rows.  (The plain per-thread
 // loads this replaces were held up by the number of misses an SM keeps in flight.)
 // With the head-wise gate (4 bytes of gate per row) the inputs are plain loads.
 template <bool GATE_HEAD>     // log_alpha [N, H] (one gate per token and head) instead of [N, H, dk]
@@ -272,7 +273,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
       prep::decay_and_tiles_global<GATE_HEAD>(
           reinterpret_cast<const uint16_t *>(p.q), reinterpret_cast<const uint16_t *>(p.k), p.log_alpha,
           c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
-          decay_sh, beta_val, beta_sh, xrows, tid, !first && !kStage,
+          decay_sh, beta_val, beta_sh, xrows, tid, !first,
           kStage ? reinterpret_cast<const float *>(base + A_TB) : nullptr,
           kStage ? reinterpret_cast<const uint16_t *>(base + A_TS) : nullptr,
           kStage ? reinterpret_cast<const uint16_t *>(base + A_KH) : nullptr);
@@ -345,9 +346,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
-    if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {   // T is packed: next item's q
+    if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {
+      // T is packed and A is consumed: next item's q into the T tile, k into the A region
       const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
+      fence_async_smem();
       stage_q(nx.h, nx.c0);
+      stage_k(nx.h, nx.c0);
     }
     // zero V rows of invalid positions (tail of the sequence, pads)
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
@@ -387,7 +391,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     }
     if ((warp & 3) < 2) {
       // rows r = lr (< 64), columns 64 wg .. 64 wg + 63: -W -> rows 0..63 of the Q G | K G
-      // tile (its products are done), U_v -> the K e^{-g} region; both leave by bulk store
+      // tile (its products are done), left by bulk store; U_v straight to the item
       const int r = lr;
       float v[32];
       for (int q2 = 0; q2 < 2; ++q2) {
@@ -396,7 +400,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
         for (int j = 0; j < 32; ++j) v[j] = -v[j];
         prep::store_row32(base + A_QK + wg * 128 * 128, 128, r, q2 * 4, v);
         tmem_ld32(tm + lane_base + A_TM_UV + (uint32_t)(wg * 64 + q2 * 32), v);
-        prep::store_row32(base + A_KH + wg * 64 * 128, 64, r, q2 * 4, v);
+        prep::store_row32(it + IT_UV + wg * 64 * 128, 64, r, q2 * 4, v);
       }
     }
     fence_async_smem();
@@ -405,13 +409,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     if (tid == 0) {
       bulk_store(it + IT_WQ, base + A_QK, 64 * 128);                              // -W, block 0
       bulk_store(it + IT_WQ + 128 * 128, base + A_QK + 128 * 128, 64 * 128);      // -W, block 1
-      bulk_store(it + IT_UV, base + A_KH, 64 * 256);
       bulk_commit();       // the next item's tile writes wait for these reads
-      if (kStage && item + (int)gridDim.x < nitems) {   // next item's k once U_v has left
-        const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
-        bulk_wait_read();
-        stage_k(nx.h, nx.c0);
-      }
     }
     first = false;
   }
