@@ -241,18 +241,33 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     }
   }
   bool first = true;
+  // An item's position, span, row validity and beta (rows tid < 64) are read one item
+  // ahead, so the item starts without waiting on these global loads.
+  struct Ahead {
+    ItemPos ip;
+    SeqSpan sp;
+    bool vr;
+    float beta;
+  };
+  auto read_ahead = [&](int item) {
+    Ahead a;
+    a.ip = locate_item(p, spans, cbase, item, h0, Hg);
+    a.sp = spans[a.ip.b];
+    a.vr = tid < kC && row_ok(p, a.sp, a.ip.c0 + tid);
+    a.beta = a.vr ? __ldg(p.beta + (size_t)(a.ip.c0 + tid) * H + a.ip.h) : 0.f;
+    return a;
+  };
+  Ahead nx = read_ahead(blockIdx.x);
   for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
-    const ItemPos ip = locate_item(p, spans, cbase, item, h0, Hg);
+    const Ahead cur = nx;
+    const ItemPos ip = cur.ip;
     const int h = ip.h, c0 = ip.c0;
-    const SeqSpan sp = spans[ip.b];
     unsigned char *it = items + ip.off;
 
-    float beta_val = 0.f;      // stored to shared memory inside the prep, after its loads
+    const float beta_val = cur.beta;   // stored to shared memory inside the prep, after its loads
     if (tid < kC) {
-      const bool vr = row_ok(p, sp, c0 + tid);
-      const unsigned bits = __ballot_sync(0xFFFFFFFFu, vr);
+      const unsigned bits = __ballot_sync(0xFFFFFFFFu, cur.vr);
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
-      if (vr) beta_val = __ldg(p.beta + (size_t)(c0 + tid) * H + h);
     }
     if (tid < 4) unsafe_sh[tid] = 0u;
     if (kStage) {
@@ -346,12 +361,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
+    if (item + (int)gridDim.x < nitems) nx = read_ahead(item + gridDim.x);
     if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {
       // T is packed and A is consumed: next item's q into the T tile, k into the A region
-      const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
       fence_async_smem();
-      stage_q(nx.h, nx.c0);
-      stage_k(nx.h, nx.c0);
+      stage_q(nx.ip.h, nx.ip.c0);
+      stage_k(nx.ip.h, nx.ip.c0);
     }
     // zero V rows of invalid positions (tail of the sequence, pads)
     if ((valid_sh[0] & valid_sh[1]) != 0xFFFFFFFFu) {
@@ -380,13 +395,12 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     if (!ok) break;
     fence_after_sync();
     if (tid == 0 && item + (int)gridDim.x < nitems) {   // the T_b and V tiles are free
-      const ItemPos nx = locate_item(p, spans, cbase, item + gridDim.x, h0, Hg);
       if (kStage) {            // next item's log_alpha
-        stage_la(nx.h, nx.c0);
+        stage_la(nx.ip.h, nx.ip.c0);
       } else {                   // next item's V
         mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
-        tma_load_3d(sV, &vmap, 0, nx.h, nx.c0, &v_bar);
-        tma_load_3d(sV + 64 * 128, &vmap, 64, nx.h, nx.c0, &v_bar);
+        tma_load_3d(sV, &vmap, 0, nx.ip.h, nx.ip.c0, &v_bar);
+        tma_load_3d(sV + 64 * 128, &vmap, 64, nx.ip.h, nx.ip.c0, &v_bar);
       }
     }
     if ((warp & 3) < 2) {
