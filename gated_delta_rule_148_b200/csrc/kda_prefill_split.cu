@@ -260,6 +260,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   Ahead nx = read_ahead(blockIdx.x);
   for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
     const Ahead cur = nx;
+    if (item + (int)gridDim.x < nitems) nx = read_ahead(item + gridDim.x);   // loads overlap this item
     const ItemPos ip = cur.ip;
     const int h = ip.h, c0 = ip.c0;
     unsigned char *it = items + ip.off;
@@ -361,7 +362,6 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
-    if (item + (int)gridDim.x < nitems) nx = read_ahead(item + gridDim.x);
     if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {
       // T is packed and A is consumed: next item's q into the T tile, k into the A region
       fence_async_smem();
