@@ -161,12 +161,13 @@ struct IntraMaps {
 // T_b and V tiles (32 KB) once the W and U_v products have read them.  V follows
 // once the prep has read the staged rows.  (The plain per-thread
 // loads this replaces were held up by the number of misses an SM keeps in flight.)
-// With the head-wise gate (4 bytes of gate per row) the inputs are plain loads.
+// With the head-wise gate (4 bytes of gate per row) log_alpha is read by plain loads and
+// V has its tile from the start of the item; q and k are staged the same way.
 template <bool GATE_HEAD>     // log_alpha [N, H] (one gate per token and head) instead of [N, H, dk]
 __global__ void __launch_bounds__(kThreadsA, 2)
 intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqSpan *spans,
              const int *cbase, unsigned char *items, int h0, int Hg) {
-  constexpr bool kStage = !GATE_HEAD;
+  constexpr bool kStage = !GATE_HEAD;     // log_alpha staged (q and k always are)
   const CUtensorMap &vmap = maps.v;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t tmem_base_sh;
@@ -195,7 +196,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
     mbar_init(&v_bar, 1);
-    mbar_init(&in_bar, 3);
+    mbar_init(&in_bar, kStage ? 3 : 2);
   }
   for (int e = tid; e < 64 * 8; e += kThreadsA) {     // rows 64..127 of [T_b | 0] = 0, for good
     const int r = 64 + (e >> 3), ch = e & 7;
@@ -230,10 +231,10 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   // the V tile, so its copy overlaps that item's read-out and stores.
   if (tid == 0 && (int)blockIdx.x < nitems) {
     const ItemPos ip = locate_item(p, spans, cbase, blockIdx.x, h0, Hg);
+    stage_q(ip.h, ip.c0);
+    stage_k(ip.h, ip.c0);
     if (kStage) {
-      stage_q(ip.h, ip.c0);
       stage_la(ip.h, ip.c0);
-      stage_k(ip.h, ip.c0);
     } else {
       mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
       tma_load_3d(sV, &vmap, 0, ip.h, ip.c0, &v_bar);
@@ -271,13 +272,9 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
     }
     if (tid < 4) unsafe_sh[tid] = 0u;
-    if (kStage) {
-      ok = wait_all(&in_bar, iphase & 1, p, 4);
-      iphase++;
-      if (!ok) break;
-    } else {
-      __syncthreads();
-    }
+    ok = wait_all(&in_bar, iphase & 1, p, 4);
+    iphase++;
+    if (!ok) break;
     // ---- decay products and operand tiles (q, k from global memory; log_alpha staged or
     //      from global memory; V is already on its way or follows)
     {
@@ -291,8 +288,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
           c0, h, H, valid_sh, t, nullptr, base + A_TS, reinterpret_cast<float *>(it + IT_GC), part_sh,
           decay_sh, beta_val, beta_sh, xrows, tid, !first,
           kStage ? reinterpret_cast<const float *>(base + A_TB) : nullptr,
-          kStage ? reinterpret_cast<const uint16_t *>(base + A_TS) : nullptr,
-          kStage ? reinterpret_cast<const uint16_t *>(base + A_KH) : nullptr);
+          reinterpret_cast<const uint16_t *>(base + A_TS), reinterpret_cast<const uint16_t *>(base + A_KH));
     }
     if (kStage) {
       // the staged rows are read: rows 64..127 of [T_b | 0] back to zero, V into its tile
@@ -362,7 +358,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
-    if (kStage && tid == 0 && item + (int)gridDim.x < nitems) {
+    if (tid == 0 && item + (int)gridDim.x < nitems) {
       // T is packed and A is consumed: next item's q into the T tile, k into the A region
       fence_async_smem();
       stage_q(nx.ip.h, nx.ip.c0);
@@ -430,7 +426,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   if (!ok) {
     if (tid == 0) atomicOr(p.err, ERR_BIT_TIMEOUT);
     mbar_wait(&v_bar, (vphase - 0) & 1, 20000);
-    if (kStage) mbar_wait(&in_bar, iphase & 1, 20000);
+    mbar_wait(&in_bar, iphase & 1, 20000);
     if (phase > 0) mbar_wait(&mma_bar, (phase - 1) & 1, p.wait_cycles);
   }
   if (tid == 0) {
@@ -806,13 +802,14 @@ cudaError_t launch_split_items(const PrefillParams &p, const SeqSpan *spans, int
   if (!encode_3d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.v, p.dv, p.H, p.N, kNV,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
+  if (!encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
   if (p.gate_head) {
-    maps.la = maps.q = maps.k = maps.v;      // not used: with the head-wise gate the inputs are plain loads
+    maps.la = maps.v;      // not used: the head-wise gate (4 bytes a row) is read by plain loads
   } else if (!encode_3d(&maps.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.log_alpha, kDK, p.H, p.N, kDK,
-                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
-             !encode_3d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kDK, p.H, p.N, kDK,
-                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
-             !encode_3d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.k, kDK, p.H, p.N, kDK,
                         CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return cudaErrorNotSupported;
   }
