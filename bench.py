@@ -576,7 +576,7 @@ def bench_backward(K, W, world, device, pk, T=4096):
             "ms": ms, "algorithmic_bytes": nb,
             "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"]},
-            "note": "blockwise fp32 backward on CUDA cores (chunks of 64); its workspace traffic (chunk "
+            "note": "blockwise backward (chunks of 64), fp32 accuracy: dense products in 3xTF32 on tensor cores, the rest on CUDA cores; its workspace traffic (chunk "
                     "quantities, states at chunk starts and ends) is not algorithmic bytes"}
 
 

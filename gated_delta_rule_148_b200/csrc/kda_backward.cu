@@ -610,9 +610,66 @@ dstates_kernel(BackwardParams p, const int *cbase, const float *items, float *ds
 // thread, in registers), dM = dO U^T and dO-part of dT_b = dU V^T (4 x 4 blocks), dgamma.
 // W, K~, M, T of the chunk stay in shared memory.  Phase 2 (shared memory reused): the
 // chain through T, the pairwise terms with one thread per channel, log_alpha's sums.
+// 3xTF32 tensor-core product (mma.sync m16n8k8, fp32 accumulate): each fp32 operand is
+// split x = hi + lo with hi = tf32(x), lo = tf32(x - hi), and d += ah bh + ah bl + al bh
+// (the dropped al bl is below 2^-21 of the product), so the sums keep fp32 accuracy.
+// Fragment layout (g = lane / 4, t = lane % 4): A a0 = X[g][t], a1 = X[g+8][t],
+// a2 = X[g][t+4], a3 = X[g+8][t+4]; B b0 = Y[t][g], b1 = Y[t+4][g]; C c0 = C[g][2t],
+// c1 = C[g][2t+1], c2 = C[g+8][2t], c3 = C[g+8][2t+1].
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+__device__ __forceinline__ void mma_tf32_acc(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
+                                          const uint32_t (&bh)[2], const uint32_t (&bl)[2]) {
+  mma_tf32_acc(d, ah, bl);
+  mma_tf32_acc(d, al, bh);
+  mma_tf32_acc(d, ah, bh);
+}
+// B fragment (k0 + t, k0 + t + 4; n = n0 + g) of B[k][n] = X[n][k] (X row-major [.][ld]), split.
+__device__ __forceinline__ void load_bt_split(const float *X, int ld, int n0, int k0, int g, int t,
+                                              uint32_t (&h)[2], uint32_t (&l)[2]) {
+  split_tf32(X[(n0 + g) * ld + k0 + t], h[0], l[0]);
+  split_tf32(X[(n0 + g) * ld + k0 + t + 4], h[1], l[1]);
+}
+// B fragment of B[k][n] = X[k][n] (X row-major [.][ld]), split.
+__device__ __forceinline__ void load_b_split(const float *X, int ld, int n0, int k0, int g, int t,
+                                             uint32_t (&h)[2], uint32_t (&l)[2]) {
+  split_tf32(X[(k0 + t) * ld + n0 + g], h[0], l[0]);
+  split_tf32(X[(k0 + t + 4) * ld + n0 + g], h[1], l[1]);
+}
+// A fragment of A[r][k] = X[k][r] (X row-major [.][ld]), split; with LOWER, only entries of
+// the lower triangle of X (k >= r) are taken, the rest count as 0.
+template <bool LOWER>
+__device__ __forceinline__ void load_at_split(const float *X, int ld, int r0, int k0, int g, int t,
+                                              uint32_t (&h)[4], uint32_t (&l)[4]) {
+  const int rr[4] = {r0 + g, r0 + g + 8, r0 + g, r0 + g + 8};
+  const int kc[4] = {k0 + t, k0 + t, k0 + t + 4, k0 + t + 4};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x = (!LOWER || kc[e] >= rr[e]) ? X[kc[e] * ld + rr[e]] : 0.f;
+    split_tf32(x, h[e], l[e]);
+  }
+}
+// A fragment rows r0, r0 + 8 and columns k0 + t, k0 + t + 4 of a row-major [.][ld] tile, split.
+__device__ __forceinline__ void load_a_split(const float *X, int ld, int r0, int k0, int t, uint32_t (&h)[4],
+                                             uint32_t (&l)[4]) {
+  split_tf32(X[r0 * ld + k0 + t], h[0], l[0]);
+  split_tf32(X[(r0 + 8) * ld + k0 + t], h[1], l[1]);
+  split_tf32(X[r0 * ld + k0 + t + 4], h[2], l[2]);
+  split_tf32(X[(r0 + 8) * ld + k0 + t + 4], h[3], l[3]);
+}
+
 template <int DK, int DV>
 struct GradSmem {
-  static constexpr int LD = DK + 4, SPI = NS + 1, SPC = DK + 4;
+  static constexpr int LD = DK + 4, SPI = NS + 4, SPC = DK + 4;
   // phase 1 (T at 0 throughout)
   static constexpr int T0 = 0;
   static constexpr int W1 = T0 + C * LP, K1 = W1 + C * LD, M1 = K1 + C * LD;
@@ -764,19 +821,25 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
     Ts[(e / C) * LP + e % C] = it[IT::T + e];
   }
   if (tid < DK) dgam[tid] = 0.f;
-  // register accumulators: rows rb*4 .. +3 and channels cbk*CW .. +CW-1 of dQg, dK~, dW;
-  // rows (tid & 15)*4 .. +3 and columns (tid >> 4)*4 .. +3 of dM and dT_b
+  // rows i0 .. i0 + 3 and channels c0 .. c0 + CW - 1: the thread's share of the d(K e^g) product
+  // (phase 2); rows (tid & 15) * 4 .. and columns (tid >> 4) * 4 .. of dT_b there
   const int rb = tid >> 4, cbk = tid & 15, i0 = rb * 4, c0 = cbk * CW;
   const int mi0 = (tid & 15) * 4, mj0 = (tid >> 4) * 4;
-  float aq[4][CW], ak[4][CW], aw[4][CW], am[4][4], at[4][4];
+  // tensor-core accumulators over the d_v slices: warp wq owns n-tiles wq NTW .. of dQg, dK~
+  // and dW (columns of 8 channels) and n-tile wq of dM and dT_b (columns of 8 rows), all four
+  // 16-row m-tiles
+  constexpr int NTW = DK / 64;
+  const int lane = tid & 31, wq = tid >> 5, fg = lane >> 2, ft4 = lane & 3;
+  float fq[4][NTW][4], fk[4][NTW][4], fw[4][NTW][4], fm[4][4], ft[4][4];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
+  for (int m = 0; m < 4; ++m) {
 #pragma unroll
-    for (int u = 0; u < CW; ++u) aq[a][u] = ak[a][u] = aw[a][u] = 0.f;
+    for (int e = 0; e < 4; ++e) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) am[a][u] = at[a][u] = 0.f;
+      for (int nt = 0; nt < NTW; ++nt) fq[m][nt][e] = fk[m][nt][e] = fw[m][nt][e] = 0.f;
+      fm[m][e] = ft[m][e] = 0.f;
+    }
   }
-  const int nl = tid & 7, i2 = (tid >> 3) * 2;
   for (int n0 = 0; n0 < DV; n0 += NS) {
     __syncthreads();     // previous slice's readers are done
     load_rows<false, DK, NS, false>(Sg, n0, DV, 0, tid, [&](int c, int n, float x) { sS[n * SPC + c] = x; });
@@ -787,114 +850,112 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
                            [&](int r, int n, float x) { sV[r * SPI + n] = x; });
     tc::cp_async_wait_all();
     __syncthreads();
-    {   // U = U_v - W S and dU = M^T dO + K~ dS' (rows i2, i2 + 1; columns nl + 8 bb: lanes
-        // read neighbouring rows of S, so the float4 reads fall in distinct banks)
-      float u[2][4], du[2][4];
+    // U = U_v - W S, dU = M^T dO + K~ dS' and then dV = T_b^T dU on the tensor cores (3xTF32):
+    // 64 x NS each, warp wq the 16-row m-tile wq / 2 and the two 8-column n-tiles of half wq % 2
+    {
+      const int r0 = (wq >> 1) * 16, nb0 = (wq & 1) * 16;
+      float fu[2][4], fd[2][4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+      for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          u[a][bb] = __ldg(it + IT::UV + (size_t)(i2 + a) * DV + n0 + nl + 8 * bb);
-          du[a][bb] = 0.f;
-        }
-      for (int c = 0; c < DK; c += 4) {
-        const float4 w0 = *reinterpret_cast<const float4 *>(Wt + i2 * LD + c);
-        const float4 w1 = *reinterpret_cast<const float4 *>(Wt + (i2 + 1) * LD + c);
-        const float4 k0 = *reinterpret_cast<const float4 *>(Kt + i2 * LD + c);
-        const float4 k1 = *reinterpret_cast<const float4 *>(Kt + (i2 + 1) * LD + c);
-        const float wa[2][4] = {{w0.x, w0.y, w0.z, w0.w}, {w1.x, w1.y, w1.z, w1.w}};
-        const float ka[2][4] = {{k0.x, k0.y, k0.z, k0.w}, {k1.x, k1.y, k1.z, k1.w}};
+        for (int e = 0; e < 4; ++e) fu[nb][e] = fd[nb][e] = 0.f;
+#pragma unroll 4
+      for (int k0 = 0; k0 < DK; k0 += 8) {
+        uint32_t awh[4], awl[4], akh[4], akl[4];
+        load_a_split(Wt, LD, r0 + fg, k0, ft4, awh, awl);
+        load_a_split(Kt, LD, r0 + fg, k0, ft4, akh, akl);
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const float4 sv = *reinterpret_cast<const float4 *>(sS + (nl + 8 * bb) * SPC + c);
-          const float4 dv = *reinterpret_cast<const float4 *>(sdS + (nl + 8 * bb) * SPC + c);
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            u[a][bb] -= wa[a][0] * sv.x + wa[a][1] * sv.y + wa[a][2] * sv.z + wa[a][3] * sv.w;
-            du[a][bb] += ka[a][0] * dv.x + ka[a][1] * dv.y + ka[a][2] * dv.z + ka[a][3] * dv.w;
-          }
+        for (int nb = 0; nb < 2; ++nb) {
+          uint32_t bh[2], bl[2];
+          load_bt_split(sS, SPC, nb0 + nb * 8, k0, fg, ft4, bh, bl);
+          mma3_tf32(fu[nb], awh, awl, bh, bl);
+          load_bt_split(sdS, SPC, nb0 + nb * 8, k0, fg, ft4, bh, bl);
+          mma3_tf32(fd[nb], akh, akl, bh, bl);
         }
       }
-      for (int r = i2; r < C; ++r) {
-        const float m0 = Mt[r * LP + i2], m1 = Mt[r * LP + i2 + 1];
+#pragma unroll 4
+      for (int k0 = 0; k0 < C; k0 += 8) {
+        uint32_t amh[4], aml[4];
+        load_at_split<false>(Mt, LP, r0, k0, fg, ft4, amh, aml);   // M is stored lower-triangular
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const float d = sdO[r * SPI + nl + 8 * bb];
-          du[0][bb] = fmaf(m0, d, du[0][bb]);
-          du[1][bb] = fmaf(m1, d, du[1][bb]);
+        for (int nb = 0; nb < 2; ++nb) {
+          uint32_t bh[2], bl[2];
+          load_b_split(sdO, SPI, nb0 + nb * 8, k0, fg, ft4, bh, bl);
+          mma3_tf32(fd[nb], amh, aml, bh, bl);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+      for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          sU[(i2 + a) * SPI + nl + 8 * bb] = u[a][bb];
-          sdU[(i2 + a) * SPI + nl + 8 * bb] = du[a][bb];
+        for (int e = 0; e < 4; ++e) {
+          const int r = r0 + fg + (e >> 1) * 8, cc = nb0 + nb * 8 + 2 * ft4 + (e & 1);
+          sU[r * SPI + cc] = __ldg(it + IT::UV + (size_t)r * DV + n0 + cc) - fu[nb][e];
+          sdU[r * SPI + cc] = fd[nb][e];
         }
-    }
-    __syncthreads();
-    {   // dV = T_b^T dU (rows i2, i2 + 1 as jr)
-      float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      for (int i = i2; i < C; ++i) {
-        const float t0 = Ts[i * LP + i2], t1 = Ts[i * LP + i2 + 1];
+      __syncthreads();
+      float fv[2][4];
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const float d = sdU[i * SPI + nl + 8 * bb];
-          dv[0][bb] = fmaf(t0, d, dv[0][bb]);
-          dv[1][bb] = fmaf(t1, d, dv[1][bb]);
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) fv[nb][e] = 0.f;
+#pragma unroll 4
+      for (int k0 = 0; k0 < C; k0 += 8) {
+        uint32_t ath[4], atl[4];
+        load_at_split<true>(Ts, LP, r0, k0, fg, ft4, ath, atl);      // T: lower triangle only
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          uint32_t bh[2], bl[2];
+          load_b_split(sdU, SPI, nb0 + nb * 8, k0, fg, ft4, bh, bl);
+          mma3_tf32(fv[nb], ath, atl, bh, bl);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        const int jr = i2 + a;
+      for (int e = 0; e < 4; ++e) {
+        const int jr = r0 + fg + (e >> 1) * 8;
         if (jr < cp.n) {
           const float bj = betaf(jr);
-          float *dst = p.gv + ((size_t)(cp.r0 + jr) * H + h) * DV + n0 + nl;
+          float *dst = p.gv + ((size_t)(cp.r0 + jr) * H + h) * DV + n0 + nb0 + 2 * ft4 + (e & 1);
 #pragma unroll
-          for (int bb = 0; bb < 4; ++bb) dst[8 * bb] = dv[a][bb] * bj;
+          for (int nb = 0; nb < 2; ++nb) dst[nb * 8] = fv[nb][e] * bj;
         }
       }
     }
-    // d_k-side shares of this slice
-#pragma unroll 2
-    for (int nn = 0; nn < NS; ++nn) {
-      float ro[4], ru[4], rd[4], cs[CW], cd[CW];
+    // d_k-side shares of this slice on the tensor cores (3xTF32, K = the slice's NS columns):
+    //   dQg += dO S^T, dK~ += U dS'^T, dW -= dU S^T (B = the slice of S or dS', [NS][DK]),
+    //   dM += dO U^T, dT_b += dU V^T (B = U or V read transposed)
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        ro[a] = sdO[(i0 + a) * SPI + nn];
-        ru[a] = sU[(i0 + a) * SPI + nn];
-        rd[a] = sdU[(i0 + a) * SPI + nn];
+    for (int kk = 0; kk < NS; kk += 8) {
+      uint32_t bsh[NTW][2], bsl[NTW][2], bdh[NTW][2], bdl[NTW][2], buh[2], bul[2], bvh[2], bvl[2];
+#pragma unroll
+      for (int nt = 0; nt < NTW; ++nt) {
+        const int n = (wq * NTW + nt) * 8 + fg;
+        split_tf32(sS[(kk + ft4) * SPC + n], bsh[nt][0], bsl[nt][0]);
+        split_tf32(sS[(kk + ft4 + 4) * SPC + n], bsh[nt][1], bsl[nt][1]);
+        split_tf32(sdS[(kk + ft4) * SPC + n], bdh[nt][0], bdl[nt][0]);
+        split_tf32(sdS[(kk + ft4 + 4) * SPC + n], bdh[nt][1], bdl[nt][1]);
+      }
+      {
+        const int j = wq * 8 + fg;
+        split_tf32(sU[j * SPI + kk + ft4], buh[0], bul[0]);
+        split_tf32(sU[j * SPI + kk + ft4 + 4], buh[1], bul[1]);
+        split_tf32(sV[j * SPI + kk + ft4], bvh[0], bvl[0]);
+        split_tf32(sV[j * SPI + kk + ft4 + 4], bvh[1], bvl[1]);
       }
 #pragma unroll
-      for (int u = 0; u < CW; u += 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(sS + nn * SPC + c0 + u);
-        const float4 y = *reinterpret_cast<const float4 *>(sdS + nn * SPC + c0 + u);
-        cs[u] = x.x; cs[u + 1] = x.y; cs[u + 2] = x.z; cs[u + 3] = x.w;
-        cd[u] = y.x; cd[u + 1] = y.y; cd[u + 2] = y.z; cd[u + 3] = y.w;
-      }
+      for (int m = 0; m < 4; ++m) {
+        uint32_t aoh[4], aol[4], auh[4], aul[4], adh[4], adl[4];
+        load_a_split(sdO, SPI, m * 16 + fg, kk, ft4, aoh, aol);
+        load_a_split(sU, SPI, m * 16 + fg, kk, ft4, auh, aul);
+        load_a_split(sdU, SPI, m * 16 + fg, kk, ft4, adh, adl);
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int u = 0; u < CW; ++u) {
-          aq[a][u] = fmaf(ro[a], cs[u], aq[a][u]);
-          ak[a][u] = fmaf(ru[a], cd[u], ak[a][u]);
-          aw[a][u] = fmaf(-rd[a], cs[u], aw[a][u]);
+        for (int nt = 0; nt < NTW; ++nt) {
+          mma3_tf32(fq[m][nt], aoh, aol, bsh[nt], bsl[nt]);
+          mma3_tf32(fk[m][nt], auh, aul, bdh[nt], bdl[nt]);
+          mma3_tf32(fw[m][nt], adh, adl, bsh[nt], bsl[nt]);
         }
-      float mo[4], md[4], mu[4], mv[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        mo[a] = sdO[(mi0 + a) * SPI + nn];
-        md[a] = sdU[(mi0 + a) * SPI + nn];
-        mu[a] = sU[(mj0 + a) * SPI + nn];
-        mv[a] = sV[(mj0 + a) * SPI + nn];
+        mma3_tf32(fm[m], aoh, aol, buh, bul);
+        mma3_tf32(ft[m], adh, adl, bvh, bvl);
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          am[a][bb] = fmaf(mo[a], mu[bb], am[a][bb]);
-          at[a][bb] = fmaf(md[a], mv[bb], at[a][bb]);
-        }
     }
     if (tid < DK) {
       float s = 0.f;
@@ -908,18 +969,33 @@ grad_kernel(BackwardParams p, const int *cbase, const float *items, const float 
   float *dQg = sm + G::DQG, *dKt = sm + G::DKT, *dW = sm + G::DW;
   float *dM = sm + G::DM, *dTb = sm + G::DTB, *gT = sm + G::GT, *kb = sm + G::KB, *dgC = sm + G::DGC;
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
+  for (int m = 0; m < 4; ++m) {
+    const int r = m * 16 + fg;
 #pragma unroll
-    for (int u = 0; u < CW; ++u) {
-      dQg[(i0 + a) * DK + c0 + u] = aq[a][u];
-      dKt[(i0 + a) * DK + c0 + u] = ak[a][u];
-      dW[(i0 + a) * DK + c0 + u] = aw[a][u];
+    for (int nt = 0; nt < NTW; ++nt) {
+      const int c = (wq * NTW + nt) * 8 + 2 * ft4;
+      dQg[r * DK + c] = fq[m][nt][0];
+      dQg[r * DK + c + 1] = fq[m][nt][1];
+      dQg[(r + 8) * DK + c] = fq[m][nt][2];
+      dQg[(r + 8) * DK + c + 1] = fq[m][nt][3];
+      dKt[r * DK + c] = fk[m][nt][0];
+      dKt[r * DK + c + 1] = fk[m][nt][1];
+      dKt[(r + 8) * DK + c] = fk[m][nt][2];
+      dKt[(r + 8) * DK + c + 1] = fk[m][nt][3];
+      dW[r * DK + c] = -fw[m][nt][0];
+      dW[r * DK + c + 1] = -fw[m][nt][1];
+      dW[(r + 8) * DK + c] = -fw[m][nt][2];
+      dW[(r + 8) * DK + c + 1] = -fw[m][nt][3];
     }
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb) {
-      dM[(mi0 + a) * LP + mj0 + bb] = (mj0 + bb <= mi0 + a) ? am[a][bb] : 0.f;
-      dTb[(mi0 + a) * LP + mj0 + bb] = at[a][bb];
-    }
+    const int j = wq * 8 + 2 * ft4;
+    dM[r * LP + j] = (j <= r) ? fm[m][0] : 0.f;
+    dM[r * LP + j + 1] = (j + 1 <= r) ? fm[m][1] : 0.f;
+    dM[(r + 8) * LP + j] = (j <= r + 8) ? fm[m][2] : 0.f;
+    dM[(r + 8) * LP + j + 1] = (j + 1 <= r + 8) ? fm[m][3] : 0.f;
+    dTb[r * LP + j] = ft[m][0];
+    dTb[r * LP + j + 1] = ft[m][1];
+    dTb[(r + 8) * LP + j] = ft[m][2];
+    dTb[(r + 8) * LP + j + 1] = ft[m][3];
   }
   load_rows<BF16, C, DK>(p.k, first * DK, (size_t)H * DK, vmask, tid, [&](int r, int c, float x) { kb[r * KP + c] = x; });
   load_gates<DK>(p, cp, h, vmask, gT, tid);
