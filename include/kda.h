@@ -266,7 +266,9 @@ kda_status kda_short_conv(const kda_conv_args *args, void *stream);
  * log_alpha <= 0) and every gradient of a chunk's rows are computed for all
  * chunks in parallel; only the state at each chunk start (forward) and its
  * gradient at each chunk end (backward) are chained over a sequence's chunks.
- * fp32 on CUDA cores.
+ * fp32 accuracy throughout: the gradient kernel's dense products run on the tensor
+ * cores with each fp32 operand split into two tf32 parts (three products), the
+ * rest on CUDA cores in fp32.
  * Fields (device pointers, caller-owned):
  *   dtype, num_seqs, total_tokens, H, dk, dv, q, k, v, log_alpha, beta,
  *   cu_seqlens, pad_mask, init_state, gate   as for kda_prefill (chunk is not
