@@ -21,7 +21,8 @@
 // (sequence, head, 32 columns of d_v), the forward chain that stores the state at
 // every chunk start; (3) the same CTAs walking the chunks backwards for dS' at every
 // chunk end (and dS_0); (4) per (chunk, head), every gradient of the chunk's rows.
-// Only (2) and (3) are serial over a sequence's chunks.  fp32 on CUDA cores.
+// Only (2) and (3) are serial over a sequence's chunks.  fp32 throughout; in (4) the
+// dense products of each d_v slice run on the tensor cores in 3xTF32 (fp32 accuracy).
 // Pads are identity steps (their inputs never read): zero gradients there.
 #include "kda_internal.cuh"
 #include "kda_tc.cuh"
