@@ -95,9 +95,9 @@ __global__ void __launch_bounds__(1024) chunk_index_kernel(PrefillParams p, cons
 // Persistent: about two CTAs per SM loop over the (chunk, head) items, so the
 // TMEM allocation, barrier set-up and constant tiles are paid once per CTA.
 // ~100 KB of shared memory lets two CTAs share an SM and hide each other's load
-// and tensor-core latency.  q, k, log_alpha are read straight from global
-// memory, V arrives by TMA; the item's tiles leave through shared memory with
-// bulk stores.
+// and tensor-core latency.  q, k, log_alpha and V arrive by TMA one item ahead
+// (staged in tiles the current item no longer needs); the item's tiles leave
+// through shared memory with bulk stores, U_v and M by direct stores.
 constexpr int kThreadsA = 256;
 constexpr uint32_t A_QK = 0;                        // [Q G | K G] 128 x 128 row tile; then [-W | .]
 constexpr uint32_t A_KH = A_QK + 128 * 256;         // K e^{-g} 64 x 128; then A [64][65] f32; then U_v
@@ -173,7 +173,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ __align__(8) uint64_t v_bar;
-  __shared__ __align__(8) uint64_t in_bar;     // the three staged inputs of an item
+  __shared__ __align__(8) uint64_t in_bar;     // an item's staged inputs: q, k (and log_alpha)
   __shared__ uint32_t valid_sh[2];
   __shared__ uint32_t unsafe_sh[4];     // channels with exact-path key rows
   __shared__ int tfirst_sh[128];        // their first exact-path key row
