@@ -243,19 +243,39 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   }
   bool first = true;
   // An item's position, span, row validity and beta (rows tid < 64) are read one item
-  // ahead, so the item starts without waiting on these global loads.
+  // ahead, so the item starts without waiting on these global loads.  The sequence of
+  // the last item looked up (its chunk range and span) stays in registers, so while the
+  // items stay in one sequence their positions need no load at all; beta is loaded for
+  // row min(c0 + tid, N - 1) (always in bounds) and masked by the row's validity only
+  // where it is used, an item later, so no instruction here waits for a load.
   struct Ahead {
     ItemPos ip;
     SeqSpan sp;
     bool vr;
-    float beta;
+    float beta;     // not yet masked by vr
   };
+  int seq_lo = 0, seq_hi = -1;      // global chunk range [seq_lo, seq_hi) of sequence seq_b
+  int seq_b = 0;
+  SeqSpan seq_sp{0, 0};
   auto read_ahead = [&](int item) {
     Ahead a;
-    a.ip = locate_item(p, spans, cbase, item, h0, Hg);
-    a.sp = spans[a.ip.b];
+    const int gchunk = item / Hg;
+    if (gchunk < seq_lo || gchunk >= seq_hi) {
+      a.ip = locate_item(p, spans, cbase, item, h0, Hg);
+      seq_b = a.ip.b;
+      seq_lo = cbase[seq_b];
+      seq_hi = cbase[seq_b + 1];
+      seq_sp = spans[seq_b];
+    } else {
+      a.ip.b = seq_b;
+      a.ip.h = h0 + item % Hg;
+      a.ip.c0 = seq_sp.begin + (gchunk - seq_lo) * kC;
+      a.ip.off = ((size_t)gchunk * p.H + a.ip.h) * ITEM_BYTES;
+    }
+    a.sp = seq_sp;
     a.vr = tid < kC && row_ok(p, a.sp, a.ip.c0 + tid);
-    a.beta = a.vr ? __ldg(p.beta + (size_t)(a.ip.c0 + tid) * H + a.ip.h) : 0.f;
+    a.beta = 0.f;
+    if (tid < kC) a.beta = __ldg(p.beta + (size_t)min(a.ip.c0 + tid, p.N - 1) * H + a.ip.h);
     return a;
   };
   Ahead nx = read_ahead(blockIdx.x);
@@ -266,7 +286,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     const int h = ip.h, c0 = ip.c0;
     unsigned char *it = items + ip.off;
 
-    const float beta_val = cur.beta;   // stored to shared memory inside the prep, after its loads
+    const float beta_val = cur.vr ? cur.beta : 0.f;   // stored to shared memory inside the prep
     if (tid < kC) {
       const unsigned bits = __ballot_sync(0xFFFFFFFFu, cur.vr);
       if ((tid & 31) == 0) valid_sh[tid >> 5] = bits;
