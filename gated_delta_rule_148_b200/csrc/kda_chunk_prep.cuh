@@ -59,6 +59,11 @@ __device__ __forceinline__ float kh_entry(float k, float eg, int r, int c, const
   return 0.f;
 }
 
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
 struct PrepTiles {
   unsigned char *qg;      // Q G rows (K-major row tile `qg_R` rows, starting row `qg_row0`)
   int qg_R, qg_row0;
@@ -236,22 +241,41 @@ __device__ __forceinline__ void decay_and_tiles_global(
   const uint32_t col128 = (uint32_t)(kb * 128 * 128 + (c & 7) * 2);
   const uint32_t col64 = (uint32_t)(kb * 64 * 128 + (c & 7) * 2);
   float e0 = pre0, e1 = pre1;
+  // e^{g} never increases down the rows (every alpha <= 1), so when this thread's last row
+  // is well above the range threshold (the factor 2 covers the rounding of pre * t against
+  // the running product), every row passes the range test: it is skipped, same values.
+  auto rows = [&](auto fast) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = qt * 16 + i;
-    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
-    const float qa = __uint_as_float(qv[i] << 16), qb = __uint_as_float(qv[i] & 0xFFFF0000u);
-    const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
-    e0 *= a0[i];
-    e1 *= a1[i];
-    const uint32_t qgv = pack_bf16x2(qa * e0, qb * e1);
-    *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
-    if (gq) *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
-    *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
-        pack_bf16x2(ka * e0, kb2 * e1);
-    *reinterpret_cast<uint32_t *>(t.kh + col64 + (uint32_t)(r * 128) + sw) =
-        pack_bf16x2(kh_entry(ka, e0, r, c, xr, mk0), kh_entry(kb2, e1, r, c + 1, xr, mk1));
-  }
+    for (int i = 0; i < 16; ++i) {
+      const int r = qt * 16 + i;
+      const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
+      const float qa = __uint_as_float(qv[i] << 16), qb = __uint_as_float(qv[i] & 0xFFFF0000u);
+      const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
+      e0 *= a0[i];
+      e1 *= a1[i];
+      const uint32_t qgv = pack_bf16x2(qa * e0, qb * e1);
+      *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
+      if (gq) *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
+      *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
+          pack_bf16x2(ka * e0, kb2 * e1);
+      float h0, h1;
+      if constexpr (decltype(fast)::value) {
+        float v0, v1;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(v0) : "f"(e0));
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(v1) : "f"(e1));
+        h0 = ka * v0;
+        h1 = kb2 * v1;
+      } else {
+        h0 = kh_entry(ka, e0, r, c, xr, mk0);
+        h1 = kh_entry(kb2, e1, r, c + 1, xr, mk1);
+      }
+      *reinterpret_cast<uint32_t *>(t.kh + col64 + (uint32_t)(r * 128) + sw) = pack_bf16x2(h0, h1);
+    }
+  };
+  if (pre0 * t0 > 2.f * kFastMinDecay && pre1 * t1 > 2.f * kFastMinDecay)
+    rows(BoolTag<true>{});
+  else
+    rows(BoolTag<false>{});
   float s0 = suf0, s1 = suf1;
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
