@@ -328,15 +328,28 @@ __device__ __forceinline__ void extract_gram(uint32_t tm_cols, unsigned char *mt
   }
 }
 
-// T_b = T Diag(beta) (lower part of T in Ts [64][65] f32) -> bf16 rows 0..63 of `ttile` (R rows).
+// T_b = T Diag(beta) (lower part of T in Ts [64][LDT] f32) -> bf16 rows 0..63 of `ttile` (R rows).
+// With LDT a multiple of 4 the row is read 16 bytes at a time.
+template <int LDT = 65>
 __device__ __forceinline__ void pack_tb(const float *Ts, const float *beta, unsigned char *ttile,
                                         int R, int tid) {
   const int r = tid >> 2, qq = tid & 3;      // row r, columns 16qq .. 16qq+15
   float t[16];
+  if constexpr (LDT % 4 == 0) {
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int i = qq * 16 + u;
-    t[u] = (i <= r) ? Ts[r * 65 + i] * beta[i] : 0.f;
+    for (int u = 0; u < 16; u += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(Ts + r * LDT + qq * 16 + u);
+      const float4 b = *reinterpret_cast<const float4 *>(beta + qq * 16 + u);
+      const float xv[4] = {x.x * b.x, x.y * b.y, x.z * b.z, x.w * b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) t[u + e] = (qq * 16 + u + e <= r) ? xv[e] : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int i = qq * 16 + u;
+      t[u] = (i <= r) ? Ts[r * LDT + i] * beta[i] : 0.f;
+    }
   }
 #pragma unroll
   for (int j = 0; j < 16; j += 8) {

@@ -104,12 +104,13 @@ constexpr uint32_t A_KH = A_QK + 128 * 256;         // K e^{-g} 64 x 128; then A
 constexpr uint32_t A_TB = A_KH + 17 * 1024;         // [T_b | 0]     128 x 64 row tile
 constexpr uint32_t A_V = A_TB + 128 * 128;          // V  64 rows x 2 blocks of 64
 constexpr uint32_t A_TS = A_V + 64 * 256;           // K e^{g_C-g} 64 x 128 tile; then T [64][65] f32
-constexpr uint32_t A_XS = A_TS + 64 * 65 * 4;       // inverse scratch (32 x 33 f32)
+constexpr int kLDA = 68;                            // row stride of the A and T f32 tiles (16-byte rows)
+constexpr uint32_t A_XS = A_TS + 64 * kLDA * 4;     // inverse scratch (32 x 33 f32)
 constexpr uint32_t A_USED = A_XS + 32 * 33 * 4;
 constexpr uint32_t A_SMEM = A_USED + 1024;
 static_assert(A_TB % 1024 == 0 && A_V % 1024 == 0 && A_KH % 1024 == 0 && A_TS % 1024 == 0,
               "swizzled tiles are 1024-aligned");
-static_assert(64 * 65 * 4 <= A_TB - A_KH, "A fits the K e^{-g} region");
+static_assert(64 * kLDA * 4 <= A_TB - A_KH, "A fits the K e^{-g} region");
 constexpr uint32_t A_TM_GW = 0, A_TM_UV = 128, A_TM_COLS = 256;
 
 __device__ __forceinline__ bool row_ok(const PrefillParams &p, const SeqSpan &sp, int pos) {
@@ -179,7 +180,7 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   __shared__ int tfirst_sh[128];        // their first exact-path key row
   const prep::ExactRows xrows{unsafe_sh, tfirst_sh};
   __shared__ float decay_sh[kDK];
-  __shared__ float beta_sh[kC];
+  __shared__ __align__(16) float beta_sh[kC];   // read 16 bytes at a time by pack_tb
   __shared__ float part_sh[4][kDK];
 
   if (device_error_latched(p.err)) return;
@@ -364,16 +365,18 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
         const int r = lr - kC;
         const float br = beta_sh[r];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 32; j += 4) {
           const int i = wg * 32 + j;
-          As[r * 65 + i] = (i < r) ? br * v[j] : 0.f;
+          *reinterpret_cast<float4 *>(As + r * kLDA + i) =
+              make_float4(i < r ? br * v[j] : 0.f, i + 1 < r ? br * v[j + 1] : 0.f,
+                          i + 2 < r ? br * v[j + 2] : 0.f, i + 3 < r ? br * v[j + 3] : 0.f);
         }
       }
     }
     if (tid == 0) bulk_wait_read();     // K e^{g_C-g} has left the T region
     __syncthreads();
-    tri::unit_lower_inverse_64(As, Ts, Xs, tid);
-    prep::pack_tb(Ts, beta_sh, base + A_TB, 128, tid);
+    tri::unit_lower_inverse_64<kLDA>(As, Ts, Xs, tid);
+    prep::pack_tb<kLDA>(Ts, beta_sh, base + A_TB, 128, tid);
     fence_async_smem();
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;

@@ -21,7 +21,7 @@
 namespace kda {
 namespace tri {
 
-constexpr int LD = 65;
+constexpr int kLD = 65;     // default row stride of the [64][.] f32 tiles
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
@@ -80,6 +80,7 @@ __device__ __forceinline__ void store_acc(float *Z, int ldz, const float (&acc)[
 //   P0 = [[D0, 0], [-D1 A10 D0, D1]],  P1 = [[D2, 0], [-D3 A32 D2, D3]];
 // then the lower-left 32 x 32 block -P1 (A_LL P0), with one warp per 16 x 16
 // output tile.  The block products are tensor-core MMAs.
+template <int LD = kLD>      // row stride of As and Ts (floats)
 __device__ __forceinline__ void unit_lower_inverse_64(const float *__restrict__ As,
                                                       float *__restrict__ Ts,
                                                       float *__restrict__ scratch, int tid) {
