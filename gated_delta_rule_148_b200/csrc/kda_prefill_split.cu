@@ -312,14 +312,14 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
           reinterpret_cast<const uint16_t *>(base + A_TS), reinterpret_cast<const uint16_t *>(base + A_KH));
     }
     if (kStage) {
-      // the staged rows are read: rows 64..127 of [T_b | 0] back to zero, V into its tile
-      fence_async_smem();
-      __syncthreads();
+      // every thread read its staged rows before the prep's internal barrier: rows 64..127
+      // of [T_b | 0] back to zero, V into its tile
       for (int e = tid; e < 64 * 8; e += kThreadsA) {
         const int r = 64 + (e >> 3), ch = e & 7;
         *reinterpret_cast<uint4 *>(base + A_TB + row_tile_chunk(r, 0, ch, 128)) = make_uint4(0, 0, 0, 0);
       }
       if (tid == 0) {
+        fence_async_smem();
         mbar_arrive_expect_tx(&v_bar, 2 * 64 * 128);
         tma_load_3d(sV, &vmap, 0, h, c0, &v_bar);
         tma_load_3d(sV + 64 * 128, &vmap, 64, h, c0, &v_bar);
