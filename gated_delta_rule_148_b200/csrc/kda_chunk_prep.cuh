@@ -174,118 +174,143 @@ __device__ __forceinline__ void decay_and_tiles_global(
     float *gdecay, float (*part)[kDK], float *decay, float beta_val, float *beta_out,
     const ExactRows &xr, int tid, bool wait_bulk = false, const float *sla = nullptr,
     const uint16_t *sq = nullptr, const uint16_t *sk = nullptr) {
-  const int cp = tid & 63, qt = tid >> 6, c = 2 * cp;
-  const uint32_t vbits = valid[qt >> 1] >> ((qt & 1) * 16);
-  float a0[16], a1[16];
-  uint32_t qv[16], kv[16];
+  // thread: channels c .. c+3 (c = 4 (tid % 32)), rows 8 qt .. 8 qt + 7 (qt = tid / 32); 16-byte
+  // log_alpha and 8-byte q, k, tile accesses
+  const int cq = tid & 31, qt = tid >> 5, c = 4 * cq;
+  const uint32_t vbits = (valid[qt >> 2] >> ((qt & 3) * 8)) & 0xFFu;
+  float a[8][4];
+  uint2 qv[8], kv[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const bool vr = (vbits >> i) & 1u;
-    const size_t row = ((size_t)(c0 + qt * 16 + i) * H + h) * kDK + c;
-    float2 la = make_float2(0.f, 0.f);
-    qv[i] = 0u;
-    kv[i] = 0u;
+    const int rr = qt * 8 + i;
+    const size_t row = ((size_t)(c0 + rr) * H + h) * kDK + c;
+    float4 la = make_float4(0.f, 0.f, 0.f, 0.f);
+    qv[i] = make_uint2(0u, 0u);
+    kv[i] = make_uint2(0u, 0u);
     if (vr) {
       if (GATE_HEAD) {
-        const float gv = __ldg(log_alpha + (size_t)(c0 + qt * 16 + i) * H + h);
-        la = make_float2(gv, gv);
+        const float gv = __ldg(log_alpha + (size_t)(c0 + rr) * H + h);
+        la = make_float4(gv, gv, gv, gv);
       } else if (sla) {
-        la = *reinterpret_cast<const float2 *>(sla + (qt * 16 + i) * kDK + c);
+        la = *reinterpret_cast<const float4 *>(sla + rr * kDK + c);
       } else {
-        la = __ldg(reinterpret_cast<const float2 *>(log_alpha + row));
+        la = __ldg(reinterpret_cast<const float4 *>(log_alpha + row));
       }
       if (sq) {
-        qv[i] = *reinterpret_cast<const uint32_t *>(sq + (qt * 16 + i) * kDK + c);
-        kv[i] = *reinterpret_cast<const uint32_t *>(sk + (qt * 16 + i) * kDK + c);
+        qv[i] = *reinterpret_cast<const uint2 *>(sq + rr * kDK + c);
+        kv[i] = *reinterpret_cast<const uint2 *>(sk + rr * kDK + c);
       } else {
-        qv[i] = __ldg(reinterpret_cast<const unsigned int *>(q + row));
-        kv[i] = __ldg(reinterpret_cast<const unsigned int *>(k + row));
+        qv[i] = __ldg(reinterpret_cast<const uint2 *>(q + row));
+        kv[i] = __ldg(reinterpret_cast<const uint2 *>(k + row));
       }
     }
-    a0[i] = la.x;
-    a1[i] = la.y;
+    a[i][0] = la.x;
+    a[i][1] = la.y;
+    a[i][2] = la.z;
+    a[i][3] = la.w;
   }
-  float t0 = 1.f, t1 = 1.f;
+  float tt[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    a0[i] = __expf(a0[i]);
-    a1[i] = __expf(a1[i]);
-    t0 *= a0[i];
-    t1 *= a1[i];
-  }
-  part[qt][c] = t0;
-  part[qt][c + 1] = t1;
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      a[i][e] = __expf(a[i][e]);
+      tt[e] *= a[i][e];
+    }
+  *reinterpret_cast<float4 *>(&part[qt][c]) = make_float4(tt[0], tt[1], tt[2], tt[3]);
   if (tid < kC) beta_out[tid] = beta_val;
   if (tid < kDK) xr.tfirst[tid] = kC;
   // the tiles may still be read by bulk stores thread 0 issued earlier; the tile
   // writes below come after this barrier
   if (wait_bulk && tid == 0) tc::bulk_wait_read();
   __syncthreads();
-  float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
+  float pre[4] = {1.f, 1.f, 1.f, 1.f}, suf[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    const float x0 = part[qq][c], x1 = part[qq][c + 1];
-    if (qq < qt) { pre0 *= x0; pre1 *= x1; }
-    if (qq > qt) { suf0 *= x0; suf1 *= x1; }
+  for (int qq = 0; qq < 8; ++qq) {
+    const float4 x = *reinterpret_cast<const float4 *>(&part[qq][c]);
+    const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (qq < qt) pre[e] *= xv[e];
+      if (qq > qt) suf[e] *= xv[e];
+    }
   }
-  const float GC0 = pre0 * t0 * suf0, GC1 = pre1 * t1 * suf1;   // e^{g_C}
   if (qt == 0) {
-    decay[c] = GC0;
-    decay[c + 1] = GC1;
-    if (gdecay) *reinterpret_cast<float2 *>(gdecay + c) = make_float2(GC0, GC1);
+    const float4 gc = make_float4(pre[0] * tt[0] * suf[0], pre[1] * tt[1] * suf[1], pre[2] * tt[2] * suf[2],
+                                  pre[3] * tt[3] * suf[3]);   // e^{g_C}
+    *reinterpret_cast<float4 *>(decay + c) = gc;
+    if (gdecay) *reinterpret_cast<float4 *>(gdecay + c) = gc;
   }
-  bool mk0 = false, mk1 = false;
+  bool mk[4] = {false, false, false, false};
   const int kb = c >> 6, ch = (c & 63) >> 3;
   const uint32_t colq = (uint32_t)(kb * t.qg_R * 128 + (c & 7) * 2);
   const uint32_t colk = (uint32_t)(kb * t.kg_R * 128 + (c & 7) * 2);
   const uint32_t col128 = (uint32_t)(kb * 128 * 128 + (c & 7) * 2);
   const uint32_t col64 = (uint32_t)(kb * 64 * 128 + (c & 7) * 2);
-  float e0 = pre0, e1 = pre1;
+  auto unpack = [](uint2 w, float (&x)[4]) {
+    x[0] = __uint_as_float(w.x << 16);
+    x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(w.y << 16);
+    x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  };
+  auto pack4 = [](const float (&x)[4]) { return make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3])); };
+  float ev[4] = {pre[0], pre[1], pre[2], pre[3]};
   // e^{g} never increases down the rows (every alpha <= 1), so when this thread's last row
   // is well above the range threshold (the factor 2 covers the rounding of pre * t against
   // the running product), every row passes the range test: it is skipped, same values.
   auto rows = [&](auto fast) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = qt * 16 + i;
-      const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
-      const float qa = __uint_as_float(qv[i] << 16), qb = __uint_as_float(qv[i] & 0xFFFF0000u);
-      const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
-      e0 *= a0[i];
-      e1 *= a1[i];
-      const uint32_t qgv = pack_bf16x2(qa * e0, qb * e1);
-      *reinterpret_cast<uint32_t *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
-      if (gq) *reinterpret_cast<uint32_t *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
-      *reinterpret_cast<uint32_t *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) =
-          pack_bf16x2(ka * e0, kb2 * e1);
-      float h0, h1;
-      if constexpr (decltype(fast)::value) {
-        float v0, v1;
-        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(v0) : "f"(e0));
-        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(v1) : "f"(e1));
-        h0 = ka * v0;
-        h1 = kb2 * v1;
-      } else {
-        h0 = kh_entry(ka, e0, r, c, xr, mk0);
-        h1 = kh_entry(kb2, e1, r, c + 1, xr, mk1);
+    for (int i = 0; i < 8; ++i) {
+      const int r = qt * 8 + i;
+      const uint32_t sw = (uint32_t)((ch ^ (r & 7)) << 4);
+      float qf[4], kf[4], x[4];
+      unpack(qv[i], qf);
+      unpack(kv[i], kf);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ev[e] *= a[i][e];
+        x[e] = qf[e] * ev[e];
       }
-      *reinterpret_cast<uint32_t *>(t.kh + col64 + (uint32_t)(r * 128) + sw) = pack_bf16x2(h0, h1);
+      const uint2 qgv = pack4(x);
+      *reinterpret_cast<uint2 *>(t.qg + colq + (uint32_t)((t.qg_row0 + r) * 128) + sw) = qgv;
+      if (gq) *reinterpret_cast<uint2 *>(gq + col128 + (uint32_t)((64 + r) * 128) + sw) = qgv;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = kf[e] * ev[e];
+      *reinterpret_cast<uint2 *>(t.kg + colk + (uint32_t)((t.kg_row0 + r) * 128) + sw) = pack4(x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (decltype(fast)::value) {
+          float inv;
+          asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(ev[e]));
+          x[e] = kf[e] * inv;
+        } else {
+          x[e] = kh_entry(kf[e], ev[e], r, c + e, xr, mk[e]);
+        }
+      }
+      *reinterpret_cast<uint2 *>(t.kh + col64 + (uint32_t)(r * 128) + sw) = pack4(x);
     }
   };
-  if (pre0 * t0 > 2.f * kFastMinDecay && pre1 * t1 > 2.f * kFastMinDecay)
+  bool fast = true;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) fast = fast && (pre[e] * tt[e] > 2.f * kFastMinDecay);
+  if (fast)
     rows(BoolTag<true>{});
   else
     rows(BoolTag<false>{});
-  float s0 = suf0, s1 = suf1;
+  float sv[4] = {suf[0], suf[1], suf[2], suf[3]};
 #pragma unroll
-  for (int i = 15; i >= 0; --i) {
-    const int r = qt * 16 + i;
-    const uint32_t sw = (uint32_t)((ch ^ (i & 7)) << 4);
-    const float ka = __uint_as_float(kv[i] << 16), kb2 = __uint_as_float(kv[i] & 0xFFFF0000u);
-    const uint32_t rr = (uint32_t)(r * 128) + sw;
-    *reinterpret_cast<uint32_t *>(gkt + col64 + rr) = pack_bf16x2(ka * s0, kb2 * s1);
-    s0 *= a0[i];
-    s1 *= a1[i];
+  for (int i = 7; i >= 0; --i) {
+    const int r = qt * 8 + i;
+    const uint32_t sw = (uint32_t)((ch ^ (r & 7)) << 4);
+    float kf[4], x[4];
+    unpack(kv[i], kf);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[e] = kf[e] * sv[e];
+      sv[e] *= a[i][e];
+    }
+    *reinterpret_cast<uint2 *>(gkt + col64 + (uint32_t)(r * 128) + sw) = pack4(x);
   }
 }
 

@@ -179,9 +179,9 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
   __shared__ uint32_t unsafe_sh[4];     // channels with exact-path key rows
   __shared__ int tfirst_sh[128];        // their first exact-path key row
   const prep::ExactRows xrows{unsafe_sh, tfirst_sh};
-  __shared__ float decay_sh[kDK];
+  __shared__ __align__(16) float decay_sh[kDK];   // written 16 bytes at a time by the prep
   __shared__ __align__(16) float beta_sh[kC];   // read 16 bytes at a time by pack_tb
-  __shared__ float part_sh[4][kDK];
+  __shared__ __align__(16) float part_sh[8][kDK];   // per row group of the decay prep
 
   if (device_error_latched(p.err)) return;
   const int H = p.H;
