@@ -381,8 +381,9 @@ intra_kernel(PrefillParams p, const __grid_constant__ IntraMaps maps, const SeqS
     ok = wait_all(&v_bar, vphase & 1, p, 2);
     vphase++;
     if (!ok) break;
-    if (tid == 0 && item + (int)gridDim.x < nitems) {
+    if (tid == 32 && item + (int)gridDim.x < nitems) {
       // T is packed and A is consumed: next item's q into the T tile, k into the A region
+      // (from warp 1, so thread 0 goes straight on to the W and U_v products)
       fence_async_smem();
       stage_q(nx.ip.h, nx.ip.c0);
       stage_k(nx.ip.h, nx.ip.c0);
